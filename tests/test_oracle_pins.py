@@ -1,0 +1,254 @@
+"""Pins for the CPU oracle: each test checks it against something other than
+itself (exact rational arithmetic, numpy's IEEE conversions, numpy's fp64
+matmul, integer matmul, hand-worked values, closed forms), chosen so that a
+dropped term, a wrong sign, a wrong group index or a transposed operand fails
+at least one of them.
+"""
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+from gemm_w4a16_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _f16(bits):
+    return np.asarray(bits, dtype=np.uint16).view(np.float16)
+
+
+# ------------------------------------------------------------------ fp16 ----
+
+def test_fp16_decode_every_pattern_matches_numpy():
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    ours = oracle.fp16_to_double(bits)
+    ref = _f16(bits).astype(np.float64)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan], ref[~nan])
+    assert np.array_equal(np.signbit(ours[~nan]), np.signbit(ref[~nan]))
+
+
+def test_fp16_encode_roundtrips_every_pattern():
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    vals = _f16(bits).astype(np.float64)
+    keep = ~np.isnan(vals)
+    assert np.array_equal(oracle.fp16_from_double(vals[keep]), bits[keep])
+
+
+def test_fp16_encode_every_dequant_product_matches_numpy():
+    """All (q - z) in [-15, 15] times every finite fp16 scale, both signs."""
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    s = _f16(bits).astype(np.float64)
+    s = s[np.isfinite(s)]
+    d = np.arange(-15, 16, dtype=np.float64)
+    prod = (d[:, None] * s[None, :]).ravel()
+    ours = oracle.fp16_from_double(prod)
+    with np.errstate(over="ignore"):
+        ref = prod.astype(np.float16).view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+def test_fp16_encode_ties_subnormals_overflow_and_random():
+    rng = np.random.default_rng(1)
+    finite = _f16(np.arange(0x7c00, dtype=np.uint16)).astype(np.float64)
+    mids = (finite[:-1] + finite[1:]) / 2          # exact ties between neighbours
+    near = np.concatenate([mids, np.nextafter(mids, 0), np.nextafter(mids, 1)])
+    rand = np.ldexp(rng.uniform(0.5, 1.0, 200000), rng.integers(-30, 18, 200000))
+    edge = np.array([65504.0, 65519.99, 65520.0, 70000.0, 2.0**-25, 2.0**-26,
+                     3 * 2.0**-26, 2.0**-14 - 2.0**-25, 1e-30, 0.0])
+    x = np.concatenate([near, rand, edge])
+    x = np.concatenate([x, -x])
+    ours = oracle.fp16_from_double(x)
+    with np.errstate(over="ignore"):
+        ref = x.astype(np.float16).view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+def test_dequant_hand_worked_cases():
+    rows = []
+    with open(os.path.join(GOLDEN, "dequant_cases.txt")) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                q, z, s, w = line.split()
+                rows.append((int(q), int(z), int(s, 16), int(w, 16)))
+    assert len(rows) >= 10
+    G = 128
+    M = len(rows)
+    q = np.zeros((M, G), np.uint8)
+    zeros = np.zeros((M, 1), np.uint8)
+    scales = np.zeros((M, 1), np.uint16)
+    for i, (qq, zz, ss, _) in enumerate(rows):
+        q[i, :] = qq
+        zeros[i, 0] = zz
+        scales[i, 0] = ss
+    W = oracle.dequant(q, zeros, scales, G)
+    for i, (_, _, _, w) in enumerate(rows):
+        assert np.all(W[i] == w), (i, hex(W[i, 0]), hex(w))
+
+
+# ------------------------------------------------------------- dequant ----
+
+def test_dequant_group_indexing_against_numpy_definition():
+    """Groups run along K within one row: k // G picks the scale column."""
+    p = synth.make_problem(M=37, K=512, N=1, seed=3)
+    W = oracle.dequant(p.q, p.zeros, p.scales, 128)
+    g = np.arange(512) // 128
+    d = p.q.astype(np.float64) - p.zeros[:, g].astype(np.float64)
+    ref = (d * _f16(p.scales)[:, g].astype(np.float64)).astype(np.float16)
+    assert np.array_equal(W, ref.view(np.uint16))
+
+
+def test_dequant_other_group_sizes():
+    rng = np.random.default_rng(5)
+    for G in (32, 64, 256):
+        q, z, s = synth.draw_weights(rng, 9, 512, G)
+        W = oracle.dequant(q, z, s, G)
+        g = np.arange(512) // G
+        ref = ((q.astype(np.float64) - z[:, g]) * _f16(s)[:, g].astype(np.float64))
+        assert np.array_equal(W, ref.astype(np.float16).view(np.uint16))
+
+
+# ------------------------------------------------------------- product ----
+
+def test_brute_force_exact_rational():
+    """Exact rational sums; the fp64 oracle must sit within the recursive
+    summation bound (K - 1) * 2^-53 * sum |w x| of them."""
+    p = synth.make_problem(M=5, K=256, N=3, seed=11)
+    y = oracle.gemm(p.q, p.zeros, p.scales, p.x, 128)
+    s = _f16(p.scales).astype(np.float64)
+    x = _f16(p.x).astype(np.float64)
+    for m in range(p.M):
+        w = []
+        for k in range(p.K):
+            g = k // 128
+            exact = Fraction(int(p.q[m, k]) - int(p.zeros[m, g])) * Fraction(s[m, g])
+            w.append(Fraction(float(np.float16(float(exact)))))   # one RNE rounding
+        for n in range(p.N):
+            terms = [w[k] * Fraction(x[n, k]) for k in range(p.K)]
+            exact_y = sum(terms, Fraction(0))
+            bound = (p.K - 1) * 2.0**-53 * float(sum(abs(t) for t in terms))
+            assert abs(Fraction(y[n, m]) - exact_y) <= Fraction(bound), (m, n)
+
+
+def test_matches_numpy_fp64_matmul():
+    p = synth.make_problem(M=200, K=384, N=7, seed=2)
+    W = oracle.dequant(p.q, p.zeros, p.scales, 128)
+    ref = _f16(p.x).astype(np.float64) @ _f16(W).astype(np.float64).T
+    y = oracle.gemm(p.q, p.zeros, p.scales, p.x, 128)
+    assert y.shape == (7, 200)
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_hand_worked_gemm():
+    G, K = 128, 128
+    q = np.zeros((2, K), np.uint8)
+    q[0, :] = 9
+    q[1, :] = np.arange(K) % 16
+    zeros = np.array([[8], [0]], np.uint8)
+    scales = np.array([[0x3800], [0x3C00]], np.uint16)      # 0.5, 1.0
+    x = np.empty((2, K), np.float16)
+    x[0, :] = 1
+    x[1, :] = np.where(np.arange(K) % 2 == 0, 1, -1)
+    y = oracle.gemm(q, zeros, scales, x.view(np.uint16), G)
+    with open(os.path.join(GOLDEN, "gemm_closed_form.txt")) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                n, m, v = line.split()
+                assert y[int(n), int(m)] == float(v)
+
+
+def test_q_equal_z_gives_exact_zero():
+    p = synth.make_problem(M=64, K=512, N=4, seed=4)
+    g = np.arange(512) // 128
+    q = np.ascontiguousarray(p.zeros[:, g])
+    y = oracle.gemm(q, p.zeros, p.scales, p.x, 128)
+    assert np.all(y == 0.0)
+
+
+def test_unit_scale_zero_eight_integer_inputs_exact():
+    """s = 1, z = 8, x in {-1, 0, 1}: the result is an integer matmul."""
+    rng = np.random.default_rng(6)
+    M, K, N = 96, 256, 5
+    q = rng.integers(0, 16, (M, K), dtype=np.uint8)
+    zeros = np.full((M, K // 128), 8, np.uint8)
+    scales = np.full((M, K // 128), 0x3C00, np.uint16)
+    xi = rng.integers(-1, 2, (N, K))
+    y = oracle.gemm(q, zeros, scales, xi.astype(np.float16).view(np.uint16), 128)
+    ref = xi.astype(np.int64) @ (q.astype(np.int64) - 8).T
+    assert np.array_equal(y, ref.astype(np.float64))
+
+
+def test_scale_enters_per_group_and_sign():
+    """Flipping z and q around 8 negates every output; doubling one group's
+    scale changes only that group's share."""
+    p = synth.make_problem(M=16, K=256, N=2, seed=8)
+    y = oracle.gemm(p.q, p.zeros, p.scales, p.x, 128)
+    y_neg = oracle.gemm((15 - p.q).astype(np.uint8), (15 - p.zeros).astype(np.uint8),
+                        p.scales, p.x, 128)
+    assert np.array_equal(y_neg, -y)
+    s2 = p.scales.copy()
+    s2[:, 1] = (_f16(p.scales[:, 1]).astype(np.float64) * 2).astype(np.float16).view(np.uint16)
+    y2 = oracle.gemm(p.q, p.zeros, s2, p.x, 128)
+    W = _f16(oracle.dequant(p.q, p.zeros, p.scales, 128)).astype(np.float64)
+    xs = _f16(p.x).astype(np.float64)
+    second = xs[:, 128:] @ W[:, 128:].T
+    np.testing.assert_allclose(y2 - y, second, rtol=1e-12, atol=1e-12)
+
+
+def test_gemv_equals_column_of_gemm():
+    p = synth.make_problem(M=130, K=256, N=9, seed=9)
+    y = oracle.gemm(p.q, p.zeros, p.scales, p.x, 128)
+    for j in range(p.N):
+        yj = oracle.gemm(p.q, p.zeros, p.scales, p.x[j:j + 1], 128)
+        assert np.array_equal(yj[0], y[j])
+
+
+def test_rows_subset_matches_full():
+    p = synth.make_problem(M=300, K=256, N=3, seed=10)
+    y = oracle.gemm(p.q, p.zeros, p.scales, p.x, 128)
+    rows = np.array([0, 7, 299, 150, 7])
+    ys = oracle.gemm_rows(p.q, p.zeros, p.scales, p.x, rows, 128)
+    assert np.array_equal(ys, y[:, rows])
+
+
+def test_thread_count_does_not_change_result():
+    p = synth.make_problem(M=257, K=512, N=3, seed=12)
+    old = oracle.get_threads()
+    try:
+        oracle.set_threads(1)
+        y1 = oracle.gemm(p.q, p.zeros, p.scales, p.x, 128)
+        oracle.set_threads(max(2, os.cpu_count() or 2))
+        y2 = oracle.gemm(p.q, p.zeros, p.scales, p.x, 128)
+    finally:
+        oracle.set_threads(old)
+    assert np.array_equal(y1, y2)
+
+
+def test_rejects_bad_shapes():
+    p = synth.make_problem(M=4, K=256, N=1, seed=0)
+    with pytest.raises(ValueError):
+        oracle.gemm(p.q[:, :200], p.zeros, p.scales, p.x[:, :200], 128)
+    with pytest.raises(ValueError):
+        oracle.gemm(p.q, p.zeros, p.scales, p.x[:, :128], 128)
+
+
+# --------------------------------------------------------- synth inputs ----
+
+def test_synthetic_distributions():
+    p = synth.make_problem(M=512, K=4096, N=4, seed=0, outlier_frac=0.01)
+    assert p.q.min() == 0 and p.q.max() == 15
+    assert p.zeros.min() == 0 and p.zeros.max() == 15
+    s = _f16(p.scales).astype(np.float64)
+    assert s.min() >= 0.001 - 1e-6 and s.max() <= 0.02 + 1e-5
+    assert len(p.outliers) == 41 and len(set(p.outliers.tolist())) == 41
+    x = np.abs(_f16(p.x).astype(np.float64))
+    others = np.setdiff1d(np.arange(4096), p.outliers)
+    assert x[:, p.outliers].mean() > 10 * x[:, others].mean()
+    again = synth.make_problem(M=512, K=4096, N=4, seed=0, outlier_frac=0.01)
+    assert np.array_equal(again.q, p.q) and np.array_equal(again.x, p.x)
