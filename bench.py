@@ -1,0 +1,581 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 W4A16 group-128 linear layer.
+
+Default workload (one "step"): a LLaMA-7B-shaped decode step at N = 1 token --
+32 layers x {fused QKV 12288x4096, O 4096x4096, fused gate/up 22016x4096,
+down 4096x11008}, 128 distinct packed weight sets resident in HBM (3.37 GB, far
+beyond the 126 MB L2, so no flush is needed), each projection one w4a16_gemm
+call, the step captured once in a CUDA graph.  The metric is algorithmic HBM
+bytes per second (packed int4 weights + 2.5 B per group of metadata + fp16 X
+and Y), reported against the measured HBM copy bandwidth.
+
+One JSON line on stdout (rank 0).  Multi-GPU runs (torchrun) are replicas:
+every rank runs its own copy of the step (weak scaling), no collective on the
+data path; time is the max over ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+    python bench.py --workload qkv_n1|prefill|sweep ...   (secondary workloads)
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "W4A16 g128 GEMV HBM GB/s & GEMM TFLOPS on 1 B200, % of roofline"
+GROUP = 128
+LLAMA7B_LAYER = [("qkv", 12288, 4096), ("o", 4096, 4096), ("gate_up", 22016, 4096),
+                 ("down", 4096, 11008)]
+N_LAYERS = 32
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def alg_bytes(M, K, N):
+    """Algorithmic bytes of one call: int4 weights, 2.5 B/group metadata, X, Y."""
+    return M * K // 2 + (M * K // GROUP) * 5 // 2 + 2 * K * N + 2 * M * N
+
+
+def alg_flops(M, K, N):
+    return 2 * M * N * K
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------ distributed --
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def dist_init(backend):
+    import datetime
+
+    import torch.distributed as dist
+
+    if not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(value: float, dist=None, device=None) -> float:
+    """Max of a float over all ranks (identity without a process group)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return value
+    import torch
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, dist=None, device=None) -> float:
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return value
+    import torch
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+
+    def summary(self, t0=None, t1=None):
+        rows = []
+        for ts, line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((ts, float(parts[0]), float(parts[1]), parts[3:]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        inside = [r for r in rows if t0 is None or (t0 <= r[0] <= t1)] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in inside:
+            for name, v in zip(names, r[3][1:]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r[1] for r in inside),
+                "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": sorted(reasons), "samples": len(inside)}
+
+
+# ---------------------------------------------------------- decode step ----
+
+def build_decode_step(device, seed=0, n_layers=N_LAYERS):
+    """128 distinct packed weight sets plus per-call X and Y (flat buffers)."""
+    import torch
+
+    from gemm_w4a16_b200 import synth, w4a16
+
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    calls = []
+    x_total = sum(K for _, _, K in LLAMA7B_LAYER) * n_layers
+    y_total = sum(M for _, M, _ in LLAMA7B_LAYER) * n_layers
+    x_flat = torch.empty(x_total, dtype=torch.float16, device=device)
+    y_flat = torch.empty(y_total, dtype=torch.float16, device=device)
+    xo = yo = 0
+    for layer in range(n_layers):
+        for name, M, K in LLAMA7B_LAYER:
+            q, z, s = synth.make_weights_torch(M, K, GROUP, gen, device)
+            w = w4a16.pack(q, s, z)
+            del q, z, s
+            x = x_flat[xo:xo + K].view(1, K)
+            x.copy_(synth.make_activations_torch(1, K, gen, device))
+            y = y_flat[yo:yo + M].view(1, M)
+            xo += K
+            yo += M
+            calls.append((name, w, x, y))
+    torch.cuda.synchronize(device)
+    return calls, x_flat, y_flat
+
+
+def run_calls(calls, path=0):
+    from gemm_w4a16_b200 import w4a16
+
+    for _, w, x, y in calls:
+        if path:
+            w4a16.gemm_ex(w, x, Y=y, path=path)
+        else:
+            w4a16.gemm(w, x, Y=y)
+
+
+def capture(fn, device):
+    import torch
+
+    s = torch.cuda.Stream(device=device)
+    s.wait_stream(torch.cuda.current_stream(device))
+    with torch.cuda.stream(s):
+        fn()            # warm the launch path once outside capture
+    torch.cuda.current_stream(device).wait_stream(s)
+    torch.cuda.synchronize(device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize(device)
+    return g
+
+
+def time_graph(g, steps, warmup, device, pre=None, post=None):
+    """ms per step of graph replays, CUDA events on the replay stream."""
+    import torch
+
+    stream = torch.cuda.current_stream(device)
+    for _ in range(warmup):
+        if pre:
+            pre()
+        g.replay()
+        if post:
+            post()
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        if pre:
+            pre()
+        g.replay()
+        if post:
+            post()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    return e0.elapsed_time(e1) / steps
+
+
+# ------------------------------------------------------- CPU (oracle) leg --
+
+def _oracle_layer(rows=None, seed=0):
+    """Canonical host arrays of one synthetic layer (optionally its first rows)."""
+    import numpy as np
+
+    from gemm_w4a16_b200 import synth
+
+    rng = np.random.default_rng(seed)
+    layer = []
+    for name, M, K in LLAMA7B_LAYER:
+        m = M if rows is None else min(rows, M)
+        q, z, s = synth.draw_weights(rng, m, K, GROUP)
+        x, _ = synth.draw_activations(rng, 1, K)
+        layer.append((m, K, q, z, s, x))
+    return layer
+
+
+def _oracle_pass(layer):
+    import oracle
+
+    nbytes = 0
+    for M, K, q, z, s, x in layer:
+        oracle.gemm(q, z, s, x, GROUP)
+        nbytes += alg_bytes(M, K, 1)
+    return nbytes
+
+
+def oracle_decode_sample(target_s=12.0, max_layers=N_LAYERS, seed=0):
+    """Time the CPU oracle, as it stands, over whole synthetic layers of the
+    decode step until about target_s seconds of work; returns GB/s."""
+    import oracle
+
+    layer = _oracle_layer(seed=seed)
+    nbytes = 0
+    layers = 0
+    t0 = time.perf_counter()
+    while layers < max_layers:
+        nbytes += _oracle_pass(layer)
+        layers += 1
+        if time.perf_counter() - t0 >= target_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": oracle.get_threads(),
+            "kind": "oracle",
+            "sample": f"{layers} full layer(s) of the 4 LLaMA-7B projections at N=1 "
+                      f"({layers * 4} oracle products, {nbytes / 1e6:.0f} MB algorithmic, "
+                      f"{dt:.1f} s)"}
+
+
+REF_ROWS = 128   # rows of each projection per reference-arm step
+
+
+def main_reference(args):
+    """The reference arm: the CPU oracle, as it stands, on the host cores.
+    One step = the first REF_ROWS output rows of each of the four projections
+    of one layer at N = 1 (a bounded sample of the decode step)."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+
+    oracle.set_threads(os.cpu_count() or 1)
+    layer = _oracle_layer(rows=REF_ROWS)
+    for _ in range(args.warmup):
+        _oracle_pass(layer)
+    t0 = time.perf_counter()
+    nbytes = 0
+    for _ in range(args.steps):
+        nbytes += _oracle_pass(layer)
+    dt = time.perf_counter() - t0
+    value = nbytes / dt / 1e9
+    sample = (f"per step: first {REF_ROWS} rows of each of the 4 LLaMA-7B projections "
+              f"at N=1 ({nbytes // max(args.steps, 1)} algorithmic bytes)")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3 / max(args.steps, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "llama7b_decode_step_n1", "group": GROUP,
+                       "step": sample},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle.get_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------- our path ----
+
+def main_ours(args):
+    import torch
+
+    from gemm_w4a16_b200 import build as lib_build
+    from gemm_w4a16_b200 import w4a16
+
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device"}), flush=True)
+        return 1
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist = dist_init("nccl") if world > 1 else None
+    if rank == 0:
+        lib_build.build()
+    if dist is not None:
+        dist.barrier()
+    w4a16.lib()
+    peaks, peaks_src = load_peaks()
+
+    if args.workload == "sweep":
+        return sweep(args, device)
+    if args.workload == "qkv_n1":
+        return single_shape(args, device, 12288, 4096, 1)
+    if args.workload == "prefill":
+        return single_shape(args, device, 12288, 4096, 4096)
+
+    calls, x_flat, y_flat = build_decode_step(device, seed=1000 + rank)
+    step_bytes = sum(alg_bytes(w.M, w.K, 1) for _, w, _, _ in calls)
+    launches_per_step = len(calls)      # one kernel launch per projection at N = 1
+    g = capture(lambda: run_calls(calls), device)
+
+    # Device-resident timing (the headline value).
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    t_wall0 = time.time()
+    ms = time_graph(g, args.steps, args.warmup, device)
+    t_wall1 = time.time()
+    time.sleep(0.2)
+    sampler.stop()
+    ms_max = max_over_ranks(ms, dist, device)
+    total_bytes = sum_over_ranks(step_bytes * args.steps, dist, device)
+    value = total_bytes / (ms_max * args.steps * 1e-3) / 1e9
+
+    # Per-shape achieved bandwidth: each projection type alone, 32 distinct
+    # weight sets per graph so every launch reads its weights from HBM.
+    per_shape = {}
+    for name, M, K in LLAMA7B_LAYER:
+        sub = [c for c in calls if c[0] == name]
+        gs = capture(lambda sub=sub: run_calls(sub), device)
+        ms_s = time_graph(gs, max(10, args.steps // 4), 3, device) / len(sub)
+        b = alg_bytes(M, K, 1)
+        per_shape[name] = {"M": M, "K": K, "N": 1, "us": ms_s * 1e3,
+                           "GBps": b / (ms_s * 1e-3) / 1e9,
+                           "frac_hbm": b / (ms_s * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+        del gs
+
+    # End to end: H2D of every call's X from pinned host memory, the graph,
+    # D2H of every Y, all on the stream, inside the event-timed region.
+    x_host = torch.empty(x_flat.shape, dtype=x_flat.dtype, pin_memory=True)
+    y_host = torch.empty(y_flat.shape, dtype=y_flat.dtype, pin_memory=True)
+    x_host.copy_(x_flat)
+    e2e_steps = max(args.steps // 2, 1)
+    ms_e2e = time_graph(g, e2e_steps, args.warmup, device,
+                        pre=lambda: x_flat.copy_(x_host, non_blocking=True),
+                        post=lambda: y_host.copy_(y_flat, non_blocking=True))
+    ms_e2e_max = max_over_ranks(ms_e2e, dist, device)
+    e2e_value = sum_over_ranks(step_bytes, dist, device) / (ms_e2e_max * 1e-3) / 1e9
+
+    prefill = None
+    if w4a16.select_path(12288, 4096, 4096) == w4a16.PATH_TC and not args.no_prefill:
+        prefill = prefill_measure(device, peaks, args)
+
+    res = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        res = oracle_decode_sample(target_s=args.cpu_seconds)
+
+    if dist is not None:
+        del g
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    clocks = sampler.summary(t_wall0, t_wall1)
+    achieved = step_bytes / (ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16", "accumulate": "f32", "data": "synthetic",
+        "config": {"workload": "llama7b_decode_step_n1",
+                   "description": "32 layers x {qkv 12288x4096, o 4096x4096, gate_up 22016x4096, "
+                                  "down 4096x11008}, N=1, group 128, 128 distinct weight sets",
+                   "bytes_per_step": step_bytes, "global_batch": 1, "seq_len": 1,
+                   "l2": "inputs 3.37 GB per step > 126 MB L2 (no flush needed)",
+                   "launch": "cuda_graph", "parallelism": f"replicas{world}"},
+        "roofline": {"bound": "hbm", "kernel": "gemv_kernel<1>", "achieved": achieved,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks_src,
+                     "traffic": args.traffic},
+        "per_shape": per_shape,
+        "e2e": {"value": e2e_value, "unit": "GB/s",
+                "h2d_bytes_per_step": int(x_flat.numel() * 2),
+                "d2h_bytes_per_step": int(y_flat.numel() * 2), "ms_per_step": ms_e2e_max,
+                "api": "w4a16_gemm (128 calls captured in a CUDA graph) + pinned H2D/D2H"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if prefill:
+        line["prefill"] = prefill
+    if res:
+        line["cpu_baseline"] = res
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def make_device_problem(device, M, K, N, seed, outlier_frac=0.0):
+    import numpy as np
+    import torch
+
+    from gemm_w4a16_b200 import synth, w4a16
+
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    q, z, s = synth.make_weights_torch(M, K, GROUP, gen, device)
+    w = w4a16.pack(q, s, z)
+    x = synth.make_activations_torch(N, K, gen, device)
+    if outlier_frac:
+        rng = np.random.default_rng(seed)
+        idx = torch.from_numpy(rng.choice(K, int(round(outlier_frac * K)), replace=False)).to(device)
+        x[:, idx] = (x[:, idx].float() * 20).half()
+    return w, x
+
+
+def prefill_measure(device, peaks, args):
+    import torch
+
+    from gemm_w4a16_b200 import w4a16
+
+    out = {}
+    for name, M, K, N in (("qkv_n4096", 12288, 4096, 4096), ("down_n2048", 4096, 11008, 2048)):
+        w, x = make_device_problem(device, M, K, N, seed=7, outlier_frac=0.01)
+        y = torch.empty((N, M), dtype=torch.float16, device=device)
+        g = capture(lambda: w4a16.gemm(w, x, Y=y), device)
+        ms = time_graph(g, 20, 5, device)
+        tf = alg_flops(M, K, N) / (ms * 1e-3) / 1e12
+        out[name] = {"M": M, "K": K, "N": N, "us": ms * 1e3, "TFLOPS": tf,
+                     "frac_tensor": tf / peaks["bf16_tflops"],
+                     "peak": peaks["bf16_tflops"], "peak_kind": "bf16 burst (fp16 same rate)"}
+        del g, w, x, y
+    return out
+
+
+def single_shape(args, device, M, K, N):
+    """One shape, plain launches (used for ncu captures and quick timing)."""
+    import torch
+
+    from gemm_w4a16_b200 import w4a16
+
+    peaks, _ = load_peaks()
+    w, x = make_device_problem(device, M, K, N, seed=3)
+    y = torch.empty((N, M), dtype=torch.float16, device=device)
+    for _ in range(args.warmup):
+        w4a16.gemm(w, x, Y=y)
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        w4a16.gemm(w, x, Y=y)
+    e1.record()
+    torch.cuda.synchronize(device)
+    ms = e0.elapsed_time(e1) / args.steps
+    b, f = alg_bytes(M, K, N), alg_flops(M, K, N)
+    print(json.dumps({"workload": f"M={M} K={K} N={N}", "us": ms * 1e3,
+                      "GBps": b / (ms * 1e-3) / 1e9, "TFLOPS": f / (ms * 1e-3) / 1e12,
+                      "path": w4a16.select_path(M, K, N),
+                      "note": "plain launches; weights may sit in L2 across iterations"}))
+    return 0
+
+
+def sweep(args, device):
+    """N sweep on the fused QKV shape, both kernels, 16 weight copies rotated
+    (16 x 26 MB > L2) so that weights come from HBM."""
+    import torch
+
+    from gemm_w4a16_b200 import w4a16
+
+    peaks, _ = load_peaks()
+    M, K = 12288, 4096
+    copies = [make_device_problem(device, M, K, 1, seed=100 + i)[0] for i in range(16)]
+    for N in (1, 2, 4, 8, 16, 32, 64, 128, 256, 512, 1024, 2048, 4096):
+        from gemm_w4a16_b200 import synth
+        gen = torch.Generator(device=device)
+        gen.manual_seed(N)
+        x = synth.make_activations_torch(N, K, gen, device)
+        y = torch.empty((N, M), dtype=torch.float16, device=device)
+        for path in (w4a16.PATH_GEMV, w4a16.PATH_TC):
+            if path == w4a16.PATH_GEMV and N > 256:
+                continue
+            try:
+                g = capture(lambda path=path: [w4a16.gemm_ex(w, x, Y=y, path=path) for w in copies],
+                            device)
+            except w4a16.W4A16Error as e:
+                print(json.dumps({"N": N, "path": path, "error": str(e)}), flush=True)
+                continue
+            ms = time_graph(g, 5, 2, device) / len(copies)
+            b, f = alg_bytes(M, K, N), alg_flops(M, K, N)
+            gbs, tfs = b / (ms * 1e-3) / 1e9, f / (ms * 1e-3) / 1e12
+            print(json.dumps({"N": N, "path": "gemv" if path == 1 else "tc", "us": ms * 1e3,
+                              "GBps": gbs, "TFLOPS": tfs,
+                              "roof_frac": max(gbs / peaks["hbm_gbs"], tfs / peaks["bf16_tflops"]),
+                              "auto": w4a16.select_path(M, K, N)}), flush=True)
+            del g
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["decode", "qkv_n1", "prefill", "sweep"], default="decode")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="ncu DRAM bytes per launch of the dominant kernel, if captured")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return main_reference(args)
+    return main_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

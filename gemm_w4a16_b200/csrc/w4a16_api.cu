@@ -1,0 +1,139 @@
+// C-ABI entry points of libw4a16: host-side argument checks, the N-based
+// dispatcher between the CUDA-core GEMV and the tcgen05 GEMM, and status
+// mapping.  "PerfXLLM on Snapdragon 8 Gen2", section 3.3: prefill (tokens > 1)
+// is a GEMM and decode (tokens = 1) a GEMV; few tokens make the GEMM
+// memory-bound and many make it compute-bound, and each regime gets its own
+// tiling.  Here each regime gets its own kernel.
+#include "w4a16_internal.cuh"
+
+namespace w4a16 {
+// Largest N the dispatcher sends to the CUDA-core GEMV kernel; above it the
+// tensor-core kernel runs.  Chosen from the measured N sweep on the fused QKV
+// shape (M = 12288, K = 4096).
+int gemv_max_n();
+}
+
+namespace {
+
+using namespace w4a16;
+
+constexpr int kMaxM = 1 << 24;
+constexpr int kMaxK = 1 << 20;
+constexpr int kMaxN = 1 << 20;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+w4a16_status check_shape(int M, int K, int group) {
+  if (M <= 0 || K <= 0) return W4A16_ERR_INVALID_ARG;
+  if (group != kGroup || K % kGroup != 0) return W4A16_ERR_UNSUPPORTED;
+  if (M > kMaxM || K > kMaxK) return W4A16_ERR_UNSUPPORTED;
+  return W4A16_OK;
+}
+
+w4a16_status map_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return W4A16_OK;
+  if (e == cudaErrorNotSupported) return W4A16_ERR_UNSUPPORTED;
+  return W4A16_ERR_CUDA;
+}
+
+int select_path_impl(int M, int K, int N) {
+  if (M <= 0 || K <= 0 || N <= 0 || K % kGroup) return -1;
+  return N <= gemv_max_n() ? W4A16_PATH_GEMV : W4A16_PATH_TC;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* w4a16_status_string(int status) {
+  switch (status) {
+    case W4A16_OK: return "ok";
+    case W4A16_ERR_INVALID_ARG: return "invalid argument";
+    case W4A16_ERR_UNSUPPORTED: return "unsupported size or group";
+    case W4A16_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case W4A16_ERR_CUDA: return "CUDA error";
+    case W4A16_ERR_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+w4a16_status w4a16_packed_sizes(int M, int K, int group, size_t* wq_bytes,
+                                size_t* scales_bytes, size_t* zeros_bytes) {
+  if (!wq_bytes || !scales_bytes || !zeros_bytes) return W4A16_ERR_INVALID_ARG;
+  w4a16_status st = check_shape(M, K, group);
+  if (st != W4A16_OK) return st;
+  const size_t mp = (size_t)ceil_div(M, kRowBlock) * kRowBlock;
+  const size_t kg = (size_t)K / kGroup;
+  *wq_bytes = mp * (size_t)K / 2;
+  *scales_bytes = mp * kg * 2;
+  *zeros_bytes = mp * kg / 2;
+  return W4A16_OK;
+}
+
+w4a16_status w4a16_pack(const uint8_t* q, const uint16_t* scales, const uint8_t* zeros,
+                        int M, int K, int group, void* wq_packed, void* scales_packed,
+                        void* zeros_packed, void* stream) {
+  if (!q || !scales || !zeros || !wq_packed || !scales_packed || !zeros_packed)
+    return W4A16_ERR_INVALID_ARG;
+  w4a16_status st = check_shape(M, K, group);
+  if (st != W4A16_OK) return st;
+  if (!aligned16(wq_packed) || !aligned16(scales_packed) || !aligned16(zeros_packed) ||
+      (reinterpret_cast<uintptr_t>(scales) & 1u))
+    return W4A16_ERR_MISALIGNED;
+  return map_cuda(launch_pack(q, scales, zeros, M, K, static_cast<uint8_t*>(wq_packed),
+                              static_cast<uint16_t*>(scales_packed),
+                              static_cast<uint8_t*>(zeros_packed),
+                              static_cast<cudaStream_t>(stream)));
+}
+
+int w4a16_select_path(int M, int K, int N) { return select_path_impl(M, K, N); }
+
+w4a16_status w4a16_gemm_ex(const void* wq_packed, const void* scales_packed,
+                           const void* zeros_packed, const uint16_t* X, uint16_t* Y,
+                           int M, int K, int N, int group, int path, void* stream) {
+  if (!wq_packed || !scales_packed || !zeros_packed || !X || !Y) return W4A16_ERR_INVALID_ARG;
+  if (N <= 0 || path < W4A16_PATH_AUTO || path > W4A16_PATH_TC) return W4A16_ERR_INVALID_ARG;
+  w4a16_status st = check_shape(M, K, group);
+  if (st != W4A16_OK) return st;
+  if (N > kMaxN) return W4A16_ERR_UNSUPPORTED;
+  if (!aligned16(wq_packed) || !aligned16(scales_packed) || !aligned16(zeros_packed) ||
+      !aligned16(X) || !aligned16(Y))
+    return W4A16_ERR_MISALIGNED;
+  if (path == W4A16_PATH_AUTO) path = select_path_impl(M, K, N);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint8_t* wq = static_cast<const uint8_t*>(wq_packed);
+  const uint16_t* sp = static_cast<const uint16_t*>(scales_packed);
+  const uint8_t* zp = static_cast<const uint8_t*>(zeros_packed);
+  cudaError_t e = (path == W4A16_PATH_TC) ? launch_gemm_tc(wq, sp, zp, X, Y, M, K, N, s)
+                                          : launch_gemv(wq, sp, zp, X, Y, M, K, N, s);
+  return map_cuda(e);
+}
+
+w4a16_status w4a16_gemm(const void* wq_packed, const void* scales_packed,
+                        const void* zeros_packed, const uint16_t* X, uint16_t* Y,
+                        int M, int K, int N, int group, void* stream) {
+  return w4a16_gemm_ex(wq_packed, scales_packed, zeros_packed, X, Y, M, K, N, group,
+                       W4A16_PATH_AUTO, stream);
+}
+
+w4a16_status w4a16_dequant_debug(const void* wq_packed, const void* scales_packed,
+                                 const void* zeros_packed, uint16_t* W_out,
+                                 int M, int K, int group, void* stream) {
+  if (!wq_packed || !scales_packed || !zeros_packed || !W_out) return W4A16_ERR_INVALID_ARG;
+  w4a16_status st = check_shape(M, K, group);
+  if (st != W4A16_OK) return st;
+  if (!aligned16(wq_packed) || !aligned16(scales_packed) || !aligned16(zeros_packed) ||
+      !aligned16(W_out))
+    return W4A16_ERR_MISALIGNED;
+  return map_cuda(launch_dequant(static_cast<const uint8_t*>(wq_packed),
+                                 static_cast<const uint16_t*>(scales_packed),
+                                 static_cast<const uint8_t*>(zeros_packed), W_out, M, K,
+                                 static_cast<cudaStream_t>(stream)));
+}
+
+w4a16_status w4a16_device_status(void* stream, int* status) {
+  if (!status) return W4A16_ERR_INVALID_ARG;
+  return map_cuda(read_and_clear_device_status(static_cast<cudaStream_t>(stream), status));
+}
+
+}  // extern "C"

@@ -1,0 +1,134 @@
+// Shared device helpers and internal launch declarations of libw4a16.
+//
+// Packed weight layout (see include/w4a16.h): 128-row blocks, 32-code chunks of
+// 16 bytes, row-minor inside a chunk column, so one 16-byte load per thread of
+// a warp reads 32 consecutive rows' chunks as 512 contiguous bytes.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "../../include/w4a16.h"
+
+namespace w4a16 {
+
+constexpr int kGroup = 128;      // quantisation group along K
+constexpr int kRowBlock = 128;   // rows per packed block
+constexpr int kChunkK = 32;      // codes per 16-byte chunk
+
+__host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// ---------------------------------------------------------------- loads ----
+
+// 16-byte streaming load through the non-coherent path, no L1 allocation:
+// every weight byte is read exactly once per call.
+__device__ __forceinline__ uint4 ldg_stream_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+
+// 16-byte read-only load that may stay in L1 (activations, shared by a warp).
+__device__ __forceinline__ uint4 ldg_ro_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t orv) {
+  uint32_t d;
+  // (a & b) | c  ->  immLut = (0xF0 & 0xCC) | 0xAA = 0xEA
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(mask), "r"(orv));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t h2_sub(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t h2_mul(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t h2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// Per-(row, group) constants of the in-register dequantisation.
+struct GroupConsts {
+  uint32_t z1024;   // half2(1024 + z, 1024 + z)
+  uint32_t zneg64;  // half2(-(64 + z), -(64 + z))
+  uint32_t s2;      // half2(s, s)
+};
+
+__device__ __forceinline__ GroupConsts make_group_consts(uint32_t z, uint16_t s) {
+  GroupConsts c;
+  uint32_t a = 0x6400u | z;          // fp16 1024 + z (ulp 1 in [1024, 2048))
+  uint32_t b = 0xD400u | (z << 4);   // fp16 -(64 + z) (ulp 1/16 in [64, 128))
+  c.z1024 = a | (a << 16);
+  c.zneg64 = b | (b << 16);
+  c.s2 = (uint32_t)s | ((uint32_t)s << 16);
+  return c;
+}
+
+// Dequantise the 8 codes of one packed 32-bit word into 4 half2 values
+// (k offsets (0,1), (2,3), (4,5), (6,7)), each exactly fp16_RN((q - z) * s):
+//  * OR-ing a code into the mantissa of fp16 1024 gives 1024 + q exactly;
+//    a code left in bits 4..7 gives 1024 + 16 q exactly;
+//  * subtracting 1024 + z, or fma by 1/16 then adding -(64 + z), gives the
+//    exact small integer q - z (every intermediate is representable);
+//  * one fp16 multiply by s then rounds the exact product once, to nearest
+//    even, which is the definition.
+__device__ __forceinline__ void dequant_word(uint32_t w, const GroupConsts& c, uint32_t out[4]) {
+  const uint32_t kMagic = 0x64006400u;
+  const uint32_t kSixteenth = 0x2C002C00u;  // half2(1/16, 1/16)
+  uint32_t w8 = w >> 8;
+  uint32_t e0 = lop3_and_or(w, 0x000F000Fu, kMagic);
+  uint32_t e1 = lop3_and_or(w, 0x00F000F0u, kMagic);
+  uint32_t e2 = lop3_and_or(w8, 0x000F000Fu, kMagic);
+  uint32_t e3 = lop3_and_or(w8, 0x00F000F0u, kMagic);
+  out[0] = h2_mul(h2_sub(e0, c.z1024), c.s2);
+  out[1] = h2_mul(h2_fma(e1, kSixteenth, c.zneg64), c.s2);
+  out[2] = h2_mul(h2_sub(e2, c.z1024), c.s2);
+  out[3] = h2_mul(h2_fma(e3, kSixteenth, c.zneg64), c.s2);
+}
+
+// Zero code of row r (0..127) in the 64-byte zero block of one (block, group).
+__device__ __forceinline__ uint32_t zero_code(const uint8_t* zblock, int r) {
+  return (zblock[r >> 1] >> ((r & 1) * 4)) & 0xFu;
+}
+
+// ------------------------------------------------------- launch helpers ----
+
+// GEMV (CUDA cores): N in 1..kGemvMaxTokens per launch.
+constexpr int kGemvMaxTokens = 4;
+
+cudaError_t launch_gemv(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros,
+                        const uint16_t* X, uint16_t* Y, int M, int K, int N,
+                        cudaStream_t stream);
+
+cudaError_t launch_pack(const uint8_t* q, const uint16_t* scales, const uint8_t* zeros,
+                        int M, int K, uint8_t* wq_p, uint16_t* s_p, uint8_t* z_p,
+                        cudaStream_t stream);
+
+cudaError_t launch_dequant(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros,
+                           uint16_t* W, int M, int K, cudaStream_t stream);
+
+// Tensor-core path.  Returns cudaErrorNotSupported when the sizes are outside
+// what the kernel handles.
+cudaError_t launch_gemm_tc(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros,
+                           const uint16_t* X, uint16_t* Y, int M, int K, int N,
+                           cudaStream_t stream);
+
+cudaError_t read_and_clear_device_status(cudaStream_t stream, int* status);
+
+}  // namespace w4a16

@@ -1,0 +1,189 @@
+"""ctypes binding of libw4a16 (include/w4a16.h), same entry-point names.
+
+Argument marshalling only: every step of the layer runs in the CUDA library.
+PyTorch supplies device memory and the current stream.  If the library is
+missing the calls raise; there is no fallback of any kind.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from dataclasses import dataclass
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libw4a16.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_CUDA, ERR_TIMEOUT = range(6)
+PATH_AUTO, PATH_GEMV, PATH_TC = 0, 1, 2
+GROUP = 128
+
+EXPORTED = (
+    "w4a16_status_string", "w4a16_packed_sizes", "w4a16_pack", "w4a16_gemm",
+    "w4a16_gemm_ex", "w4a16_select_path", "w4a16_dequant_debug",
+    "w4a16_device_status",
+)
+
+_lib = None
+_lock = threading.Lock()
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_szp = ctypes.POINTER(ctypes.c_size_t)
+
+
+class W4A16Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+def lib():
+    """Load libw4a16.so; raise if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with gemm_w4a16_b200/build.py "
+                    "(there is no fallback implementation)")
+            L = ctypes.CDLL(LIB_PATH)
+            L.w4a16_status_string.argtypes = [_i]
+            L.w4a16_status_string.restype = ctypes.c_char_p
+            L.w4a16_packed_sizes.argtypes = [_i, _i, _i, _szp, _szp, _szp]
+            L.w4a16_packed_sizes.restype = _i
+            L.w4a16_pack.argtypes = [_vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp]
+            L.w4a16_pack.restype = _i
+            L.w4a16_gemm.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]
+            L.w4a16_gemm.restype = _i
+            L.w4a16_gemm_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
+            L.w4a16_gemm_ex.restype = _i
+            L.w4a16_select_path.argtypes = [_i, _i, _i]
+            L.w4a16_select_path.restype = _i
+            L.w4a16_dequant_debug.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _vp]
+            L.w4a16_dequant_debug.restype = _i
+            L.w4a16_device_status.argtypes = [_vp, ctypes.POINTER(_i)]
+            L.w4a16_device_status.restype = _i
+            _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().w4a16_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != OK:
+        raise W4A16Error(status, where)
+
+
+def _stream_ptr(stream):
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return _vp(stream.cuda_stream)
+
+
+def _ptr(t):
+    return _vp(t.data_ptr()) if t is not None else _vp(0)
+
+
+def packed_sizes(M: int, K: int, group: int = GROUP):
+    """(wq_bytes, scales_bytes, zeros_bytes) of the packed layout."""
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().w4a16_packed_sizes(M, K, group, ctypes.byref(a), ctypes.byref(b),
+                                    ctypes.byref(c)), "w4a16_packed_sizes")
+    return a.value, b.value, c.value
+
+
+def select_path(M: int, K: int, N: int) -> int:
+    return int(lib().w4a16_select_path(M, K, N))
+
+
+@dataclass
+class PackedWeight:
+    """The three packed device buffers of one M x K weight."""
+
+    wq: "object"       # torch.uint8 [wq_bytes]
+    scales: "object"   # torch.uint8 [scales_bytes] (fp16 values)
+    zeros: "object"    # torch.uint8 [zeros_bytes]
+    M: int
+    K: int
+    group: int = GROUP
+
+    @property
+    def nbytes(self) -> int:
+        return self.wq.numel() + self.scales.numel() + self.zeros.numel()
+
+
+def empty_packed(M: int, K: int, device, group: int = GROUP) -> PackedWeight:
+    import torch
+
+    a, b, c = packed_sizes(M, K, group)
+    mk = lambda n: torch.empty(n, dtype=torch.uint8, device=device)
+    return PackedWeight(mk(a), mk(b), mk(c), M, K, group)
+
+
+def pack(q, scales, zeros, group: int = GROUP, out: PackedWeight | None = None,
+         stream=None) -> PackedWeight:
+    """Canonical device tensors (q uint8 [M,K], scales fp16 [M,K/G], zeros
+    uint8 [M,K/G]) -> packed buffers, via w4a16_pack."""
+    M, K = q.shape
+    for t in (q, scales, zeros):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("pack expects contiguous CUDA tensors")
+    if out is None:
+        out = empty_packed(M, K, q.device, group)
+    _check(lib().w4a16_pack(_ptr(q), _ptr(scales), _ptr(zeros), M, K, group,
+                            _ptr(out.wq), _ptr(out.scales), _ptr(out.zeros),
+                            _stream_ptr(stream)), "w4a16_pack")
+    return out
+
+
+def gemm_ex(w: PackedWeight, X, Y=None, path: int = PATH_AUTO, stream=None):
+    """Y [N, M] fp16 = X [N, K] fp16 . dequant(W)^T via w4a16_gemm_ex."""
+    import torch
+
+    N, K = X.shape
+    if K != w.K or X.dtype != torch.float16 or not X.is_cuda or not X.is_contiguous():
+        raise ValueError("X must be a contiguous CUDA fp16 [N, K] tensor")
+    if Y is None:
+        Y = torch.empty((N, w.M), dtype=torch.float16, device=X.device)
+    _check(lib().w4a16_gemm_ex(_ptr(w.wq), _ptr(w.scales), _ptr(w.zeros), _ptr(X),
+                               _ptr(Y), w.M, K, N, w.group, path, _stream_ptr(stream)),
+           "w4a16_gemm_ex")
+    return Y
+
+
+def gemm(w: PackedWeight, X, Y=None, stream=None):
+    """Y [N, M] fp16 = X [N, K] fp16 . dequant(W)^T via w4a16_gemm."""
+    import torch
+
+    N, K = X.shape
+    if K != w.K or X.dtype != torch.float16 or not X.is_cuda or not X.is_contiguous():
+        raise ValueError("X must be a contiguous CUDA fp16 [N, K] tensor")
+    if Y is None:
+        Y = torch.empty((N, w.M), dtype=torch.float16, device=X.device)
+    _check(lib().w4a16_gemm(_ptr(w.wq), _ptr(w.scales), _ptr(w.zeros), _ptr(X), _ptr(Y),
+                            w.M, K, N, w.group, _stream_ptr(stream)), "w4a16_gemm")
+    return Y
+
+
+def dequant_debug(w: PackedWeight, W_out=None, stream=None):
+    """fp16 W [M, K] from the packed buffers via w4a16_dequant_debug."""
+    import torch
+
+    if W_out is None:
+        W_out = torch.empty((w.M, w.K), dtype=torch.float16, device=w.wq.device)
+    _check(lib().w4a16_dequant_debug(_ptr(w.wq), _ptr(w.scales), _ptr(w.zeros),
+                                     _ptr(W_out), w.M, w.K, w.group, _stream_ptr(stream)),
+           "w4a16_dequant_debug")
+    return W_out
+
+
+def device_status(stream=None) -> int:
+    """Synchronise and read/clear the device wait-timeout status."""
+    st = _i(0)
+    _check(lib().w4a16_device_status(_stream_ptr(stream), ctypes.byref(st)),
+           "w4a16_device_status")
+    return st.value

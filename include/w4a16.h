@@ -1,0 +1,143 @@
+/*
+ * w4a16.h -- C ABI of the B200 (sm_100a) W4A16 group-128 linear layer.
+ *
+ * The operation ("PerfXLLM on Snapdragon 8 Gen2", section 3.3 item 1, GEMM
+ * definition; item 2, GEMV as its n = 1 case; section 3.1, AWQ weight-only
+ * int4 quantisation with group_size 128 and a scale and a zero per group):
+ *
+ *     Y[n][m] = sum_k  w[m][k] * X[n][k],     w[m][k] = fp16_RN((q[m][k] - z[m][g]) * s[m][g]),
+ *     g = k / 128,  q, z in 0..15 (unsigned 4-bit),  s fp16,  X, Y fp16,
+ *
+ * i.e. Y = X . dequant(W)^T with X token-major [N][K] and Y token-major [N][M]
+ * (the same memory as column-major X[K][N] and Y[M][N]).  The products are
+ * accumulated in fp32 and Y is rounded once to fp16 (round to nearest even).
+ *
+ * Conventions for every entry point
+ *   - Buffers are owned by the caller.  The library allocates no device
+ *     memory and never synchronises the stream it is given.
+ *   - Pointers named "device" must be device (or managed) memory of the
+ *     current CUDA device; every one must be 16-byte aligned.
+ *   - Argument checks run on the host before any launch and return an error
+ *     code without touching the GPU.  Launch failures are reported as
+ *     W4A16_ERR_CUDA.  Nothing is thrown and nothing exits.
+ *   - Calls are asynchronous on `stream` (0 = the legacy default stream).
+ */
+#ifndef W4A16_H
+#define W4A16_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define W4A16_API __attribute__((visibility("default")))
+#else
+#define W4A16_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    W4A16_OK = 0,
+    W4A16_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, bad path */
+    W4A16_ERR_UNSUPPORTED = 2,  /* group != 128, K % 128 != 0, sizes too big */
+    W4A16_ERR_MISALIGNED = 3,   /* a pointer is not 16-byte aligned */
+    W4A16_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+    W4A16_ERR_TIMEOUT = 5       /* a bounded device-side wait ran out */
+} w4a16_status;
+
+/* Kernel selection for w4a16_gemm_ex. */
+typedef enum {
+    W4A16_PATH_AUTO = 0,     /* choose by N (the dispatcher) */
+    W4A16_PATH_GEMV = 1,     /* CUDA-core decode kernel (memory-bound, small N) */
+    W4A16_PATH_TC = 2        /* tcgen05 tensor-core kernel (large N) */
+} w4a16_path;
+
+/* Human-readable name of a status code.  Never returns NULL. */
+W4A16_API const char* w4a16_status_string(int status);
+
+/*
+ * Packed-weight sizes, in bytes, for an M x K weight with the given group.
+ *
+ * Packed layout (all three buffers are padded to Mp = ceil(M / 128) * 128 rows;
+ * padding rows hold q = 0, z = 0, s = 0, i.e. zero weights):
+ *   wq     : Mp * K / 2 bytes.  16-byte chunk (b, c, r) at byte offset
+ *            ((b * K/32 + c) * 128 + r) * 16 holds the 32 codes
+ *            q[128 b + r][32 c + j], j = 0..31, as four little-endian 32-bit
+ *            words; word j/8 keeps the 8 codes of j = 8t..8t+7 with the code of
+ *            offset o = j % 8 in nibble p = o/2 (o even) or 4 + o/2 (o odd),
+ *            nibble p occupying bits 4p..4p+3.  A row's codes for offsets
+ *            (2i, 2i+1) thus sit 16 bits apart, which lets one mask-and-or
+ *            form both as fp16 values 1024 + q.
+ *   scales : Mp * K/128 * 2 bytes, fp16 at ((b * K/128 + g) * 128 + r).
+ *   zeros  : Mp * K/128 / 2 bytes, byte ((b * K/128 + g) * 64 + r/2), low
+ *            nibble for even r, high nibble for odd r.
+ * Metadata is 2.5 bytes per group of 128 weights (about 1 % of the fp16
+ * weight size, 3.9 % of the int4 size).
+ *
+ * Returns W4A16_ERR_INVALID_ARG for null outputs or M, K <= 0,
+ * W4A16_ERR_UNSUPPORTED for group != 128 or K % 128 != 0.
+ */
+W4A16_API w4a16_status w4a16_packed_sizes(int M, int K, int group,
+                                size_t* wq_bytes, size_t* scales_bytes,
+                                size_t* zeros_bytes);
+
+/*
+ * Canonical -> packed layout (offline; not on the per-token path).
+ *   q       device uint8  [M][K], values 0..15 (higher bits are ignored)
+ *   scales  device fp16   [M][K/128]
+ *   zeros   device uint8  [M][K/128], values 0..15 (higher bits are ignored)
+ *   wq_packed, scales_packed, zeros_packed: device outputs of the sizes
+ *   w4a16_packed_sizes returns.  Inputs need only natural alignment; the
+ *   outputs must be 16-byte aligned.
+ */
+W4A16_API w4a16_status w4a16_pack(const uint8_t* q, const uint16_t* scales, const uint8_t* zeros,
+                        int M, int K, int group,
+                        void* wq_packed, void* scales_packed, void* zeros_packed,
+                        void* stream);
+
+/*
+ * Y[N][M] = X[N][K] . dequant(W)[M][K]^T   (fp16 in, fp32 accumulate, fp16 out)
+ *   wq_packed, scales_packed, zeros_packed: device, packed as above.
+ *   X  device fp16 [N][K] (token-major), 16-byte aligned.
+ *   Y  device fp16 [N][M] (token-major), 16-byte aligned; fully overwritten.
+ *   M >= 1, N >= 1, K a positive multiple of 128, group == 128.
+ * The result is deterministic: the same inputs give the same bits.
+ */
+W4A16_API w4a16_status w4a16_gemm(const void* wq_packed, const void* scales_packed,
+                        const void* zeros_packed, const uint16_t* X, uint16_t* Y,
+                        int M, int K, int N, int group, void* stream);
+
+/* As w4a16_gemm, with the kernel forced (w4a16_path).  W4A16_PATH_AUTO is the
+ * same as w4a16_gemm.  Used by tests and the benchmark to time both paths. */
+W4A16_API w4a16_status w4a16_gemm_ex(const void* wq_packed, const void* scales_packed,
+                           const void* zeros_packed, const uint16_t* X, uint16_t* Y,
+                           int M, int K, int N, int group, int path, void* stream);
+
+/* The path w4a16_gemm would take for these sizes (a w4a16_path value other
+ * than AUTO), or -1 if the sizes are invalid.  Host only; touches no GPU. */
+W4A16_API int w4a16_select_path(int M, int K, int N);
+
+/*
+ * Writes the dequantised weight W[m][k] = fp16_RN((q - z) * s) as fp16,
+ * row-major [M][K], from the packed buffers.  The values are bit-identical to
+ * what the GEMM kernels multiply; parity checks compare them with an
+ * independent CPU computation.
+ */
+W4A16_API w4a16_status w4a16_dequant_debug(const void* wq_packed, const void* scales_packed,
+                                 const void* zeros_packed, uint16_t* W_out,
+                                 int M, int K, int group, void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device-side status word
+ * that bounded waits inside the tensor-core kernel set when they give up.
+ * Writes W4A16_OK or W4A16_ERR_TIMEOUT to *status.  Not for the hot path.
+ */
+W4A16_API w4a16_status w4a16_device_status(void* stream, int* status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A16_H */

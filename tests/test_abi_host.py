@@ -1,0 +1,108 @@
+"""Host-side checks of the C-ABI library: it loads, exports every entry point
+the header declares, computes packed sizes in closed form, and rejects bad
+arguments before touching a GPU.  No kernel runs here."""
+import ctypes
+import json
+import os
+import re
+
+import pytest
+
+from gemm_w4a16_b200 import build as lib_build
+from gemm_w4a16_b200 import w4a16
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "w4a16.h")
+GOLDEN = os.path.join(ROOT, "tests", "golden")
+
+
+@pytest.fixture(scope="module")
+def L():
+    lib_build.build()
+    return w4a16.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(w4a16_[a-z_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 8
+    assert set(names) == set(w4a16.EXPORTED)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for code in range(6):
+        assert w4a16.status_string(code)
+    assert w4a16.status_string(99) == "unknown status"
+
+
+def test_packed_sizes_closed_form(L):
+    for M, K in [(256, 256), (12288, 4096), (4096, 11008), (128256, 4096), (200, 384), (1, 128)]:
+        wq, s, z = w4a16.packed_sizes(M, K)
+        mp = -(-M // 128) * 128
+        assert wq == mp * K // 2
+        assert s == mp * (K // 128) * 2
+        assert z == mp * (K // 128) // 2
+
+
+def test_pages_footprint_facts(L):
+    """Section 3.1 of the PerfXLLM page: int4 is 1/4 of fp16 and scale+zero
+    add about 1 %; 7B parameters in fp16 take about 14 GB."""
+    facts = json.load(open(os.path.join(GOLDEN, "pages_facts.json")))
+    G = facts["group_size"]["value"]
+    M, K = facts["gemm_sweep_M"]["value"], facts["gemm_sweep_K"]["value"]
+    assert G == 128 and (M, K) == (12288, 4096)
+    wq, s, z = w4a16.packed_sizes(M, K, G)
+    fp16 = M * K * 2
+    assert wq / fp16 == facts["int4_vs_fp16_ratio"]["value"]
+    overhead = (s + z) / fp16
+    assert abs(overhead - facts["scale_zero_overhead_fraction"]["value"]) < 0.001
+    assert abs(overhead - 2.5 / 256) < 1e-12
+    assert abs(facts["fp16_7b_bytes"]["params"] * 2 - facts["fp16_7b_bytes"]["value"]) < 0.05e9
+
+
+def test_rejects_bad_arguments_without_launching(L):
+    bad = ctypes.c_void_p(0x1001)      # never dereferenced: checks fail first
+    good = ctypes.c_void_p(0x10000)
+    null = ctypes.c_void_p(0)
+    g = L.w4a16_gemm_ex
+    args = lambda **kw: [kw.get("wq", good), good, good, kw.get("x", good), kw.get("y", good),
+                         kw.get("M", 256), kw.get("K", 256), kw.get("N", 1),
+                         kw.get("group", 128), kw.get("path", 0), null]
+    assert g(*args(wq=null)) == w4a16.ERR_INVALID_ARG
+    assert g(*args(y=null)) == w4a16.ERR_INVALID_ARG
+    assert g(*args(M=0)) == w4a16.ERR_INVALID_ARG
+    assert g(*args(N=0)) == w4a16.ERR_INVALID_ARG
+    assert g(*args(N=-3)) == w4a16.ERR_INVALID_ARG
+    assert g(*args(K=-128)) == w4a16.ERR_INVALID_ARG
+    assert g(*args(path=7)) == w4a16.ERR_INVALID_ARG
+    assert g(*args(group=64)) == w4a16.ERR_UNSUPPORTED
+    assert g(*args(K=200)) == w4a16.ERR_UNSUPPORTED
+    assert g(*args(x=bad)) == w4a16.ERR_MISALIGNED
+    assert g(*args(wq=bad)) == w4a16.ERR_MISALIGNED
+    assert L.w4a16_gemm(good, good, good, good, bad, 256, 256, 1, 128, null) == w4a16.ERR_MISALIGNED
+    assert L.w4a16_dequant_debug(good, good, good, null, 256, 256, 128, null) == w4a16.ERR_INVALID_ARG
+    assert L.w4a16_dequant_debug(good, good, good, bad, 256, 256, 128, null) == w4a16.ERR_MISALIGNED
+    assert L.w4a16_pack(good, good, good, 256, 256, 100, good, good, good, null) == w4a16.ERR_UNSUPPORTED
+    assert L.w4a16_pack(good, good, null, 256, 256, 128, good, good, good, null) == w4a16.ERR_INVALID_ARG
+    assert L.w4a16_pack(good, good, good, 256, 256, 128, bad, good, good, null) == w4a16.ERR_MISALIGNED
+    sz = ctypes.c_size_t()
+    assert L.w4a16_packed_sizes(256, 256, 128, None, ctypes.byref(sz), ctypes.byref(sz)) == \
+        w4a16.ERR_INVALID_ARG
+    assert L.w4a16_device_status(null, None) == w4a16.ERR_INVALID_ARG
+
+
+def test_select_path_is_monotone_in_n(L):
+    assert w4a16.select_path(0, 4096, 1) == -1
+    assert w4a16.select_path(4096, 100, 1) == -1
+    assert w4a16.select_path(12288, 4096, 1) == w4a16.PATH_GEMV
+    paths = [w4a16.select_path(12288, 4096, n) for n in (1, 2, 4, 8, 16, 64, 256, 4096)]
+    first_tc = paths.index(w4a16.PATH_TC) if w4a16.PATH_TC in paths else len(paths)
+    assert all(p == w4a16.PATH_GEMV for p in paths[:first_tc])
+    assert all(p == w4a16.PATH_TC for p in paths[first_tc:])
