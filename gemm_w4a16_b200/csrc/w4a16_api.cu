@@ -18,7 +18,7 @@ namespace {
 using namespace w4a16;
 
 constexpr int kMaxM = 1 << 24;
-constexpr int kMaxK = 1 << 20;
+constexpr int kMaxK = 1 << 16;
 constexpr int kMaxN = 1 << 20;
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
