@@ -362,6 +362,8 @@ def main_ours(args):
         return single_shape(args, device, 12288, 4096, 1)
     if args.workload == "prefill":
         return single_shape(args, device, 12288, 4096, 4096)
+    if args.workload == "shape":
+        return single_shape(args, device, args.M, args.K, args.N, args.path)
 
     calls, x_flat, y_flat = build_decode_step(device, seed=1000 + rank)
     step_bytes = sum(alg_bytes(w.M, w.K, 1) for _, w, _, _ in calls)
@@ -494,7 +496,7 @@ def prefill_measure(device, peaks, args):
     return out
 
 
-def single_shape(args, device, M, K, N):
+def single_shape(args, device, M, K, N, path=0):
     """One shape, plain launches (used for ncu captures and quick timing)."""
     import torch
 
@@ -504,19 +506,19 @@ def single_shape(args, device, M, K, N):
     w, x = make_device_problem(device, M, K, N, seed=3)
     y = torch.empty((N, M), dtype=torch.float16, device=device)
     for _ in range(args.warmup):
-        w4a16.gemm(w, x, Y=y)
+        w4a16.gemm_ex(w, x, Y=y, path=path)
     torch.cuda.synchronize(device)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(args.steps):
-        w4a16.gemm(w, x, Y=y)
+        w4a16.gemm_ex(w, x, Y=y, path=path)
     e1.record()
     torch.cuda.synchronize(device)
     ms = e0.elapsed_time(e1) / args.steps
     b, f = alg_bytes(M, K, N), alg_flops(M, K, N)
     print(json.dumps({"workload": f"M={M} K={K} N={N}", "us": ms * 1e3,
                       "GBps": b / (ms * 1e-3) / 1e9, "TFLOPS": f / (ms * 1e-3) / 1e12,
-                      "path": w4a16.select_path(M, K, N),
+                      "path": path or w4a16.select_path(M, K, N),
                       "note": "plain launches; weights may sit in L2 across iterations"}))
     return 0
 
@@ -563,7 +565,12 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["decode", "qkv_n1", "prefill", "sweep"], default="decode")
+    ap.add_argument("--workload", choices=["decode", "qkv_n1", "prefill", "sweep", "shape"],
+                    default="decode")
+    ap.add_argument("--M", type=int, default=12288)
+    ap.add_argument("--K", type=int, default=4096)
+    ap.add_argument("--N", type=int, default=1)
+    ap.add_argument("--path", type=int, default=0, help="0 auto, 1 GEMV, 2 tensor cores")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")

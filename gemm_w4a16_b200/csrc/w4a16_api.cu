@@ -133,7 +133,18 @@ w4a16_status w4a16_dequant_debug(const void* wq_packed, const void* scales_packe
 
 w4a16_status w4a16_device_status(void* stream, int* status) {
   if (!status) return W4A16_ERR_INVALID_ARG;
-  return map_cuda(read_and_clear_device_status(static_cast<cudaStream_t>(stream), status));
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  int a = 0, b = 0;
+  if (e == cudaSuccess) e = read_and_clear_tc_status(&a);
+  if (e == cudaSuccess) e = read_and_clear_gemv_status(&b);
+  if (e != cudaSuccess) return map_cuda(e);
+  *status = (a || b) ? W4A16_ERR_TIMEOUT : W4A16_OK;
+  return W4A16_OK;
+}
+
+w4a16_status w4a16_selftest_wait_timeout(long long limit_cycles, void* stream) {
+  if (limit_cycles < 0 || limit_cycles > (1LL << 32)) return W4A16_ERR_INVALID_ARG;
+  return map_cuda(launch_wait_timeout_selftest(limit_cycles, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -5,21 +5,22 @@
 // shared memory to cut global traffic.  On sm_100a the tile is 128 weight
 // rows x BN tokens, K in stages of 64:
 //
-//   warp 0        producer: per stage one TMA tile of X (BN x 64 fp16, 128-byte
+//   warp 4        producer: per stage one TMA tile of X (BN x 64 fp16, 128-byte
 //                 swizzle, rows past N zero-filled) and bulk copies of the
 //                 stage's packed codes (128 rows x 64 codes = 4 KB, contiguous
 //                 in the packed layout) and of its group's scales and zeros.
-//   warps 4..11   dequantisers: one weight row per thread (warp w serves TMEM
-//                 lanes 32 (w % 4) ..), half a stage each; the exact
+//   warps 8..23   dequantisers: four groups of four warps take the stages in
+//                 turn (four stages in flight); one weight row per thread
+//                 (warp w serves TMEM lanes 32 (w % 4) ..), 64 codes; the exact
 //                 in-register dequant (the same one the GEMV uses) writes
 //                 fp16 W straight into tensor memory with tcgen05.st, where
 //                 it is the MMA's A operand -- W never round-trips through
 //                 shared memory, so shared-memory bandwidth is left to X.
-//   warp 1        MMA issuer: tcgen05.mma kind::f16 (A from TMEM, B = X from
+//   warp 5        MMA issuer: tcgen05.mma kind::f16 (A from TMEM, B = X from
 //                 shared memory, fp32 accumulator in TMEM), 4 MMAs of K = 16
 //                 per stage; tcgen05.commit releases the stage, the A slot
 //                 and, at the end of a tile, the accumulator.
-//   warps 12..15  epilogue: tcgen05.ld of the fp32 accumulator, one RNE
+//   warps 0..3    epilogue: tcgen05.ld of the fp32 accumulator, one RNE
 //                 conversion to fp16, stores of Y[n][m].
 //
 // Persistent CTAs (one per SM) walk the tile list round-robin; accumulators
@@ -37,19 +38,21 @@
 
 namespace w4a16 {
 
-__device__ int g_device_status = 0;
+__device__ int g_tc_status = 0;
 
 namespace {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;
-constexpr int kThreads = 512;
+// Warp roles: 0..3 epilogue (TMEM lane quadrants 0..3), 4 producer, 5 MMA
+// issuer and TMEM owner, 6..7 idle, 8.. dequantiser groups of 4 warps.
+constexpr int kDqGroups = 4;                     // stages dequantised concurrently
+constexpr int kFirstDqWarp = 8;
+constexpr int kThreads = (kFirstDqWarp + 4 * kDqGroups) * 32;
 constexpr int kWBytes = kBM * kBK / 2;       // packed codes of one stage
 constexpr int kSBytes = kBM * 2;             // scales of the stage's group
 constexpr int kZBytes = kBM / 2;             // zeros of the stage's group
-constexpr int kASlots = 4;                   // TMEM A slots (32 columns each)
 constexpr int kAColsPerSlot = kBK / 2;       // 64 fp16 = 32 columns
-constexpr long long kWaitLimitCycles = 4000000000LL;   // about 2 s
 
 __host__ __device__ constexpr int round_up(int a, int b) { return (a + b - 1) / b * b; }
 
@@ -57,9 +60,17 @@ template <int BN>
 struct Cfg {
   static constexpr int kXBytes = BN * kBK * 2;
   static constexpr int kStageBytes = round_up(kXBytes + kWBytes + kSBytes + kZBytes, 1024);
-  static constexpr int kStages = (200 * 1024 / kStageBytes) < 8 ? (200 * 1024 / kStageBytes) : 8;
-  static constexpr int kAccBufs = (2 * BN + kASlots * kAColsPerSlot <= 512) ? 2 : 1;
+  // As many stages as fit in about 200 KB (a multiple of the dequantiser
+  // group count, at most 24): the ring is what keeps copies in flight.
+  static constexpr int kStagesFit = (200 * 1024 / kStageBytes) / kDqGroups * kDqGroups;
+  static constexpr int kStages = kStagesFit < 24 ? kStagesFit : 24;
+  static constexpr int kAccBufs = (2 * BN + kDqGroups * kAColsPerSlot <= 512) ? 2 : 1;
   static constexpr int kACol0 = kAccBufs * BN;
+  // TMEM A slots (32 columns each): all the columns the accumulators leave,
+  // a multiple of the dequantiser group count, at most 12.  The slot ring is
+  // what lets dequantisation run ahead of MMA completion.
+  static constexpr int kASlotsFit = (512 - kACol0) / kAColsPerSlot / kDqGroups * kDqGroups;
+  static constexpr int kASlots = kASlotsFit < 12 ? kASlotsFit : 12;
   static constexpr int kColsUsed = kACol0 + kASlots * kAColsPerSlot;
   static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
                                    : kColsUsed <= 256 ? 256 : 512;
@@ -70,7 +81,8 @@ struct Cfg {
   static constexpr int kBarBytes = 8 * (2 * kStages + 2 * kASlots + 2 * kAccBufs + 1) + 16;
   static constexpr int kSmemUsed = kStages * kStageBytes + kBarBytes + 1024;
   static constexpr int kSmemBytes = kSmemUsed < 120 * 1024 ? 120 * 1024 : kSmemUsed;
-  static_assert(kStages >= 2, "stage ring too small");
+  static_assert(kStages >= kDqGroups && kStages % kDqGroups == 0, "stage ring");
+  static_assert(kASlots >= kDqGroups && kASlots % kDqGroups == 0, "TMEM A slot ring");
   static_assert(kColsUsed <= 512, "TMEM overflow");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
 };
@@ -87,30 +99,6 @@ struct Shared {
   volatile int* abort_flag;
 };
 
-// Bounded mbarrier wait.  Returns false (after recording a timeout) if the
-// phase does not complete in time, or if another role has aborted.
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                         bool honor_abort = true) {
-  if (ptx::mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (true) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
-    if (honor_abort && *abort_flag) return false;
-    if (clock64() - t0 > kWaitLimitCycles) {
-      *abort_flag = 1;
-      atomicExch(&g_device_status, 1);
-      return false;
-    }
-  }
-}
-
-// Warp-collective form: every lane waits (so every lane acquires the phase),
-// then the warp agrees on one outcome before any .sync.aligned instruction.
-__device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  const bool ok = wait_bar(bar, parity, abort_flag);
-  return __all_sync(0xffffffffu, ok);
-}
-
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __restrict__ wq,
@@ -125,8 +113,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
   sh.full = bars;
   sh.empty = sh.full + C::kStages;
   sh.a_full = sh.empty + C::kStages;
-  sh.a_empty = sh.a_full + kASlots;
-  sh.acc_full = sh.a_empty + kASlots;
+  sh.a_empty = sh.a_full + C::kASlots;
+  sh.acc_full = sh.a_empty + C::kASlots;
   sh.acc_empty = sh.acc_full + C::kAccBufs;
   sh.drain = sh.acc_empty + C::kAccBufs;
   sh.tmem_ptr = reinterpret_cast<uint32_t*>(sh.drain + 1);
@@ -144,10 +132,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kStages; ++i) {
       ptx::mbar_init(&sh.full[i], 1);
-      ptx::mbar_init(&sh.empty[i], 8 + 1);     // 8 dequant warps + 1 MMA commit
+      ptx::mbar_init(&sh.empty[i], 4 + 1);     // 4 dequant warps + 1 MMA commit
     }
-    for (int i = 0; i < kASlots; ++i) {
-      ptx::mbar_init(&sh.a_full[i], 8);
+    for (int i = 0; i < C::kASlots; ++i) {
+      ptx::mbar_init(&sh.a_full[i], 4);
       ptx::mbar_init(&sh.a_empty[i], 1);
     }
     for (int i = 0; i < C::kAccBufs; ++i) {
@@ -159,7 +147,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(&tmap_x);
   }
-  if (warp == 1) {
+  if (warp == 5) {
     ptx::tmem_alloc(sh.tmem_ptr, C::kTmemCols);
     ptx::tmem_relinquish();
   }
@@ -168,7 +156,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
   ptx::tc_fence_after();
   const uint32_t tmem = *sh.tmem_ptr;
 
-  if (warp == 0) {
+  if (warp == 4) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int s = 0;
@@ -179,7 +167,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
         const int mt = t % mt_n, nt = t / mt_n;
         const uint8_t* wblk = wq + (size_t)mt * kc_n * kRowBlock * 16;
         for (int ks = 0; ks < ks_n; ++ks) {
-          if (!wait_bar(&sh.empty[s], ph ^ 1, sh.abort_flag)) { ok = false; break; }
+          if (!wait_bar(&sh.empty[s], ph ^ 1, sh.abort_flag, &g_tc_status)) { ok = false; break; }
           uint8_t* st = smem + s * C::kStageBytes;
           ptx::mbar_arrive_expect_tx(&sh.full[s], C::kTx);
           ptx::tma_load_2d(st, &tmap_x, &sh.full[s], ks * kBK, nt * BN);
@@ -196,9 +184,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
       }
       // Drain: every copy issued into this CTA's shared memory has landed.
       for (int i = 0; i < C::kStages; ++i)
-        if (issued_mask & (1u << i)) wait_bar(&sh.full[i], (issued_par >> i) & 1u, sh.abort_flag, false);
+        if (issued_mask & (1u << i)) wait_bar(&sh.full[i], (issued_par >> i) & 1u, sh.abort_flag, &g_tc_status, false);
     }
-  } else if (warp == 1) {
+  } else if (warp == 5) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       int s = 0, a = 0, b = 0;
@@ -206,11 +194,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
       bool ok = true;
       const uint32_t x_base = ptx::smem_addr(smem);
       for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
-        if (!wait_bar(&sh.acc_empty[b], bph ^ 1, sh.abort_flag)) break;
+        if (!wait_bar(&sh.acc_empty[b], bph ^ 1, sh.abort_flag, &g_tc_status)) break;
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem + b * BN;
         for (int ks = 0; ks < ks_n; ++ks) {
-          if (!wait_bar(&sh.full[s], ph, sh.abort_flag) || !wait_bar(&sh.a_full[a], aph, sh.abort_flag)) {
+          if (!wait_bar(&sh.full[s], ph, sh.abort_flag, &g_tc_status) || !wait_bar(&sh.a_full[a], aph, sh.abort_flag, &g_tc_status)) {
             ok = false;
             break;
           }
@@ -224,7 +212,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
           ptx::mma_commit(&sh.empty[s]);
           ptx::mma_commit(&sh.a_empty[a]);
           if (++s == C::kStages) { s = 0; ph ^= 1; }
-          if (++a == kASlots) { a = 0; aph ^= 1; }
+          if (++a == C::kASlots) { a = 0; aph ^= 1; }
         }
         if (!ok) break;
         ptx::mma_commit(&sh.acc_full[b]);
@@ -232,44 +220,51 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
       }
       // Drain: all MMAs issued by this thread have completed.
       ptx::mma_commit(sh.drain);
-      wait_bar(sh.drain, 0, sh.abort_flag, false);
+      wait_bar(sh.drain, 0, sh.abort_flag, &g_tc_status, false);
     }
-  } else if (warp >= 4 && warp < 12) {
+  } else if (warp >= kFirstDqWarp) {
     // -------------------------------------------------------- dequantisers
+    // Group gi takes every kDqGroups-th stage of this CTA's sequence (so
+    // kDqGroups stages are in flight at once); stage i goes to TMEM A slot
+    // i % kASlots; each thread dequantises the 64 codes of one row.
+    const int gi = (warp - kFirstDqWarp) >> 2;
     const int quad = warp & 3;
-    const int half = (warp - 4) >> 2;
     const int row = quad * 32 + lane;
-    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-    int s = 0, a = 0;
-    uint32_t ph = 0, aph = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
-      for (int ks = 0; ks < ks_n; ++ks) {
-        if (!wait_bar_warp(&sh.full[s], ph, sh.abort_flag)) { ok = false; break; }
-        const uint8_t* st = smem + s * C::kStageBytes;
-        const uint4 v = *reinterpret_cast<const uint4*>(st + C::kXBytes + half * (kRowBlock * 16) + row * 16);
-        const uint16_t sv = reinterpret_cast<const uint16_t*>(st + C::kXBytes + kWBytes)[row];
-        const uint32_t zb = st[C::kXBytes + kWBytes + kSBytes + (row >> 1)];
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&sh.empty[s]);
-        const GroupConsts gc = make_group_consts((zb >> ((row & 1) * 4)) & 0xFu, sv);
-        uint32_t h[16];
-        dequant_word(v.x, gc, &h[0]);
-        dequant_word(v.y, gc, &h[4]);
-        dequant_word(v.z, gc, &h[8]);
-        dequant_word(v.w, gc, &h[12]);
-        if (!wait_bar_warp(&sh.a_empty[a], aph ^ 1, sh.abort_flag)) { ok = false; break; }
-        ptx::tc_fence_after();
-        ptx::tmem_st_x16(lane_base + C::kACol0 + a * kAColsPerSlot + 16 * half, h);
-        ptx::tmem_wait_st();
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&sh.a_full[a]);
-        if (++s == C::kStages) { s = 0; ph ^= 1; }
-        if (++a == kASlots) { a = 0; aph ^= 1; }
-      }
+    const uint32_t a_lane = tmem + ((uint32_t)(quad * 32) << 16) + C::kACol0;
+    const int my_tiles = (tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+    const long long n_stages = (long long)my_tiles * ks_n;
+    for (long long i = gi; i < n_stages; i += kDqGroups) {
+      const int s = (int)(i % C::kStages);
+      const uint32_t ph = (uint32_t)((i / C::kStages) & 1);
+      const int a = (int)(i % C::kASlots);
+      const uint32_t aph = (uint32_t)((i / C::kASlots) & 1);
+      if (!wait_bar_warp(&sh.full[s], ph, sh.abort_flag, &g_tc_status)) break;
+      const uint8_t* st = smem + s * C::kStageBytes;
+      const uint4 v0 = *reinterpret_cast<const uint4*>(st + C::kXBytes + row * 16);
+      const uint4 v1 = *reinterpret_cast<const uint4*>(st + C::kXBytes + kRowBlock * 16 + row * 16);
+      const uint16_t sv = reinterpret_cast<const uint16_t*>(st + C::kXBytes + kWBytes)[row];
+      const uint32_t zb = st[C::kXBytes + kWBytes + kSBytes + (row >> 1)];
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&sh.empty[s]);
+      const GroupConsts gc = make_group_consts((zb >> ((row & 1) * 4)) & 0xFu, sv);
+      uint32_t h[32];
+      dequant_word(v0.x, gc, &h[0]);
+      dequant_word(v0.y, gc, &h[4]);
+      dequant_word(v0.z, gc, &h[8]);
+      dequant_word(v0.w, gc, &h[12]);
+      dequant_word(v1.x, gc, &h[16]);
+      dequant_word(v1.y, gc, &h[20]);
+      dequant_word(v1.z, gc, &h[24]);
+      dequant_word(v1.w, gc, &h[28]);
+      if (!wait_bar_warp(&sh.a_empty[a], aph ^ 1, sh.abort_flag, &g_tc_status)) break;
+      ptx::tc_fence_after();
+      ptx::tmem_st_x32(a_lane + a * kAColsPerSlot, h);
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&sh.a_full[a]);
     }
-  } else if (warp >= 12) {
+  } else if (warp < 4) {
     // ------------------------------------------------------------ epilogue
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
@@ -278,7 +273,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
     uint32_t bph = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
       const int mt = t % mt_n, nt = t / mt_n;
-      if (!wait_bar_warp(&sh.acc_full[b], bph, sh.abort_flag)) break;
+      if (!wait_bar_warp(&sh.acc_full[b], bph, sh.abort_flag, &g_tc_status)) break;
       ptx::tc_fence_after();
       const int m = mt * kBM + row;
       const int n0 = nt * BN;
@@ -304,7 +299,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
 
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 5) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::kTmemCols);
   }
@@ -388,17 +383,33 @@ cudaError_t launch_gemm_tc(const uint8_t* wq, const uint16_t* scales, const uint
   return launch_bn<128>(wq, scales, zeros, X, Y, M, K, N, stream);
 }
 
-cudaError_t read_and_clear_device_status(cudaStream_t stream, int* status) {
-  cudaError_t e = cudaStreamSynchronize(stream);
+namespace {
+
+// One thread waits on an mbarrier whose phase nothing completes, with a short
+// cycle budget: the wait must give up, record the timeout and return.
+__global__ void wait_timeout_selftest_kernel(long long limit) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&bar, 1);
+    abort_flag = 0;
+    ptx::fence_mbar_init();
+    wait_bar(&bar, 0, &abort_flag, &g_tc_status, true, limit);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_wait_timeout_selftest(long long limit_cycles, cudaStream_t stream) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(limit_cycles);
+  return cudaGetLastError();
+}
+
+cudaError_t read_and_clear_tc_status(int* v) {
+  cudaError_t e = cudaMemcpyFromSymbol(v, g_tc_status, sizeof(int));
   if (e != cudaSuccess) return e;
-  int v = 0;
-  e = cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int));
-  if (e != cudaSuccess) return e;
-  int zero = 0;
-  e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
-  if (e != cudaSuccess) return e;
-  *status = v ? W4A16_ERR_TIMEOUT : W4A16_OK;
-  return cudaSuccess;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_tc_status, &zero, sizeof(int));
 }
 
 }  // namespace w4a16

@@ -2,38 +2,46 @@
 //
 // "PerfXLLM on Snapdragon 8 Gen2", section 3.3 item 2: the GEMV is memory
 // bound; its design goals there are vectorised loads, unrolling to keep many
-// loads in flight, the zero and scale of each int4 group kept close to the
-// compute, and tiling both dimensions of the weight (rows and K) for
-// parallelism.  On sm_100a that becomes:
+// loads in flight, the zero and scale of each int4 group kept in shared
+// memory, the vector read through a texture-like path, and tiling both
+// dimensions of the weight (rows and K) for parallelism.  On sm_100a:
 //
-//  * thread = one weight row; a warp covers 32 rows and reads 32 x 16 bytes
-//    = 512 contiguous bytes of the packed layout per load instruction;
-//  * each warp owns a range of whole groups along K and walks it with the
-//    next group's loads (4 x 16 B + scale + zero per thread) in flight while
-//    the current group is dequantised: double-buffered registers;
-//  * per-(row, group) scale and zero go straight to registers with the
-//    weight loads (each is read once; there is no reuse for shared memory to
-//    capture in this mapping);
-//  * the CTA's slice of the activations is staged once in shared memory
-//    (the analogue of the page's image-typed vector reads) and read back as
-//    broadcast 16-byte loads, one per 8 codes and token;
-//  * split-K: warps of a CTA reduce through shared memory, and CTAs of a
-//    thread-block cluster (up to 8 along K) reduce through distributed shared
-//    memory into the cluster's rank-0 CTA, always in a fixed order, so the
-//    result is deterministic (no atomics).
-//  * products accumulate in fp32 with the mixed-precision fma.rn.f32.f16.
+//  * a CTA owns one 128-row block of the packed weight and a range of whole
+//    groups along K; a producer warp streams each group (8 KB of codes, 256 B
+//    of scales, 64 B of zeros, contiguous in the packed layout) into a
+//    6-stage shared-memory ring with bulk asynchronous copies, so tens of KB
+//    per CTA are in flight without holding registers;
+//  * the CTA's slice of the activations is staged once in shared memory and
+//    read back as broadcast 16-byte loads;
+//  * two consumer warpgroups take alternate groups; thread = one weight row;
+//    the exact in-register dequant (dequant_word) feeds fma.rn.f32.f16 into
+//    four independent fp32 chains per token;
+//  * split-K: the two warpgroups reduce through shared memory, and CTAs of a
+//    thread-block cluster (up to 8 along K) through distributed shared memory
+//    into the cluster's rank-0 CTA, in a fixed order (deterministic, no
+//    atomics);
+//  * every mbarrier wait is bounded (device status word on expiry).
 #include "w4a16_internal.cuh"
+#include "sm100_ptx.cuh"
 
 #include <algorithm>
 
 namespace w4a16 {
+
+__device__ int g_gemv_status = 0;
+
 namespace {
 
-constexpr int kGemvWarps = 4;                 // warps splitting K inside a CTA
-constexpr int kGemvThreads = kGemvWarps * 32;
-constexpr int kRowsPerCta = 32;               // one row per lane
+constexpr int kGvHalves = 2;                          // consumer warpgroups (alternate groups)
+constexpr int kGvConsumerWarps = 4 * kGvHalves;
+constexpr int kGvProducerWarp = kGvConsumerWarps;
+constexpr int kGvThreads = (kGvConsumerWarps + 1) * 32;
+constexpr int kGvWBytes = 4 * kRowBlock * 16;         // one group of 128 rows: 8 KB
+constexpr int kGvStageBytes = kGvWBytes + kRowBlock * 2 + kRowBlock / 2;   // + scales + zeros
+constexpr int kGvStages = 6;                          // multiple of kGvHalves
 constexpr int kMaxCluster = 8;
-constexpr int kMaxXSmem = 96 * 1024;          // largest staged activation slice
+constexpr int kMaxXSmem = 64 * 1024;                  // largest staged activation slice
+static_assert(kGvStages % kGvHalves == 0, "stage ring");
 
 __device__ __forceinline__ void fma_h2(float& acc, uint32_t w, uint32_t x) {
   asm("{\n\t.reg .f16 wl, wh, xl, xh;\n\t"
@@ -44,121 +52,144 @@ __device__ __forceinline__ void fma_h2(float& acc, uint32_t w, uint32_t x) {
       : "+f"(acc) : "r"(w), "r"(x));
 }
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-// One group (128 codes) of one row: four 16-byte chunks plus its scale and
-// zero byte.
-struct GroupRegs {
-  uint4 v[4];
-  uint16_t s;
-  uint32_t z;
+struct GvLayout {
+  int x_off, red_off, cred_off, bar_off, total;
 };
 
+__host__ __device__ inline GvLayout gv_layout(int nt, int gspan, int cl) {
+  GvLayout L;
+  L.x_off = kGvStages * kGvStageBytes;
+  L.red_off = L.x_off + nt * gspan * kGroup * 2;
+  L.cred_off = L.red_off + kGvHalves * nt * kRowBlock * 4;
+  L.bar_off = L.cred_off + (cl > 1 ? cl * nt * kRowBlock * 4 : 0);
+  L.total = L.bar_off + 8 * (2 * kGvStages + 1) + 16;
+  return L;
+}
+
 template <int NT>
-__global__ void __launch_bounds__(kGemvThreads, NT == 1 ? 8 : 4)
-gemv_kernel(const uint4* __restrict__ wq, const uint16_t* __restrict__ s_p,
+__global__ void __launch_bounds__(kGvThreads)
+gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
             const uint8_t* __restrict__ z_p, const uint16_t* __restrict__ X,
             uint16_t* __restrict__ Y, int M, int K, int cl) {
-  extern __shared__ uint4 xs[];                 // [NT][kspan] fp16, 8 per uint4
-  __shared__ float red[kGemvWarps][NT][32];
-  __shared__ float cred[kMaxCluster][NT][32];
-
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int tile = blockIdx.x / cl;
-  const int crank = blockIdx.x % cl;
-  const int r0 = tile * kRowsPerCta;
-  const int b = r0 / kRowBlock;
-  const int r = (r0 % kRowBlock) + lane;   // row inside the 128-row block
-  const int kc_n = K / kChunkK;
+  extern __shared__ __align__(128) uint8_t smem[];
   const int kg = K / kGroup;
+  const int kc_n = K / kChunkK;
+  const int gspan = ceil_div(kg, cl);
+  const GvLayout L = gv_layout(NT, gspan, cl);
+  uint4* xs = reinterpret_cast<uint4*>(smem + L.x_off);
+  float* red = reinterpret_cast<float*>(smem + L.red_off);     // [halves][NT][128]
+  float* cred = reinterpret_cast<float*>(smem + L.cred_off);   // [cl][NT][128], rank 0 only
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off);
+  uint64_t* empty = full + kGvStages;
+  uint64_t* xbar = empty + kGvStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(xbar + 1);
 
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int b = blockIdx.x / cl;
+  const int crank = blockIdx.x % cl;
+  const int ga = (kg * crank) / cl, gb = (kg * (crank + 1)) / cl;
+  const int ng = gb - ga;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kGvStages; ++i) {
+      ptx::mbar_init(&full[i], 1);
+      ptx::mbar_init(&empty[i], 4);              // the 4 warps of one consumer half
+    }
+    ptx::mbar_init(xbar, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
   if (cl > 1) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 
-  // Whole groups along K: first split across the cluster, then across warps.
-  const int ga = (kg * crank) / cl, gb = (kg * (crank + 1)) / cl;
-  const int g0 = ga + ((gb - ga) * warp) / kGemvWarps;
-  const int g1 = ga + ((gb - ga) * (warp + 1)) / kGemvWarps;
-  const int kspan8 = (gb - ga) * (kGroup / 8);   // uint4 per token in the slice
-
-  const uint4* wrow = wq + (size_t)b * kc_n * kRowBlock + r;   // chunk c at wrow[c * 128]
-  const uint16_t* srow = s_p + (size_t)b * kg * kRowBlock + r;  // group g at srow[g * 128]
-  const uint8_t* zrow = z_p + (size_t)b * kg * (kRowBlock / 2) + (r >> 1);
-  const int zshift = (r & 1) * 4;
-
-  auto load_group = [&](int g, GroupRegs& gr) {
+  float tot[NT];
+  if (warp == kGvProducerWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && ng > 0) {
+      ptx::mbar_arrive_expect_tx(xbar, (uint32_t)(NT * ng * kGroup * 2));
+      for (int n = 0; n < NT; ++n)
+        ptx::bulk_load(reinterpret_cast<uint8_t*>(xs) + n * ng * kGroup * 2,
+                       X + (size_t)n * K + (size_t)ga * kGroup, (uint32_t)(ng * kGroup * 2), xbar);
+      const uint8_t* wblk = wq + (size_t)b * kc_n * kRowBlock * 16;
+      const uint16_t* sblk = s_p + (size_t)b * kg * kRowBlock;
+      const uint8_t* zblk = z_p + (size_t)b * kg * (kRowBlock / 2);
+      int last = -1;
+      for (int i = 0; i < ng; ++i) {
+        const int st = i % kGvStages;
+        const uint32_t ph = (uint32_t)((i / kGvStages) & 1);
+        if (!wait_bar(&empty[st], ph ^ 1, abort_flag, &g_gemv_status)) break;
+        uint8_t* dst = smem + st * kGvStageBytes;
+        const int g = ga + i;
+        ptx::mbar_arrive_expect_tx(&full[st], kGvStageBytes);
+        ptx::bulk_load(dst, wblk + (size_t)g * kGvWBytes, kGvWBytes, &full[st]);
+        ptx::bulk_load(dst + kGvWBytes, sblk + (size_t)g * kRowBlock, kRowBlock * 2, &full[st]);
+        ptx::bulk_load(dst + kGvWBytes + kRowBlock * 2, zblk + (size_t)g * (kRowBlock / 2), kRowBlock / 2,
+                       &full[st]);
+        last = i;
+      }
+      // Drain: every copy issued into this CTA's shared memory has landed.
+      for (int i = (last - kGvStages + 1 > 0 ? last - kGvStages + 1 : 0); i <= last; ++i)
+        wait_bar(&full[i % kGvStages], (uint32_t)((i / kGvStages) & 1), abort_flag, &g_gemv_status, false);
+      wait_bar(xbar, 0, abort_flag, &g_gemv_status, false);
+    }
+    __syncwarp();
+  } else {
+    // ----------------------------------------------------------- consumers
+    // Thread = weight row r of block b; consumer half h takes groups
+    // i = h, h + 2, ...; four independent fp32 chains per token.
+    const int h = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;
+    float acc[NT][4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) gr.v[j] = ldg_stream_v4(wrow + (size_t)(g * 4 + j) * kRowBlock);
-    gr.s = __ldg(srow + (size_t)g * kRowBlock);
-    gr.z = __ldg(zrow + (size_t)g * (kRowBlock / 2));
-  };
-
-  float acc[NT][4];
+    for (int n = 0; n < NT; ++n)
 #pragma unroll
-  for (int n = 0; n < NT; ++n)
+      for (int t = 0; t < 4; ++t) acc[n][t] = 0.f;
+    bool ok = ng == 0 || wait_bar_warp(xbar, 0, abort_flag, &g_gemv_status);
+    for (int i = h; ok && i < ng; i += kGvHalves) {
+      const int st = i % kGvStages;
+      const uint32_t ph = (uint32_t)((i / kGvStages) & 1);
+      if (!wait_bar_warp(&full[st], ph, abort_flag, &g_gemv_status)) break;
+      const uint8_t* src = smem + st * kGvStageBytes;
+      uint4 v[4];
 #pragma unroll
-    for (int t = 0; t < 4; ++t) acc[n][t] = 0.f;
-
-  auto compute_group = [&](int g, const GroupRegs& gr) {
-    const GroupConsts gc = make_group_consts((gr.z >> zshift) & 0xFu, gr.s);
-    const int xo = (g - ga) * (kGroup / 8);
+      for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const uint4*>(src + j * kRowBlock * 16 + r * 16);
+      const uint16_t sv = reinterpret_cast<const uint16_t*>(src + kGvWBytes)[r];
+      const uint32_t zb = src[kGvWBytes + kRowBlock * 2 + (r >> 1)];
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&empty[st]);
+      const GroupConsts gc = make_group_consts((zb >> ((r & 1) * 4)) & 0xFu, sv);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t words[4] = {gr.v[j].x, gr.v[j].y, gr.v[j].z, gr.v[j].w};
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t words[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        uint32_t h[4];
-        dequant_word(words[t], gc, h);
+        for (int t = 0; t < 4; ++t) {
+          uint32_t hw[4];
+          dequant_word(words[t], gc, hw);
 #pragma unroll
-        for (int n = 0; n < NT; ++n) {
-          const uint4 xv = xs[n * kspan8 + xo + j * 4 + t];
-          fma_h2(acc[n][t], h[0], xv.x);
-          fma_h2(acc[n][t], h[1], xv.y);
-          fma_h2(acc[n][t], h[2], xv.z);
-          fma_h2(acc[n][t], h[3], xv.w);
+          for (int n = 0; n < NT; ++n) {
+            const uint4 xv = xs[n * ng * (kGroup / 8) + i * (kGroup / 8) + j * 4 + t];
+            fma_h2(acc[n][t], hw[0], xv.x);
+            fma_h2(acc[n][t], hw[1], xv.y);
+            fma_h2(acc[n][t], hw[2], xv.z);
+            fma_h2(acc[n][t], hw[3], xv.w);
+          }
         }
       }
     }
-  };
-
-  // First group's loads go out before the activation slice is staged, so
-  // their latency overlaps the staging.
-  GroupRegs ga_regs, gb_regs;
-  if (g0 < g1) load_group(g0, ga_regs);
-  {
-    const uint4* xsrc = reinterpret_cast<const uint4*>(X);
-    const int k8 = K / 8;
-    for (int i = threadIdx.x; i < NT * kspan8; i += kGemvThreads) {
-      const int n = i / kspan8, o = i - n * kspan8;
-      xs[i] = __ldg(xsrc + (size_t)n * k8 + ga * (kGroup / 8) + o);
-    }
-  }
-  __syncthreads();
-
-  // Double-buffered walk over the warp's groups: the next group's loads are
-  // in flight while the current one is dequantised and multiplied.
-  for (int g = g0; g < g1; g += 2) {
-    if (g + 1 < g1) load_group(g + 1, gb_regs);
-    compute_group(g, ga_regs);
-    if (g + 1 < g1) {
-      if (g + 2 < g1) load_group(g + 2, ga_regs);
-      compute_group(g + 1, gb_regs);
-    }
-  }
-
 #pragma unroll
-  for (int n = 0; n < NT; ++n) red[warp][n][lane] = (acc[n][0] + acc[n][1]) + (acc[n][2] + acc[n][3]);
+    for (int n = 0; n < NT; ++n)
+      red[(h * NT + n) * kRowBlock + r] = (acc[n][0] + acc[n][1]) + (acc[n][2] + acc[n][3]);
+  }
   __syncthreads();
 
-  float tot[NT];
-  if (warp == 0) {
+  const int r = threadIdx.x;   // rows for the reduction: threads 0..127
+  if (r < kRowBlock) {
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
       float sum = 0.f;
 #pragma unroll
-      for (int w = 0; w < kGemvWarps; ++w) sum += red[w][n][lane];
+      for (int h = 0; h < kGvHalves; ++h) sum += red[(h * NT + n) * kRowBlock + r];
       tot[n] = sum;
     }
   }
@@ -167,10 +198,10 @@ gemv_kernel(const uint4* __restrict__ wq, const uint16_t* __restrict__ s_p,
     // Every CTA of the cluster has started once this wait returns, so its
     // shared memory may be written remotely.
     asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-    if (warp == 0) {
+    if (r < kRowBlock) {
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
-        uint32_t local = smem_u32(&cred[crank][n][lane]);
+        const uint32_t local = ptx::smem_addr(&cred[(crank * NT + n) * kRowBlock + r]);
         uint32_t remote;
         asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(0));
         asm volatile("st.shared::cluster.f32 [%0], %1;" :: "r"(remote), "f"(tot[n]) : "memory");
@@ -178,18 +209,18 @@ gemv_kernel(const uint4* __restrict__ wq, const uint16_t* __restrict__ s_p,
     }
     asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-    if (crank != 0 || warp != 0) return;
+    if (crank != 0 || r >= kRowBlock) return;
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
       float sum = 0.f;
-      for (int c = 0; c < cl; ++c) sum += cred[c][n][lane];
+      for (int c = 0; c < cl; ++c) sum += cred[(c * NT + n) * kRowBlock + r];
       tot[n] = sum;
     }
-  } else if (warp != 0) {
+  } else if (r >= kRowBlock) {
     return;
   }
 
-  const int m = r0 + lane;
+  const int m = b * kRowBlock + r;
   if (m < M) {
 #pragma unroll
     for (int n = 0; n < NT; ++n) Y[(size_t)n * M + m] = __half_as_ushort(__float2half_rn(tot[n]));
@@ -208,27 +239,24 @@ int sm_count() {
   return cached[dev];
 }
 
-int x_smem_bytes(int K, int cl, int nt) {
-  const int kg = K / kGroup;
-  return nt * ceil_div(kg, cl) * kGroup * 2;
-}
-
 template <int NT>
-cudaError_t launch_nt(const uint4* wq, const uint16_t* s_p, const uint8_t* z_p, const uint16_t* X,
-                      uint16_t* Y, int M, int K, int cl, int tiles, cudaStream_t stream) {
+cudaError_t launch_nt(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p, const uint16_t* X,
+                      uint16_t* Y, int M, int K, int cl, cudaStream_t stream) {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(gemv_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kMaxXSmem);
+                                         200 * 1024);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
+  const int blocks = ceil_div(M, kRowBlock);
+  const GvLayout L = gv_layout(NT, ceil_div(K / kGroup, cl), cl);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(tiles * cl), 1, 1);
-  cfg.blockDim = dim3(kGemvThreads, 1, 1);
-  cfg.dynamicSmemBytes = (size_t)x_smem_bytes(K, cl, NT);
+  cfg.gridDim = dim3((unsigned)(blocks * cl), 1, 1);
+  cfg.blockDim = dim3(kGvThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)L.total;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -242,41 +270,44 @@ cudaError_t launch_nt(const uint4* wq, const uint16_t* s_p, const uint8_t* z_p, 
 
 }  // namespace
 
-// Cluster size along K.  One wave of CTAs (every CTA resident at once) with as
-// many CTAs as fit, while each warp keeps at least two whole groups so the
-// double-buffered loads have something to overlap; larger if the activation
-// slice would not fit in shared memory.
+// Cluster size along K: the smallest power of two that gives every SM at
+// least two CTAs, keeps two or more groups per CTA, and fits the staged
+// activation slice in shared memory.
 int gemv_cluster_size(int M, int K, int sms, int nt) {
-  const int tiles = ceil_div(M, kRowsPerCta);
+  const int blocks = ceil_div(M, kRowBlock);
   const int kg = K / kGroup;
-  const int resident = sms * (nt == 1 ? 8 : 4);
   int cl = 1;
-  while (cl < kMaxCluster && tiles * cl * 2 <= resident && kg / (2 * cl) >= 2 * kGemvWarps) cl *= 2;
-  while (cl < kMaxCluster && x_smem_bytes(K, cl, nt) > kMaxXSmem) cl *= 2;
+  while (cl < kMaxCluster && blocks * cl < 2 * sms && kg / (2 * cl) >= 2) cl *= 2;
+  while (cl < kMaxCluster && nt * ceil_div(kg, cl) * kGroup * 2 > kMaxXSmem) cl *= 2;
   return cl;
 }
 
 cudaError_t launch_gemv(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros,
                         const uint16_t* X, uint16_t* Y, int M, int K, int N,
                         cudaStream_t stream) {
-  const int tiles = ceil_div(M, kRowsPerCta);
-  const uint4* w4 = reinterpret_cast<const uint4*>(wq);
   for (int n0 = 0; n0 < N; n0 += kGemvMaxTokens) {
     const int nt = std::min(kGemvMaxTokens, N - n0);
     const int cl = gemv_cluster_size(M, K, sm_count(), nt);
-    if (x_smem_bytes(K, cl, nt) > kMaxXSmem) return cudaErrorNotSupported;
+    if (nt * ceil_div(K / kGroup, cl) * kGroup * 2 > kMaxXSmem) return cudaErrorNotSupported;
     const uint16_t* Xn = X + (size_t)n0 * K;
     uint16_t* Yn = Y + (size_t)n0 * M;
     cudaError_t e;
     switch (nt) {
-      case 1: e = launch_nt<1>(w4, scales, zeros, Xn, Yn, M, K, cl, tiles, stream); break;
-      case 2: e = launch_nt<2>(w4, scales, zeros, Xn, Yn, M, K, cl, tiles, stream); break;
-      case 3: e = launch_nt<3>(w4, scales, zeros, Xn, Yn, M, K, cl, tiles, stream); break;
-      default: e = launch_nt<4>(w4, scales, zeros, Xn, Yn, M, K, cl, tiles, stream); break;
+      case 1: e = launch_nt<1>(wq, scales, zeros, Xn, Yn, M, K, cl, stream); break;
+      case 2: e = launch_nt<2>(wq, scales, zeros, Xn, Yn, M, K, cl, stream); break;
+      case 3: e = launch_nt<3>(wq, scales, zeros, Xn, Yn, M, K, cl, stream); break;
+      default: e = launch_nt<4>(wq, scales, zeros, Xn, Yn, M, K, cl, stream); break;
     }
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
+}
+
+cudaError_t read_and_clear_gemv_status(int* v) {
+  cudaError_t e = cudaMemcpyFromSymbol(v, g_gemv_status, sizeof(int));
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_gemv_status, &zero, sizeof(int));
 }
 
 }  // namespace w4a16

@@ -129,6 +129,13 @@ cudaError_t launch_gemm_tc(const uint8_t* wq, const uint16_t* scales, const uint
                            const uint16_t* X, uint16_t* Y, int M, int K, int N,
                            cudaStream_t stream);
 
-cudaError_t read_and_clear_device_status(cudaStream_t stream, int* status);
+// Read-and-clear of the per-kernel-family device status words (1 = a bounded
+// wait ran out).
+cudaError_t read_and_clear_tc_status(int* v);
+cudaError_t read_and_clear_gemv_status(int* v);
+
+// Diagnostic: a kernel whose bounded wait must run out (see
+// w4a16_selftest_wait_timeout).
+cudaError_t launch_wait_timeout_selftest(long long limit_cycles, cudaStream_t stream);
 
 }  // namespace w4a16

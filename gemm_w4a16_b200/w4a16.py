@@ -21,7 +21,7 @@ GROUP = 128
 EXPORTED = (
     "w4a16_status_string", "w4a16_packed_sizes", "w4a16_pack", "w4a16_gemm",
     "w4a16_gemm_ex", "w4a16_select_path", "w4a16_dequant_debug",
-    "w4a16_device_status",
+    "w4a16_device_status", "w4a16_selftest_wait_timeout",
 )
 
 _lib = None
@@ -63,6 +63,8 @@ def lib():
             L.w4a16_dequant_debug.restype = _i
             L.w4a16_device_status.argtypes = [_vp, ctypes.POINTER(_i)]
             L.w4a16_device_status.restype = _i
+            L.w4a16_selftest_wait_timeout.argtypes = [ctypes.c_longlong, _vp]
+            L.w4a16_selftest_wait_timeout.restype = _i
             _lib = L
     return _lib
 
@@ -187,3 +189,9 @@ def device_status(stream=None) -> int:
     _check(lib().w4a16_device_status(_stream_ptr(stream), ctypes.byref(st)),
            "w4a16_device_status")
     return st.value
+
+
+def selftest_wait_timeout(limit_cycles: int = 2_000_000, stream=None) -> None:
+    """Launch the diagnostic kernel whose bounded wait must run out."""
+    _check(lib().w4a16_selftest_wait_timeout(int(limit_cycles), _stream_ptr(stream)),
+           "w4a16_selftest_wait_timeout")

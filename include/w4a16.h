@@ -136,6 +136,16 @@ W4A16_API w4a16_status w4a16_dequant_debug(const void* wq_packed, const void* sc
  */
 W4A16_API w4a16_status w4a16_device_status(void* stream, int* status);
 
+/*
+ * Diagnostic for the failure-detection path: launches one tiny kernel that
+ * waits on an mbarrier nothing ever completes, with a budget of limit_cycles
+ * SM clock cycles (0 .. 2^32).  The wait gives up, records a timeout in the
+ * device status word and the kernel returns normally, so the next
+ * w4a16_device_status reports W4A16_ERR_TIMEOUT and the CUDA context stays
+ * usable.  Returns W4A16_ERR_INVALID_ARG for a limit outside that range.
+ */
+W4A16_API w4a16_status w4a16_selftest_wait_timeout(long long limit_cycles, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

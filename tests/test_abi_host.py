@@ -96,6 +96,9 @@ def test_rejects_bad_arguments_without_launching(L):
     assert L.w4a16_packed_sizes(256, 256, 128, None, ctypes.byref(sz), ctypes.byref(sz)) == \
         w4a16.ERR_INVALID_ARG
     assert L.w4a16_device_status(null, None) == w4a16.ERR_INVALID_ARG
+    L.w4a16_selftest_wait_timeout.argtypes = [ctypes.c_longlong, ctypes.c_void_p]
+    assert L.w4a16_selftest_wait_timeout(-1, null) == w4a16.ERR_INVALID_ARG
+    assert L.w4a16_selftest_wait_timeout(1 << 40, null) == w4a16.ERR_INVALID_ARG
 
 
 def test_select_path_is_monotone_in_n(L):
