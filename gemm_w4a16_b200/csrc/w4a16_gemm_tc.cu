@@ -3,31 +3,35 @@
 // "PerfXLLM on Snapdragon 8 Gen2", section 3.3 item 1: with many tokens the
 // GEMM is compute bound; it gets its own tiling, with the operands staged in
 // shared memory to cut global traffic.  On sm_100a the tile is 128 weight
-// rows x BN tokens, K in stages of 64:
+// rows x BN tokens, K walked in slots of 128 (one quantisation group):
 //
-//   warp 4        producer: per stage one TMA tile of X (BN x 64 fp16, 128-byte
-//                 swizzle, rows past N zero-filled) and bulk copies of the
-//                 stage's packed codes (128 rows x 64 codes = 4 KB, contiguous
-//                 in the packed layout) and of its group's scales and zeros.
-//   warps 8..23   dequantisers: four groups of four warps take the stages in
-//                 turn (four stages in flight); one weight row per thread
-//                 (warp w serves TMEM lanes 32 (w % 4) ..), 64 codes; the exact
-//                 in-register dequant (the same one the GEMV uses) writes
-//                 fp16 W straight into tensor memory with tcgen05.st, where
-//                 it is the MMA's A operand -- W never round-trips through
-//                 shared memory, so shared-memory bandwidth is left to X.
-//   warp 5        MMA issuer: tcgen05.mma kind::f16 (A from TMEM, B = X from
-//                 shared memory, fp32 accumulator in TMEM), 4 MMAs of K = 16
-//                 per stage; tcgen05.commit releases the stage, the A slot
-//                 and, at the end of a tile, the accumulator.
-//   warps 0..3    epilogue: tcgen05.ld of the fp32 accumulator, one RNE
+//   warp 4        producer: X only.  One 3D TMA copy per X stage brings
+//                 kXSlabs slabs of 64 k x BN tokens (128-byte swizzle, the
+//                 K-major layout the MMA reads; rows past N and k past K are
+//                 zero-filled).  Copies are 16-64 KB: on B200 an SM's bulk
+//                 copy engine completes roughly one copy per several hundred
+//                 cycles whatever its size, so few large copies are what
+//                 keeps it ahead.
+//   warps 8..23   dequantisers: four groups of four warps take the K slots in
+//                 turn.  Thread = one weight row: it loads its row's 64 bytes
+//                 of codes (4 coalesced 16-byte loads, 512 contiguous bytes
+//                 per warp) and the group's scale and zero straight from
+//                 global memory, one slot ahead, dequantises exactly
+//                 (dequant_word) and writes the fp16 row slice into tensor
+//                 memory with tcgen05.st: the MMA's A operand never touches
+//                 shared memory.
+//   warp 5        MMA issuer: 8 x tcgen05.mma kind::f16 (M = 128, N = BN,
+//                 K = 16) per slot, A from TMEM, B = X from shared memory,
+//                 fp32 accumulator in TMEM; tcgen05.commit frees the A slot,
+//                 the X stage and, at the end of a tile, the accumulator.
+//   warps 0..3    epilogue: tcgen05.ld of the accumulator, one RNE
 //                 conversion to fp16, stores of Y[n][m].
 //
-// Persistent CTAs (one per SM) walk the tile list round-robin; accumulators
-// are double-buffered in TMEM when they fit so the epilogue of one tile
-// overlaps the main loop of the next.  Every mbarrier wait is bounded: on
-// expiry the kernel records a timeout in a device status word, stops issuing,
-// drains its copies and MMAs, frees TMEM and returns.
+// Persistent CTAs (one per SM) walk the tile list round-robin; the
+// accumulator is double-buffered in TMEM when two fit next to the A slots.
+// Every mbarrier wait is bounded: on expiry the kernel records a timeout in
+// a device status word, stops issuing, drains its copies and MMAs, frees
+// TMEM and returns.
 #include "w4a16_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -43,53 +47,44 @@ __device__ int g_tc_status = 0;
 namespace {
 
 constexpr int kBM = 128;
-constexpr int kBK = 64;
-// Warp roles: 0..3 epilogue (TMEM lane quadrants 0..3), 4 producer, 5 MMA
-// issuer and TMEM owner, 6..7 idle, 8.. dequantiser groups of 4 warps.
-constexpr int kDqGroups = 4;                     // stages dequantised concurrently
+constexpr int kSlotK = 128;                      // k per TMEM A slot (one group)
+constexpr int kAColsPerSlot = kSlotK / 2;        // fp16 pairs per 32-bit column
+constexpr int kDqGroups = 4;                     // dequantiser groups (slots in flight)
 constexpr int kFirstDqWarp = 8;
 constexpr int kThreads = (kFirstDqWarp + 4 * kDqGroups) * 32;
-constexpr int kWBytes = kBM * kBK / 2;       // packed codes of one stage
-constexpr int kSBytes = kBM * 2;             // scales of the stage's group
-constexpr int kZBytes = kBM / 2;             // zeros of the stage's group
-constexpr int kAColsPerSlot = kBK / 2;       // 64 fp16 = 32 columns
 
-__host__ __device__ constexpr int round_up(int a, int b) { return (a + b - 1) / b * b; }
+__host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
+__host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
 
 template <int BN>
 struct Cfg {
-  static constexpr int kXBytes = BN * kBK * 2;
-  static constexpr int kStageBytes = round_up(kXBytes + kWBytes + kSBytes + kZBytes, 1024);
-  // As many stages as fit in about 200 KB (a multiple of the dequantiser
-  // group count, at most 24): the ring is what keeps copies in flight.
-  static constexpr int kStagesFit = (200 * 1024 / kStageBytes) / kDqGroups * kDqGroups;
-  static constexpr int kStages = kStagesFit < 24 ? kStagesFit : 24;
+  // k per X stage: enough for a 16-64 KB copy, a multiple of the slot size.
+  static constexpr int kXK = cmax(kSlotK, cmin(512, (32768 / (BN * 2)) / kSlotK * kSlotK));
+  static constexpr int kXSlabs = kXK / 64;
+  static constexpr int kSlotsPerX = kXK / kSlotK;
+  static constexpr int kXStageBytes = BN * kXK * 2;
+  static constexpr int kXStages = cmin(8, (196 * 1024) / kXStageBytes);
   static constexpr int kAccBufs = (2 * BN + kDqGroups * kAColsPerSlot <= 512) ? 2 : 1;
   static constexpr int kACol0 = kAccBufs * BN;
-  // TMEM A slots (32 columns each): all the columns the accumulators leave,
-  // a multiple of the dequantiser group count, at most 12.  The slot ring is
-  // what lets dequantisation run ahead of MMA completion.
-  static constexpr int kASlotsFit = (512 - kACol0) / kAColsPerSlot / kDqGroups * kDqGroups;
-  static constexpr int kASlots = kASlotsFit < 12 ? kASlotsFit : 12;
+  static constexpr int kASlots = kDqGroups;
   static constexpr int kColsUsed = kACol0 + kASlots * kAColsPerSlot;
   static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
                                    : kColsUsed <= 256 ? 256 : 512;
-  static constexpr uint32_t kTx = kXBytes + kWBytes + kSBytes + kZBytes;
   static constexpr uint32_t kIdesc = ptx::idesc_f16_f32(kBM, BN);
-  // Shared memory: stages, then barriers and the TMEM address.  At least
-  // 120 KB is requested so that one CTA owns an SM (and all of its TMEM).
-  static constexpr int kBarBytes = 8 * (2 * kStages + 2 * kASlots + 2 * kAccBufs + 1) + 16;
-  static constexpr int kSmemUsed = kStages * kStageBytes + kBarBytes + 1024;
+  static constexpr int kBarBytes = 8 * (2 * kXStages + 2 * kASlots + 2 * kAccBufs + 1) + 16;
+  static constexpr int kSmemUsed = kXStages * kXStageBytes + kBarBytes + 1024;
+  // At least 120 KB so that one CTA owns an SM and all of its TMEM.
   static constexpr int kSmemBytes = kSmemUsed < 120 * 1024 ? 120 * 1024 : kSmemUsed;
-  static_assert(kStages >= kDqGroups && kStages % kDqGroups == 0, "stage ring");
-  static_assert(kASlots >= kDqGroups && kASlots % kDqGroups == 0, "TMEM A slot ring");
+  static_assert(kXStages >= 2, "X stage ring");
+  static_assert(kXSlabs <= 8, "TMA box depth");
   static_assert(kColsUsed <= 512, "TMEM overflow");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
+  static_assert((BN * 128) % 1024 == 0, "X slabs must stay 1024-byte aligned");
 };
 
 struct Shared {
-  uint64_t* full;
-  uint64_t* empty;
+  uint64_t* x_full;
+  uint64_t* x_empty;
   uint64_t* a_full;
   uint64_t* a_empty;
   uint64_t* acc_full;
@@ -97,6 +92,14 @@ struct Shared {
   uint64_t* drain;
   uint32_t* tmem_ptr;
   volatile int* abort_flag;
+};
+
+// Codes of one 128-k slot for one row (four 16-byte chunks) plus the group's
+// scale and zero, held in registers between the load and the dequantisation.
+struct SlotRegs {
+  uint4 v[4];
+  uint16_t s;
+  uint32_t z;
 };
 
 template <int BN>
@@ -108,11 +111,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kXStages * C::kXStageBytes);
   Shared sh;
-  sh.full = bars;
-  sh.empty = sh.full + C::kStages;
-  sh.a_full = sh.empty + C::kStages;
+  sh.x_full = bars;
+  sh.x_empty = sh.x_full + C::kXStages;
+  sh.a_full = sh.x_empty + C::kXStages;
   sh.a_empty = sh.a_full + C::kASlots;
   sh.acc_full = sh.a_empty + C::kASlots;
   sh.acc_empty = sh.acc_full + C::kAccBufs;
@@ -125,17 +128,19 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
   const int mt_n = ceil_div(M, kBM);
   const int nt_n = ceil_div(N, BN);
   const int tiles = mt_n * nt_n;
-  const int ks_n = K / kBK;
+  const int ks_n = K / kSlotK;                       // slots per tile
+  const int nx = ceil_div(ks_n, C::kSlotsPerX);      // X stages per tile
   const int kc_n = K / kChunkK;
   const int kg = K / kGroup;
+  const int my_tiles = (tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::kStages; ++i) {
-      ptx::mbar_init(&sh.full[i], 1);
-      ptx::mbar_init(&sh.empty[i], 4 + 1);     // 4 dequant warps + 1 MMA commit
+    for (int i = 0; i < C::kXStages; ++i) {
+      ptx::mbar_init(&sh.x_full[i], 1);
+      ptx::mbar_init(&sh.x_empty[i], 1);
     }
     for (int i = 0; i < C::kASlots; ++i) {
-      ptx::mbar_init(&sh.a_full[i], 4);
+      ptx::mbar_init(&sh.a_full[i], 4);            // the 4 warps of one dequantiser group
       ptx::mbar_init(&sh.a_empty[i], 1);
     }
     for (int i = 0; i < C::kAccBufs; ++i) {
@@ -159,38 +164,32 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
   if (warp == 4) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int s = 0;
-      uint32_t ph = 0;
+      int xs = 0;
+      uint32_t xph = 0;
       uint32_t issued_mask = 0, issued_par = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
-        const int mt = t % mt_n, nt = t / mt_n;
-        const uint8_t* wblk = wq + (size_t)mt * kc_n * kRowBlock * 16;
-        for (int ks = 0; ks < ks_n; ++ks) {
-          if (!wait_bar(&sh.empty[s], ph ^ 1, sh.abort_flag, &g_tc_status)) { ok = false; break; }
-          uint8_t* st = smem + s * C::kStageBytes;
-          ptx::mbar_arrive_expect_tx(&sh.full[s], C::kTx);
-          ptx::tma_load_2d(st, &tmap_x, &sh.full[s], ks * kBK, nt * BN);
-          ptx::bulk_load(st + C::kXBytes, wblk + (size_t)ks * 2 * kRowBlock * 16, kWBytes, &sh.full[s]);
-          const int g = ks / 2;
-          ptx::bulk_load(st + C::kXBytes + kWBytes, s_p + ((size_t)mt * kg + g) * kRowBlock, kSBytes,
-                         &sh.full[s]);
-          ptx::bulk_load(st + C::kXBytes + kWBytes + kSBytes,
-                         z_p + ((size_t)mt * kg + g) * (kRowBlock / 2), kZBytes, &sh.full[s]);
-          issued_mask |= 1u << s;
-          issued_par = (issued_par & ~(1u << s)) | (ph << s);
-          if (++s == C::kStages) { s = 0; ph ^= 1; }
+        const int nt = t / mt_n;
+        for (int xi = 0; xi < nx; ++xi) {
+          if (!wait_bar(&sh.x_empty[xs], xph ^ 1, sh.abort_flag, &g_tc_status)) { ok = false; break; }
+          ptx::mbar_arrive_expect_tx(&sh.x_full[xs], C::kXStageBytes);
+          ptx::tma_load_3d(smem + xs * C::kXStageBytes, &tmap_x, &sh.x_full[xs], 0, nt * BN,
+                           xi * C::kXSlabs);
+          issued_mask |= 1u << xs;
+          issued_par = (issued_par & ~(1u << xs)) | (xph << xs);
+          if (++xs == C::kXStages) { xs = 0; xph ^= 1; }
         }
       }
       // Drain: every copy issued into this CTA's shared memory has landed.
-      for (int i = 0; i < C::kStages; ++i)
-        if (issued_mask & (1u << i)) wait_bar(&sh.full[i], (issued_par >> i) & 1u, sh.abort_flag, &g_tc_status, false);
+      for (int i = 0; i < C::kXStages; ++i)
+        if (issued_mask & (1u << i))
+          wait_bar(&sh.x_full[i], (issued_par >> i) & 1u, sh.abort_flag, &g_tc_status, false);
     }
   } else if (warp == 5) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      int s = 0, a = 0, b = 0;
-      uint32_t ph = 0, aph = 0, bph = 0;
+      int xs = 0, a = 0, b = 0;
+      uint32_t xph = 0, aph = 0, bph = 0;
       bool ok = true;
       const uint32_t x_base = ptx::smem_addr(smem);
       for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
@@ -198,21 +197,24 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem + b * BN;
         for (int ks = 0; ks < ks_n; ++ks) {
-          if (!wait_bar(&sh.full[s], ph, sh.abort_flag, &g_tc_status) || !wait_bar(&sh.a_full[a], aph, sh.abort_flag, &g_tc_status)) {
-            ok = false;
-            break;
-          }
+          const int sub = ks % C::kSlotsPerX;
+          if (sub == 0 && !wait_bar(&sh.x_full[xs], xph, sh.abort_flag, &g_tc_status)) { ok = false; break; }
+          if (!wait_bar(&sh.a_full[a], aph, sh.abort_flag, &g_tc_status)) { ok = false; break; }
           ptx::tc_fence_after();
-          const uint32_t xs = x_base + s * C::kStageBytes;
+          const uint32_t xstage = x_base + xs * C::kXStageBytes;
 #pragma unroll
-          for (int j = 0; j < kBK / 16; ++j) {
-            ptx::mma_ts_f16(d_tmem, tmem + C::kACol0 + a * kAColsPerSlot + 8 * j,
-                            ptx::smem_desc_sw128(xs + 32 * j), C::kIdesc, (ks | j) != 0);
+          for (int j = 0; j < kSlotK / 16; ++j) {
+            const int slab = sub * 2 + (j >> 2);
+            const uint32_t baddr = xstage + slab * (BN * 128) + (j & 3) * 32;
+            ptx::mma_ts_f16(d_tmem, tmem + C::kACol0 + a * kAColsPerSlot + 8 * j, ptx::smem_desc_sw128(baddr),
+                            C::kIdesc, (ks | j) != 0);
           }
-          ptx::mma_commit(&sh.empty[s]);
           ptx::mma_commit(&sh.a_empty[a]);
-          if (++s == C::kStages) { s = 0; ph ^= 1; }
           if (++a == C::kASlots) { a = 0; aph ^= 1; }
+          if (sub == C::kSlotsPerX - 1 || ks == ks_n - 1) {
+            ptx::mma_commit(&sh.x_empty[xs]);
+            if (++xs == C::kXStages) { xs = 0; xph ^= 1; }
+          }
         }
         if (!ok) break;
         ptx::mma_commit(&sh.acc_full[b]);
@@ -224,45 +226,50 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
     }
   } else if (warp >= kFirstDqWarp) {
     // -------------------------------------------------------- dequantisers
-    // Group gi takes every kDqGroups-th stage of this CTA's sequence (so
-    // kDqGroups stages are in flight at once); stage i goes to TMEM A slot
-    // i % kASlots; each thread dequantises the 64 codes of one row.
+    // Group gi takes slots i = gi, gi + 4, ... of this CTA's sequence
+    // (tile-major, then k), slot i lives in TMEM A slot i % kASlots.
     const int gi = (warp - kFirstDqWarp) >> 2;
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t a_lane = tmem + ((uint32_t)(quad * 32) << 16) + C::kACol0;
-    const int my_tiles = (tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
-    const long long n_stages = (long long)my_tiles * ks_n;
-    for (long long i = gi; i < n_stages; i += kDqGroups) {
-      const int s = (int)(i % C::kStages);
-      const uint32_t ph = (uint32_t)((i / C::kStages) & 1);
+    const long long n_slots = (long long)my_tiles * ks_n;
+    auto load_slot = [&](long long i, SlotRegs& r) {
+      const int tl = (int)(i / ks_n);
+      const int g = (int)(i - (long long)tl * ks_n);
+      const int mt = (blockIdx.x + tl * gridDim.x) % mt_n;
+      const uint4* src = reinterpret_cast<const uint4*>(wq) + ((size_t)mt * kc_n + (size_t)g * 4) * kRowBlock + row;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) r.v[j] = ldg_stream_v4(src + j * kRowBlock);
+      r.s = __ldg(s_p + ((size_t)mt * kg + g) * kRowBlock + row);
+      r.z = __ldg(z_p + ((size_t)mt * kg + g) * (kRowBlock / 2) + (row >> 1));
+    };
+    SlotRegs cur, nxt;
+    if (gi < n_slots) load_slot(gi, cur);
+    for (long long i = gi; i < n_slots; i += kDqGroups) {
+      if (i + kDqGroups < n_slots) load_slot(i + kDqGroups, nxt);
       const int a = (int)(i % C::kASlots);
       const uint32_t aph = (uint32_t)((i / C::kASlots) & 1);
-      if (!wait_bar_warp(&sh.full[s], ph, sh.abort_flag, &g_tc_status)) break;
-      const uint8_t* st = smem + s * C::kStageBytes;
-      const uint4 v0 = *reinterpret_cast<const uint4*>(st + C::kXBytes + row * 16);
-      const uint4 v1 = *reinterpret_cast<const uint4*>(st + C::kXBytes + kRowBlock * 16 + row * 16);
-      const uint16_t sv = reinterpret_cast<const uint16_t*>(st + C::kXBytes + kWBytes)[row];
-      const uint32_t zb = st[C::kXBytes + kWBytes + kSBytes + (row >> 1)];
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&sh.empty[s]);
-      const GroupConsts gc = make_group_consts((zb >> ((row & 1) * 4)) & 0xFu, sv);
-      uint32_t h[32];
-      dequant_word(v0.x, gc, &h[0]);
-      dequant_word(v0.y, gc, &h[4]);
-      dequant_word(v0.z, gc, &h[8]);
-      dequant_word(v0.w, gc, &h[12]);
-      dequant_word(v1.x, gc, &h[16]);
-      dequant_word(v1.y, gc, &h[20]);
-      dequant_word(v1.z, gc, &h[24]);
-      dequant_word(v1.w, gc, &h[28]);
+      const GroupConsts gc = make_group_consts((cur.z >> ((row & 1) * 4)) & 0xFu, cur.s);
       if (!wait_bar_warp(&sh.a_empty[a], aph ^ 1, sh.abort_flag, &g_tc_status)) break;
       ptx::tc_fence_after();
-      ptx::tmem_st_x32(a_lane + a * kAColsPerSlot, h);
+#pragma unroll
+      for (int hlf = 0; hlf < 2; ++hlf) {
+        uint32_t h[32];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const uint4 v = cur.v[hlf * 2 + c];
+          dequant_word(v.x, gc, &h[c * 16 + 0]);
+          dequant_word(v.y, gc, &h[c * 16 + 4]);
+          dequant_word(v.z, gc, &h[c * 16 + 8]);
+          dequant_word(v.w, gc, &h[c * 16 + 12]);
+        }
+        ptx::tmem_st_x32(a_lane + a * kAColsPerSlot + hlf * 32, h);
+      }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&sh.a_full[a]);
+      cur = nxt;
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------ epilogue
@@ -320,15 +327,17 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// X [N][K] fp16, box 64 (K) x BN (rows), 128-byte swizzle, zero fill past N.
-cudaError_t make_x_map(CUtensorMap* map, const uint16_t* X, int N, int K, int BN) {
+// X [N][K] fp16 viewed as a 3D tensor (64 k, N rows, K/64 slabs): the box
+// (64, BN, slabs) lands as `slabs` K-major 128-byte-swizzled tiles of BN x 64,
+// the layout the MMA's B descriptor describes.  Zero fill past N and K.
+cudaError_t make_x_map(CUtensorMap* map, const uint16_t* X, int N, int K, int BN, int slabs) {
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
-  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)N};
-  cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-  cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)BN};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(X), dims, strides, box,
+  cuuint64_t dims[3] = {64, (cuuint64_t)N, (cuuint64_t)(K / 64)};
+  cuuint64_t strides[2] = {(cuuint64_t)K * 2, 128};
+  cuuint32_t box[3] = {64, (cuuint32_t)BN, (cuuint32_t)slabs};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<uint16_t*>(X), dims, strides, box,
                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
@@ -360,30 +369,13 @@ cudaError_t launch_bn(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p
     attr_set[dev] = true;
   }
   CUtensorMap map;
-  cudaError_t e = make_x_map(&map, X, N, K, BN);
+  cudaError_t e = make_x_map(&map, X, N, K, BN, C::kXSlabs);
   if (e != cudaSuccess) return e;
   const int tiles = ceil_div(M, kBM) * ceil_div(N, BN);
   const int grid = tiles < num_sms() ? tiles : num_sms();
   gemm_tc_kernel<BN><<<grid, kThreads, C::kSmemBytes, stream>>>(map, wq, s_p, z_p, Y, M, K, N);
   return cudaGetLastError();
 }
-
-}  // namespace
-
-// The CUDA-core GEMV wins below this many tokens (measured N sweep, fused
-// QKV shape); the tensor-core kernel from here on.
-int gemv_max_n() { return 1; }
-
-cudaError_t launch_gemm_tc(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros,
-                           const uint16_t* X, uint16_t* Y, int M, int K, int N, cudaStream_t stream) {
-  if (K % kBK) return cudaErrorNotSupported;
-  if (N <= 16) return launch_bn<16>(wq, scales, zeros, X, Y, M, K, N, stream);
-  if (N <= 32) return launch_bn<32>(wq, scales, zeros, X, Y, M, K, N, stream);
-  if (N <= 64) return launch_bn<64>(wq, scales, zeros, X, Y, M, K, N, stream);
-  return launch_bn<128>(wq, scales, zeros, X, Y, M, K, N, stream);
-}
-
-namespace {
 
 // One thread waits on an mbarrier whose phase nothing completes, with a short
 // cycle budget: the wait must give up, record the timeout and return.
@@ -399,6 +391,20 @@ __global__ void wait_timeout_selftest_kernel(long long limit) {
 }
 
 }  // namespace
+
+// The CUDA-core GEMV runs up to this many tokens (measured N sweep, fused QKV
+// shape); the tensor-core kernel from there on.
+int gemv_max_n() { return 1; }
+
+cudaError_t launch_gemm_tc(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros,
+                           const uint16_t* X, uint16_t* Y, int M, int K, int N, cudaStream_t stream) {
+  if (K % kSlotK) return cudaErrorNotSupported;
+  if (N <= 16) return launch_bn<16>(wq, scales, zeros, X, Y, M, K, N, stream);
+  if (N <= 32) return launch_bn<32>(wq, scales, zeros, X, Y, M, K, N, stream);
+  if (N <= 64) return launch_bn<64>(wq, scales, zeros, X, Y, M, K, N, stream);
+  if (N <= 128) return launch_bn<128>(wq, scales, zeros, X, Y, M, K, N, stream);
+  return launch_bn<256>(wq, scales, zeros, X, Y, M, K, N, stream);
+}
 
 cudaError_t launch_wait_timeout_selftest(long long limit_cycles, cudaStream_t stream) {
   wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(limit_cycles);
