@@ -38,6 +38,13 @@ LLAMA7B_LAYER = [("qkv", 12288, 4096), ("o", 4096, 4096), ("gate_up", 22016, 409
 N_LAYERS = 32
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one
+# gemv_kernel<1> launch on the fused QKV shape, from the ncu capture summarised
+# in profiles/gemv_kernel_qkv_m12288_k4096_n1.md, valid only while the kernel
+# source is unchanged (sha256 prefix of csrc/w4a16_gemv.cu).
+GEMV_TRAFFIC = {"src_sha256_prefix": "235f351f95cf46df", "qkv_dram_bytes": 26175232,
+                "qkv_alg_bytes": 26181632}
+
 
 def alg_bytes(M, K, N):
     """Algorithmic bytes of one call: int4 weights, 2.5 B/group metadata, X, Y."""
@@ -46,6 +53,22 @@ def alg_bytes(M, K, N):
 
 def alg_flops(M, K, N):
     return 2 * M * N * K
+
+
+def gemv_traffic_per_launch(alg_bytes_per_launch):
+    """ncu DRAM bytes per decode launch, scaled from the QKV capture by the
+    algorithmic bytes (every shape streams its weights once), or None when
+    the kernel source changed since the capture."""
+    import hashlib
+
+    src = os.path.join(ROOT, "gemm_w4a16_b200", "csrc", "w4a16_gemv.cu")
+    try:
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    if not h.startswith(GEMV_TRAFFIC["src_sha256_prefix"]):
+        return None
+    return GEMV_TRAFFIC["qkv_dram_bytes"] / GEMV_TRAFFIC["qkv_alg_bytes"] * alg_bytes_per_launch
 
 
 def load_peaks():
@@ -442,7 +465,8 @@ def main_ours(args):
         "roofline": {"bound": "hbm", "kernel": "gemv_kernel<1>", "achieved": achieved,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks_src,
-                     "traffic": args.traffic},
+                     "traffic": gemv_traffic_per_launch(step_bytes / len(calls)),
+                     "traffic_note": "bytes per launch, scaled from the QKV ncu capture"},
         "per_shape": per_shape,
         "e2e": {"value": e2e_value, "unit": "GB/s",
                 "h2d_bytes_per_step": int(x_flat.numel() * 2),
@@ -574,8 +598,6 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
-    ap.add_argument("--traffic", type=float, default=None,
-                    help="ncu DRAM bytes per launch of the dominant kernel, if captured")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -77,6 +77,26 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       :: "r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar)) : "memory");
 }
 
+// Hint: bring `bytes` (a multiple of 16, 16-byte aligned) of global memory
+// into L2.  Moves no data into the SM and returns nothing, so it is safe to
+// issue before the kernel has synchronised with its predecessor.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(src), "r"(bytes) : "memory");
+}
+
+// Programmatic dependent launch: wait until the preceding kernel in the
+// stream has completed and its memory operations are visible (returns at
+// once when the kernel was not launched as a dependent).
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Programmatic dependent launch: allow the next kernel in the stream to
+// begin launching (its own grid_dependency_wait still waits for this one).
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" :: "l"(tmap) : "memory");
 }

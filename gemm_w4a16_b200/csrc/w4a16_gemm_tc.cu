@@ -394,7 +394,7 @@ __global__ void wait_timeout_selftest_kernel(long long limit) {
 
 // The CUDA-core GEMV runs up to this many tokens (measured N sweep, fused QKV
 // shape); the tensor-core kernel from there on.
-int gemv_max_n() { return 1; }
+int gemv_max_n() { return 4; }
 
 cudaError_t launch_gemm_tc(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros,
                            const uint16_t* X, uint16_t* Y, int M, int K, int N, cudaStream_t stream) {

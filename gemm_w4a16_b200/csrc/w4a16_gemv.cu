@@ -7,18 +7,15 @@
 // dimensions of the weight (rows and K) for parallelism.  On sm_100a:
 //
 //  * a CTA owns one 128-row block of the packed weight and a range of whole
-//    groups along K; a producer warp streams the codes into a 4-stage
-//    shared-memory ring with bulk asynchronous copies of 16 KB (two groups,
-//    contiguous in the packed layout) -- on B200 each SM completes about one
-//    HBM-sourced bulk copy per ~650 cycles whatever its size, so copies must
-//    be large to reach HBM rate;
-//  * the scales and zeros of all the CTA's groups, and its slice of the
-//    activations, are staged once in shared memory (one copy each) and read
-//    back as broadcast loads;
-//  * two consumer warpgroups take the two groups of each stage; thread = one
-//    weight row; the exact in-register dequant (dequant_word, the same
-//    arithmetic as the definition's single fp16 rounding of (q - z) s)
-//    feeds fma.rn.f32.f16 into four independent fp32 chains per token;
+//    groups along K; a producer warp streams each group (8 KB of codes, 256 B
+//    of scales, 64 B of zeros, contiguous in the packed layout) into a
+//    6-stage shared-memory ring with bulk asynchronous copies, so tens of KB
+//    per CTA are in flight without holding registers;
+//  * the CTA's slice of the activations is staged once in shared memory and
+//    read back as broadcast 16-byte loads;
+//  * two consumer warpgroups take alternate groups; thread = one weight row;
+//    the exact in-register dequant (dequant_word) feeds fma.rn.f32.f16 into
+//    four independent fp32 chains per token;
 //  * split-K: the two warpgroups reduce through shared memory, and CTAs of a
 //    thread-block cluster (up to 8 along K) through distributed shared memory
 //    into the cluster's rank-0 CTA, in a fixed order (deterministic, no
@@ -35,16 +32,16 @@ __device__ int g_gemv_status = 0;
 
 namespace {
 
-constexpr int kGvHalves = 2;                          // consumer warpgroups
+constexpr int kGvHalves = 2;                          // consumer warpgroups (alternate groups)
 constexpr int kGvConsumerWarps = 4 * kGvHalves;
 constexpr int kGvProducerWarp = kGvConsumerWarps;
 constexpr int kGvThreads = (kGvConsumerWarps + 1) * 32;
-constexpr int kGvGroupBytes = 4 * kRowBlock * 16;     // codes of one group of 128 rows: 8 KB
-constexpr int kGvGroupsPerStage = kGvHalves;          // one group per consumer half
-constexpr int kGvStageBytes = kGvGroupsPerStage * kGvGroupBytes;   // 16 KB per bulk copy
-constexpr int kGvStages = 4;
+constexpr int kGvWBytes = 4 * kRowBlock * 16;         // one group of 128 rows: 8 KB
+constexpr int kGvStageBytes = kGvWBytes + kRowBlock * 2 + kRowBlock / 2;   // + scales + zeros
+constexpr int kGvStages = 6;                          // multiple of kGvHalves
 constexpr int kMaxCluster = 8;
-constexpr int kGvSmemLimit = 200 * 1024;
+constexpr int kMaxXSmem = 64 * 1024;                  // largest staged activation slice
+static_assert(kGvStages % kGvHalves == 0, "stage ring");
 
 __device__ __forceinline__ void fma_h2(float& acc, uint32_t w, uint32_t x) {
   asm("{\n\t.reg .f16 wl, wh, xl, xh;\n\t"
@@ -55,18 +52,13 @@ __device__ __forceinline__ void fma_h2(float& acc, uint32_t w, uint32_t x) {
       : "+f"(acc) : "r"(w), "r"(x));
 }
 
-// Shared memory of one CTA: the code ring, then (loaded once) the scales and
-// zeros of all the CTA's groups and its activation slice, then reduction
-// buffers and barriers.
 struct GvLayout {
-  int s_off, z_off, x_off, red_off, cred_off, bar_off, total;
+  int x_off, red_off, cred_off, bar_off, total;
 };
 
 __host__ __device__ inline GvLayout gv_layout(int nt, int gspan, int cl) {
   GvLayout L;
-  L.s_off = kGvStages * kGvStageBytes;
-  L.z_off = L.s_off + gspan * kRowBlock * 2;
-  L.x_off = L.z_off + gspan * (kRowBlock / 2);
+  L.x_off = kGvStages * kGvStageBytes;
   L.red_off = L.x_off + nt * gspan * kGroup * 2;
   L.cred_off = L.red_off + kGvHalves * nt * kRowBlock * 4;
   L.bar_off = L.cred_off + (cl > 1 ? cl * nt * kRowBlock * 4 : 0);
@@ -84,15 +76,13 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   const int kc_n = K / kChunkK;
   const int gspan = ceil_div(kg, cl);
   const GvLayout L = gv_layout(NT, gspan, cl);
-  const uint16_t* ss = reinterpret_cast<const uint16_t*>(smem + L.s_off);   // [group][128]
-  const uint8_t* zs = smem + L.z_off;                                        // [group][64]
-  const uint4* xs = reinterpret_cast<const uint4*>(smem + L.x_off);          // [NT][ng * 16]
+  uint4* xs = reinterpret_cast<uint4*>(smem + L.x_off);
   float* red = reinterpret_cast<float*>(smem + L.red_off);     // [halves][NT][128]
   float* cred = reinterpret_cast<float*>(smem + L.cred_off);   // [cl][NT][128], rank 0 only
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off);
   uint64_t* empty = full + kGvStages;
-  uint64_t* mbar = empty + kGvStages;                          // scales, zeros, activations
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(mbar + 1);
+  uint64_t* xbar = empty + kGvStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(xbar + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -100,14 +90,13 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   const int crank = blockIdx.x % cl;
   const int ga = (kg * crank) / cl, gb = (kg * (crank + 1)) / cl;
   const int ng = gb - ga;
-  const int n_stages = ceil_div(ng, kGvGroupsPerStage);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kGvStages; ++i) {
       ptx::mbar_init(&full[i], 1);
-      ptx::mbar_init(&empty[i], kGvConsumerWarps);
+      ptx::mbar_init(&empty[i], 4);              // the 4 warps of one consumer half
     }
-    ptx::mbar_init(mbar, 1);
+    ptx::mbar_init(xbar, 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -117,40 +106,38 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   float tot[NT];
   if (warp == kGvProducerWarp) {
     // ------------------------------------------------------------ producer
-    // Few, large copies: each stage is one 16 KB copy (two groups of codes,
-    // contiguous in the packed layout); scales, zeros and the activation
-    // slice of the whole CTA come in one copy each.
     if (lane == 0 && ng > 0) {
-      // Scales, zeros and activations first: every group needs them.
-      ptx::mbar_arrive_expect_tx(mbar, (uint32_t)(ng * (kRowBlock * 2 + kRowBlock / 2) + NT * ng * kGroup * 2));
-      ptx::bulk_load(smem + L.s_off, s_p + ((size_t)b * kg + ga) * kRowBlock, (uint32_t)(ng * kRowBlock * 2), mbar);
-      ptx::bulk_load(smem + L.z_off, z_p + ((size_t)b * kg + ga) * (kRowBlock / 2),
-                     (uint32_t)(ng * (kRowBlock / 2)), mbar);
+      ptx::mbar_arrive_expect_tx(xbar, (uint32_t)(NT * ng * kGroup * 2));
       for (int n = 0; n < NT; ++n)
-        ptx::bulk_load(smem + L.x_off + n * ng * kGroup * 2, X + (size_t)n * K + (size_t)ga * kGroup,
-                       (uint32_t)(ng * kGroup * 2), mbar);
-      const uint8_t* wblk = wq + (size_t)b * kc_n * kRowBlock * 16 + (size_t)ga * kGvGroupBytes;
+        ptx::bulk_load(reinterpret_cast<uint8_t*>(xs) + n * ng * kGroup * 2,
+                       X + (size_t)n * K + (size_t)ga * kGroup, (uint32_t)(ng * kGroup * 2), xbar);
+      const uint8_t* wblk = wq + (size_t)b * kc_n * kRowBlock * 16;
+      const uint16_t* sblk = s_p + (size_t)b * kg * kRowBlock;
+      const uint8_t* zblk = z_p + (size_t)b * kg * (kRowBlock / 2);
       int last = -1;
-      for (int i = 0; i < n_stages; ++i) {
+      for (int i = 0; i < ng; ++i) {
         const int st = i % kGvStages;
         const uint32_t ph = (uint32_t)((i / kGvStages) & 1);
         if (!wait_bar(&empty[st], ph ^ 1, abort_flag, &g_gemv_status)) break;
-        const int groups = min(kGvGroupsPerStage, ng - i * kGvGroupsPerStage);
-        ptx::mbar_arrive_expect_tx(&full[st], (uint32_t)(groups * kGvGroupBytes));
-        ptx::bulk_load(smem + st * kGvStageBytes, wblk + (size_t)i * kGvStageBytes,
-                       (uint32_t)(groups * kGvGroupBytes), &full[st]);
+        uint8_t* dst = smem + st * kGvStageBytes;
+        const int g = ga + i;
+        ptx::mbar_arrive_expect_tx(&full[st], kGvStageBytes);
+        ptx::bulk_load(dst, wblk + (size_t)g * kGvWBytes, kGvWBytes, &full[st]);
+        ptx::bulk_load(dst + kGvWBytes, sblk + (size_t)g * kRowBlock, kRowBlock * 2, &full[st]);
+        ptx::bulk_load(dst + kGvWBytes + kRowBlock * 2, zblk + (size_t)g * (kRowBlock / 2), kRowBlock / 2,
+                       &full[st]);
         last = i;
       }
       // Drain: every copy issued into this CTA's shared memory has landed.
       for (int i = (last - kGvStages + 1 > 0 ? last - kGvStages + 1 : 0); i <= last; ++i)
         wait_bar(&full[i % kGvStages], (uint32_t)((i / kGvStages) & 1), abort_flag, &g_gemv_status, false);
-      wait_bar(mbar, 0, abort_flag, &g_gemv_status, false);
+      wait_bar(xbar, 0, abort_flag, &g_gemv_status, false);
     }
     __syncwarp();
   } else {
     // ----------------------------------------------------------- consumers
-    // Thread = weight row r of block b; consumer half h takes group h of
-    // every stage; four independent fp32 chains per token.
+    // Thread = weight row r of block b; consumer half h takes groups
+    // i = h, h + 2, ...; four independent fp32 chains per token.
     const int h = warp >> 2;
     const int r = (warp & 3) * 32 + lane;
     float acc[NT][4];
@@ -158,42 +145,36 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
     for (int n = 0; n < NT; ++n)
 #pragma unroll
       for (int t = 0; t < 4; ++t) acc[n][t] = 0.f;
-    bool ok = ng == 0 || wait_bar_warp(mbar, 0, abort_flag, &g_gemv_status);
-    for (int i = 0; ok && i < n_stages; ++i) {
+    bool ok = ng == 0 || wait_bar_warp(xbar, 0, abort_flag, &g_gemv_status);
+    for (int i = h; ok && i < ng; i += kGvHalves) {
       const int st = i % kGvStages;
       const uint32_t ph = (uint32_t)((i / kGvStages) & 1);
       if (!wait_bar_warp(&full[st], ph, abort_flag, &g_gemv_status)) break;
-      const int gl = i * kGvGroupsPerStage + h;          // group index inside the CTA's range
-      if (gl < ng) {
-        const uint8_t* src = smem + st * kGvStageBytes + h * kGvGroupBytes;
-        uint4 v[4];
+      const uint8_t* src = smem + st * kGvStageBytes;
+      uint4 v[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const uint4*>(src + j * kRowBlock * 16 + r * 16);
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&empty[st]);
-        const uint16_t sv = ss[gl * kRowBlock + r];
-        const uint32_t zb = zs[gl * (kRowBlock / 2) + (r >> 1)];
-        const GroupConsts gc = make_group_consts((zb >> ((r & 1) * 4)) & 0xFu, sv);
+      for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const uint4*>(src + j * kRowBlock * 16 + r * 16);
+      const uint16_t sv = reinterpret_cast<const uint16_t*>(src + kGvWBytes)[r];
+      const uint32_t zb = src[kGvWBytes + kRowBlock * 2 + (r >> 1)];
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&empty[st]);
+      const GroupConsts gc = make_group_consts((zb >> ((r & 1) * 4)) & 0xFu, sv);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint32_t words[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t words[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            uint32_t hw[4];
-            dequant_word(words[t], gc, hw);
+        for (int t = 0; t < 4; ++t) {
+          uint32_t hw[4];
+          dequant_word(words[t], gc, hw);
 #pragma unroll
-            for (int n = 0; n < NT; ++n) {
-              const uint4 xv = xs[n * ng * (kGroup / 8) + gl * (kGroup / 8) + j * 4 + t];
-              fma_h2(acc[n][t], hw[0], xv.x);
-              fma_h2(acc[n][t], hw[1], xv.y);
-              fma_h2(acc[n][t], hw[2], xv.z);
-              fma_h2(acc[n][t], hw[3], xv.w);
-            }
+          for (int n = 0; n < NT; ++n) {
+            const uint4 xv = xs[n * ng * (kGroup / 8) + i * (kGroup / 8) + j * 4 + t];
+            fma_h2(acc[n][t], hw[0], xv.x);
+            fma_h2(acc[n][t], hw[1], xv.y);
+            fma_h2(acc[n][t], hw[2], xv.z);
+            fma_h2(acc[n][t], hw[3], xv.w);
           }
         }
-      } else {
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&empty[st]);
       }
     }
 #pragma unroll
@@ -266,7 +247,7 @@ cudaError_t launch_nt(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(gemv_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kGvSmemLimit);
+                                         200 * 1024);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
@@ -289,26 +270,16 @@ cudaError_t launch_nt(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p
 
 }  // namespace
 
-int gv_smem_bytes(int K, int cl, int nt) { return gv_layout(nt, ceil_div(K / kGroup, cl), cl).total; }
-
-// Cluster size along K.  HBM is the shared bottleneck, so the time is set by
-// the busiest SM: ceil(CTAs / SMs) CTAs of ceil(groups / cluster) groups each.
-// Pick the power-of-two cluster size (those pack evenly into GPCs) that
-// minimises that load; ties go to the smaller cluster (fewer, longer CTAs).
-// Each CTA keeps at least two groups and a shared-memory footprint that fits.
+// Cluster size along K: the smallest power of two that gives every SM at
+// least two CTAs, keeps two or more groups per CTA, and fits the staged
+// activation slice in shared memory.
 int gemv_cluster_size(int M, int K, int sms, int nt) {
   const int blocks = ceil_div(M, kRowBlock);
   const int kg = K / kGroup;
-  int best = 0;
-  long long best_load = 0;
-  for (int cl = 1; cl <= kMaxCluster; cl *= 2) {
-    if (gv_smem_bytes(K, cl, nt) > kGvSmemLimit) continue;
-    if (cl > 1 && kg / cl < 2) break;
-    const long long ctas = (long long)blocks * cl;
-    const long long load = ((ctas + sms - 1) / sms) * ceil_div(kg, cl);
-    if (best == 0 || load < best_load) { best = cl; best_load = load; }
-  }
-  return best > 0 ? best : kMaxCluster;
+  int cl = 1;
+  while (cl < kMaxCluster && blocks * cl < 2 * sms && kg / (2 * cl) >= 2) cl *= 2;
+  while (cl < kMaxCluster && nt * ceil_div(kg, cl) * kGroup * 2 > kMaxXSmem) cl *= 2;
+  return cl;
 }
 
 cudaError_t launch_gemv(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros,
@@ -317,7 +288,7 @@ cudaError_t launch_gemv(const uint8_t* wq, const uint16_t* scales, const uint8_t
   for (int n0 = 0; n0 < N; n0 += kGemvMaxTokens) {
     const int nt = std::min(kGemvMaxTokens, N - n0);
     const int cl = gemv_cluster_size(M, K, sm_count(), nt);
-    if (gv_smem_bytes(K, cl, nt) > kGvSmemLimit) return cudaErrorNotSupported;
+    if (nt * ceil_div(K / kGroup, cl) * kGroup * 2 > kMaxXSmem) return cudaErrorNotSupported;
     const uint16_t* Xn = X + (size_t)n0 * K;
     uint16_t* Yn = Y + (size_t)n0 * M;
     cudaError_t e;
