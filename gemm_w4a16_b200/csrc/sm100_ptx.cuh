@@ -41,6 +41,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking completion test of the phase with the given parity (acquire,
+// CTA scope).  Unlike try_wait it never suspends the thread.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile("{\n\t.reg .pred p;\n\t"
+               "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+               "selp.u32 %0, 1, 0, p;\n\t}"
+               : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+
 // As mbar_try_wait, but a thread whose phase is not complete is suspended in
 // hardware until the phase completes or about hint_ns nanoseconds pass, so
 // waiting warps do not take issue slots from the warps doing the work.
@@ -133,6 +144,31 @@ __device__ __forceinline__ void mma_ts_f16(uint32_t d_tmem, uint32_t a_tmem, uin
                :: "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
 }
 
+// The eight K = 16 MMAs of one 128-k slot issued back to back from one asm
+// block: A columns a[j] of TMEM, B descriptors b[j]; the first accumulates
+// only when acc_first != 0, the other seven always.  Issuing them together
+// keeps the compiler from interleaving per-MMA address arithmetic with the
+// issue, which on B200 roughly doubles the cost of each small-N MMA.
+__device__ __forceinline__ void mma_ts_f16_x8(uint32_t d_tmem, const uint32_t (&a)[8],
+                                              const uint64_t (&b)[8], uint32_t idesc,
+                                              uint32_t acc_first) {
+  asm volatile("{\n\t.reg .pred p, q;\n\t"
+               "setp.ne.b32 p, %18, 0;\n\t"
+               "setp.eq.b32 q, %17, %17;\n\t"
+               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %9, %17, p;\n\t"
+               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %10, %17, q;\n\t"
+               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %11, %17, q;\n\t"
+               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %12, %17, q;\n\t"
+               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%5], %13, %17, q;\n\t"
+               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%6], %14, %17, q;\n\t"
+               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%7], %15, %17, q;\n\t"
+               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%8], %16, %17, q;\n\t}"
+               :: "r"(d_tmem), "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]),
+                  "r"(a[6]), "r"(a[7]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "l"(b[4]),
+                  "l"(b[5]), "l"(b[6]), "l"(b[7]), "r"(idesc), "r"(acc_first)
+               : "memory");
+}
+
 // Arrive (once) on an mbarrier when every tcgen05 op this thread issued so
 // far has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
@@ -211,7 +247,7 @@ constexpr long long kWaitLimitCycles = 4000000000LL;
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                          int* status_word, bool honor_abort = true,
                                          long long limit = kWaitLimitCycles) {
-  if (ptx::mbar_try_wait(bar, parity)) return true;
+  if (ptx::mbar_test_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (ptx::mbar_try_wait_sleep(bar, parity, 200000u)) return true;

@@ -201,14 +201,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
           if (sub == 0 && !wait_bar(&sh.x_full[xs], xph, sh.abort_flag, &g_tc_status)) { ok = false; break; }
           if (!wait_bar(&sh.a_full[a], aph, sh.abort_flag, &g_tc_status)) { ok = false; break; }
           ptx::tc_fence_after();
-          const uint32_t xstage = x_base + xs * C::kXStageBytes;
+          const uint32_t xslab = x_base + xs * C::kXStageBytes + sub * 2 * (BN * 128);
+          const uint32_t acol = tmem + C::kACol0 + a * kAColsPerSlot;
+          uint32_t a_cols[8];
+          uint64_t b_desc[8];
 #pragma unroll
           for (int j = 0; j < kSlotK / 16; ++j) {
-            const int slab = sub * 2 + (j >> 2);
-            const uint32_t baddr = xstage + slab * (BN * 128) + (j & 3) * 32;
-            ptx::mma_ts_f16(d_tmem, tmem + C::kACol0 + a * kAColsPerSlot + 8 * j, ptx::smem_desc_sw128(baddr),
-                            C::kIdesc, (ks | j) != 0);
+            a_cols[j] = acol + 8 * j;
+            b_desc[j] = ptx::smem_desc_sw128(xslab + (j >> 2) * (BN * 128) + (j & 3) * 32);
           }
+          ptx::mma_ts_f16_x8(d_tmem, a_cols, b_desc, C::kIdesc, ks != 0);
           ptx::mma_commit(&sh.a_empty[a]);
           if (++a == C::kASlots) { a = 0; aph ^= 1; }
           if (sub == C::kSlotsPerX - 1 || ks == ks_n - 1) {
