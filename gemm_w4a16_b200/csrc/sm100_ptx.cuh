@@ -64,6 +64,21 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
   return ok != 0;
 }
 
+// ----------------------------------------------------------- shared memory
+
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+  uint4 r;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(addr) : "memory");
+  return r;
+}
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t r;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r) : "r"(addr) : "memory");
+  return r;
+}
+
 // ------------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, uint64_t* bar, int c0, int c1) {
@@ -167,6 +182,79 @@ __device__ __forceinline__ void mma_ts_f16_x8(uint32_t d_tmem, const uint32_t (&
                   "r"(a[6]), "r"(a[7]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "l"(b[4]),
                   "l"(b[5]), "l"(b[6]), "l"(b[7]), "r"(idesc), "r"(acc_first)
                : "memory");
+}
+
+// The four K = 16 MMAs of a 64-k slot, as mma_ts_f16_x8.
+__device__ __forceinline__ void mma_ts_f16_x4(uint32_t d_tmem, const uint32_t (&a)[4],
+                                              const uint64_t (&b)[4], uint32_t idesc,
+                                              uint32_t acc_first) {
+  asm volatile("{\n\t.reg .pred p, q;\n\t"
+               "setp.ne.b32 p, %10, 0;\n\t"
+               "setp.eq.b32 q, %9, %9;\n\t"
+               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %5, %9, p;\n\t"
+               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %6, %9, q;\n\t"
+               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %7, %9, q;\n\t"
+               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %8, %9, q;\n\t}"
+               :: "r"(d_tmem), "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "l"(b[0]), "l"(b[1]),
+                  "l"(b[2]), "l"(b[3]), "r"(idesc), "r"(acc_first)
+               : "memory");
+}
+
+__device__ __forceinline__ void mma_ts_f16_xn(uint32_t d, const uint32_t (&a)[4], const uint64_t (&b)[4],
+                                              uint32_t idesc, uint32_t acc_first) {
+  mma_ts_f16_x4(d, a, b, idesc, acc_first);
+}
+__device__ __forceinline__ void mma_ts_f16_xn(uint32_t d, const uint32_t (&a)[8], const uint64_t (&b)[8],
+                                              uint32_t idesc, uint32_t acc_first) {
+  mma_ts_f16_x8(d, a, b, idesc, acc_first);
+}
+
+// All MMAs of one A slot plus the commit that frees it, from one asm block:
+// MMA j (j < NMMA, 4 or 8) reads A columns a_col + 8 j and the B descriptor
+// desc + 2 j (+32 bytes in the 128-byte swizzled K-major row) for j < 4,
+// desc + slab16 + 2 (j - 4) past the first 64-k slab; the first MMA
+// accumulates only if acc_first != 0.  The commit then arrives on `bar`
+// once all of them have completed.
+template <int NMMA>
+__device__ __forceinline__ void mma_ts_f16_slot(uint32_t d_tmem, uint32_t a_col, uint64_t desc, uint32_t idesc,
+                                                uint32_t acc_first, uint64_t* bar, uint32_t slab16) {
+  static_assert(NMMA == 4 || NMMA == 8, "4 or 8 MMAs per slot");
+  if constexpr (NMMA == 4) {
+    asm volatile("{\n\t.reg .pred p, q;\n\t.reg .b32 a1, a2, a3;\n\t.reg .b64 b1, b2, b3;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "setp.eq.b32 q, %3, %3;\n\t"
+                 "add.u32 a1, %1, 8;\n\tadd.u32 a2, %1, 16;\n\tadd.u32 a3, %1, 24;\n\t"
+                 "add.s64 b1, %2, 2;\n\tadd.s64 b2, %2, 4;\n\tadd.s64 b3, %2, 6;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, q;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b2, %3, q;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], b3, %3, q;\n\t"
+                 "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%5];\n\t}"
+                 :: "r"(d_tmem), "r"(a_col), "l"(desc), "r"(idesc), "r"(acc_first), "r"(smem_addr(bar))
+                 : "memory");
+  } else {
+    const uint64_t desc2 = desc + slab16;
+    asm volatile("{\n\t.reg .pred p, q;\n\t.reg .b32 a1, a2, a3, a4, a5, a6, a7;\n\t"
+                 ".reg .b64 b1, b2, b3, b5, b6, b7;\n\t"
+                 "setp.ne.b32 p, %5, 0;\n\t"
+                 "setp.eq.b32 q, %4, %4;\n\t"
+                 "add.u32 a1, %1, 8;\n\tadd.u32 a2, %1, 16;\n\tadd.u32 a3, %1, 24;\n\t"
+                 "add.u32 a4, %1, 32;\n\tadd.u32 a5, %1, 40;\n\tadd.u32 a6, %1, 48;\n\tadd.u32 a7, %1, 56;\n\t"
+                 "add.s64 b1, %2, 2;\n\tadd.s64 b2, %2, 4;\n\tadd.s64 b3, %2, 6;\n\t"
+                 "add.s64 b5, %3, 2;\n\tadd.s64 b6, %3, 4;\n\tadd.s64 b7, %3, 6;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, p;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %4, q;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b2, %4, q;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], b3, %4, q;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [a4], %3, %4, q;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [a5], b5, %4, q;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [a6], b6, %4, q;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [a7], b7, %4, q;\n\t"
+                 "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%6];\n\t}"
+                 :: "r"(d_tmem), "r"(a_col), "l"(desc), "l"(desc2), "r"(idesc), "r"(acc_first),
+                    "r"(smem_addr(bar))
+                 : "memory");
+  }
 }
 
 // Arrive (once) on an mbarrier when every tcgen05 op this thread issued so
