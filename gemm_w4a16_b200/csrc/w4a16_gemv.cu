@@ -159,6 +159,8 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&empty[st]);
       const GroupConsts gc = make_group_consts((zb >> ((r & 1) * 4)) & 0xFu, sv);
+      // The group's activations: token n at xg + n * ng * 16, then fixed offsets.
+      const uint4* xg = xs + i * (kGroup / 8);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const uint32_t words[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
@@ -168,7 +170,7 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
           dequant_word(words[t], gc, hw);
 #pragma unroll
           for (int n = 0; n < NT; ++n) {
-            const uint4 xv = xs[n * ng * (kGroup / 8) + i * (kGroup / 8) + j * 4 + t];
+            const uint4 xv = xg[n * ng * (kGroup / 8) + j * 4 + t];
             fma_h2(acc[n][t], hw[0], xv.x);
             fma_h2(acc[n][t], hw[1], xv.y);
             fma_h2(acc[n][t], hw[2], xv.z);
@@ -270,16 +272,34 @@ cudaError_t launch_nt(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p
 
 }  // namespace
 
-// Cluster size along K: the smallest power of two that gives every SM at
-// least two CTAs, keeps two or more groups per CTA, and fits the staged
-// activation slice in shared memory.
+// Cluster size along K (1..8), from the measured LLaMA-7B N = 1 shapes:
+// all CTAs resident in one wave (kGvCtasPerSm per SM, set by the shared
+// memory of one CTA), and at least 2.5 CTAs per SM on average when the shape
+// allows it (fewer warps per SM hide the shared-memory and FMA latencies
+// badly); among those the smallest busiest-SM share of groups,
+// ceil(CTAs / SMs) x ceil(groups / cluster), then the smaller cluster.  When
+// no cluster reaches 2.5 CTAs per SM, the most CTAs.  The staged activation
+// slice must fit.
 int gemv_cluster_size(int M, int K, int sms, int nt) {
+  constexpr int kGvCtasPerSm = 4;
   const int blocks = ceil_div(M, kRowBlock);
   const int kg = K / kGroup;
-  int cl = 1;
-  while (cl < kMaxCluster && blocks * cl < 2 * sms && kg / (2 * cl) >= 2) cl *= 2;
-  while (cl < kMaxCluster && nt * ceil_div(kg, cl) * kGroup * 2 > kMaxXSmem) cl *= 2;
-  return cl;
+  int best = 0;
+  long long best_key[3] = {0, 0, 0};
+  for (int cl = 1; cl <= kMaxCluster && cl <= kg; ++cl) {
+    if (nt * ceil_div(kg, cl) * kGroup * 2 > kMaxXSmem) continue;
+    const long long ctas = (long long)blocks * cl;
+    if (cl > 1 && ctas > (long long)kGvCtasPerSm * sms) continue;
+    const bool dense = 2 * ctas >= 5LL * sms;
+    const long long load = (long long)ceil_div((int)ctas, sms) * ceil_div(kg, cl);
+    const long long key[3] = {dense ? 0 : 1, dense ? load : -ctas, cl};
+    if (best == 0 || key[0] < best_key[0] || (key[0] == best_key[0] && (key[1] < best_key[1] ||
+        (key[1] == best_key[1] && key[2] < best_key[2])))) {
+      best = cl;
+      for (int i = 0; i < 3; ++i) best_key[i] = key[i];
+    }
+  }
+  return best > 0 ? best : kMaxCluster;
 }
 
 cudaError_t launch_gemv(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros,
