@@ -74,7 +74,7 @@ struct Cfg {
   // k per TMEM A slot: half a quantisation group with few tokens (the
   // dequantiser groups then alternate between two slots each, see kASlots),
   // a whole group otherwise; fp16 pairs per 32-bit TMEM column.
-  static constexpr int kSlotK = BN <= 64 ? 64 : 128;
+  static constexpr int kSlotK = BN <= 128 ? 64 : 128;
   static constexpr int kAColsPerSlot = kSlotK / 2;
   static constexpr int kChunks = kSlotK / kChunkK;   // 16-byte chunks per row and slot
   static constexpr int kMmas = kSlotK / 16;          // K = 16 MMAs per slot
@@ -87,7 +87,7 @@ struct Cfg {
   // 4 B scale pair, 4 B zero quad).
   // With many tokens (compute bound) one slot of prefetch in registers is
   // enough and the shared memory goes to the X ring instead.
-  static constexpr bool kUseRing = BN <= 64;
+  static constexpr bool kUseRing = BN <= 128;
   static constexpr int kWDepth = kUseRing ? 6 : 0;
   static constexpr int kWCodeBytes = kDqGroups * kWDepth * kRowBlock * kChunks * 16;
   static constexpr int kWMetaBytes = kDqGroups * kWDepth * kRowBlock * 4;
@@ -97,8 +97,8 @@ struct Cfg {
   // A slots in TMEM: with few tokens the MMA of a slot takes about as long
   // as its dequantisation, so twice as many slots as dequantiser groups let
   // each group fill one slot while the MMAs read its other one.
-  static constexpr int kASlots = BN <= 64 ? 2 * kDqGroups : kDqGroups;
-  static constexpr int kIssuers = BN <= 64 ? 4 : 1;
+  static constexpr int kASlots = BN <= 128 ? 2 * kDqGroups : kDqGroups;
+  static constexpr int kIssuers = BN <= 64 ? 4 : BN <= 128 ? 2 : 1;
   static constexpr int kAccCols = kIssuers * BN;
   static constexpr int kAccBufs = (2 * kAccCols + kASlots * kAColsPerSlot <= 512) ? 2 : 1;
   static constexpr int kACol0 = kAccBufs * kAccCols;
