@@ -42,7 +42,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # gemv_kernel<1> launch on the fused QKV shape, from the ncu capture summarised
 # in profiles/gemv_kernel_qkv_m12288_k4096_n1.md, valid only while the kernel
 # source is unchanged (sha256 prefix of csrc/w4a16_gemv.cu).
-GEMV_TRAFFIC = {"src_sha256_prefix": "235f351f95cf46df", "qkv_dram_bytes": 26175232,
+GEMV_TRAFFIC = {"src_sha256_prefix": "6ce6410852d6b000", "qkv_dram_bytes": 26175488,
                 "qkv_alg_bytes": 26181632}
 
 
