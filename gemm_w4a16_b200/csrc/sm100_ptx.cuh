@@ -32,15 +32,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                :: "r"(smem_addr(bar)), "r"(bytes) : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile("{\n\t.reg .pred p;\n\t"
-               "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-               "selp.u32 %0, 1, 0, p;\n\t}"
-               : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
-  return ok != 0;
-}
-
 // Non-blocking completion test of the phase with the given parity (acquire,
 // CTA scope).  Unlike try_wait it never suspends the thread.
 __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
@@ -52,7 +43,7 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// As mbar_try_wait, but a thread whose phase is not complete is suspended in
+// mbarrier.try_wait with a time hint: a thread whose phase is not complete is suspended in
 // hardware until the phase completes or about hint_ns nanoseconds pass, so
 // waiting warps do not take issue slots from the warps doing the work.
 __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
@@ -81,13 +72,6 @@ __device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
 
 // ------------------------------------------------------------------- TMA
 
-__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, uint64_t* bar, int c0, int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];"
-      :: "r"(smem_addr(dst)), "l"(tmap), "r"(c0), "r"(c1), "r"(smem_addr(bar)) : "memory");
-}
-
 __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, uint64_t* bar, int c0, int c1, int c2) {
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
@@ -101,26 +85,6 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
       :: "r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar)) : "memory");
-}
-
-// Hint: bring `bytes` (a multiple of 16, 16-byte aligned) of global memory
-// into L2.  Moves no data into the SM and returns nothing, so it is safe to
-// issue before the kernel has synchronised with its predecessor.
-__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(src), "r"(bytes) : "memory");
-}
-
-// Programmatic dependent launch: wait until the preceding kernel in the
-// stream has completed and its memory operations are visible (returns at
-// once when the kernel was not launched as a dependent).
-__device__ __forceinline__ void grid_dependency_wait() {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-
-// Programmatic dependent launch: allow the next kernel in the stream to
-// begin launching (its own grid_dependency_wait still waits for this one).
-__device__ __forceinline__ void grid_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
@@ -148,65 +112,6 @@ __device__ __forceinline__ void tc_fence_before() {
 
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-// D[tmem] (+)= A[tmem] * B[smem desc], kind::f16, fp32 accumulate.
-__device__ __forceinline__ void mma_ts_f16(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                           uint32_t idesc, uint32_t accumulate) {
-  asm volatile("{\n\t.reg .pred p;\n\t"
-               "setp.ne.b32 p, %4, 0;\n\t"
-               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-               :: "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
-}
-
-// The eight K = 16 MMAs of one 128-k slot issued back to back from one asm
-// block: A columns a[j] of TMEM, B descriptors b[j]; the first accumulates
-// only when acc_first != 0, the other seven always.  Issuing them together
-// keeps the compiler from interleaving per-MMA address arithmetic with the
-// issue, which on B200 roughly doubles the cost of each small-N MMA.
-__device__ __forceinline__ void mma_ts_f16_x8(uint32_t d_tmem, const uint32_t (&a)[8],
-                                              const uint64_t (&b)[8], uint32_t idesc,
-                                              uint32_t acc_first) {
-  asm volatile("{\n\t.reg .pred p, q;\n\t"
-               "setp.ne.b32 p, %18, 0;\n\t"
-               "setp.eq.b32 q, %17, %17;\n\t"
-               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %9, %17, p;\n\t"
-               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %10, %17, q;\n\t"
-               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %11, %17, q;\n\t"
-               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %12, %17, q;\n\t"
-               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%5], %13, %17, q;\n\t"
-               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%6], %14, %17, q;\n\t"
-               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%7], %15, %17, q;\n\t"
-               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%8], %16, %17, q;\n\t}"
-               :: "r"(d_tmem), "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]),
-                  "r"(a[6]), "r"(a[7]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "l"(b[4]),
-                  "l"(b[5]), "l"(b[6]), "l"(b[7]), "r"(idesc), "r"(acc_first)
-               : "memory");
-}
-
-// The four K = 16 MMAs of a 64-k slot, as mma_ts_f16_x8.
-__device__ __forceinline__ void mma_ts_f16_x4(uint32_t d_tmem, const uint32_t (&a)[4],
-                                              const uint64_t (&b)[4], uint32_t idesc,
-                                              uint32_t acc_first) {
-  asm volatile("{\n\t.reg .pred p, q;\n\t"
-               "setp.ne.b32 p, %10, 0;\n\t"
-               "setp.eq.b32 q, %9, %9;\n\t"
-               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %5, %9, p;\n\t"
-               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %6, %9, q;\n\t"
-               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %7, %9, q;\n\t"
-               "tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %8, %9, q;\n\t}"
-               :: "r"(d_tmem), "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "l"(b[0]), "l"(b[1]),
-                  "l"(b[2]), "l"(b[3]), "r"(idesc), "r"(acc_first)
-               : "memory");
-}
-
-__device__ __forceinline__ void mma_ts_f16_xn(uint32_t d, const uint32_t (&a)[4], const uint64_t (&b)[4],
-                                              uint32_t idesc, uint32_t acc_first) {
-  mma_ts_f16_x4(d, a, b, idesc, acc_first);
-}
-__device__ __forceinline__ void mma_ts_f16_xn(uint32_t d, const uint32_t (&a)[8], const uint64_t (&b)[8],
-                                              uint32_t idesc, uint32_t acc_first) {
-  mma_ts_f16_x8(d, a, b, idesc, acc_first);
 }
 
 // All MMAs of one A slot plus the commit that frees it, from one asm block:
@@ -262,15 +167,6 @@ __device__ __forceinline__ void mma_ts_f16_slot(uint32_t d_tmem, uint32_t a_col,
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                :: "r"(smem_addr(bar)) : "memory");
-}
-
-// Each thread of the warp writes 16 consecutive 32-bit columns of its lane.
-__device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t (&v)[16]) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-               "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
-               :: "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]),
-                  "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]),
-                  "r"(v[13]), "r"(v[14]), "r"(v[15]) : "memory");
 }
 
 // Each thread of the warp writes 32 consecutive 32-bit columns of its lane.

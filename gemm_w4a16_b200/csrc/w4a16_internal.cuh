@@ -30,14 +30,6 @@ __device__ __forceinline__ uint4 ldg_stream_v4(const void* p) {
   return r;
 }
 
-// 16-byte read-only load that may stay in L1 (activations, shared by a warp).
-__device__ __forceinline__ uint4 ldg_ro_v4(const void* p) {
-  uint4 r;
-  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
-  return r;
-}
-
 __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t orv) {
   uint32_t d;
   // (a & b) | c  ->  immLut = (0xF0 & 0xCC) | 0xAA = 0xEA

@@ -49,9 +49,9 @@ typedef enum {
 
 /* Kernel selection for w4a16_gemm_ex. */
 typedef enum {
-    W4A16_PATH_AUTO = 0,     /* choose by N (the dispatcher) */
-    W4A16_PATH_GEMV = 1,     /* CUDA-core decode kernel (memory-bound, small N) */
-    W4A16_PATH_TC = 2        /* tcgen05 tensor-core kernel (large N) */
+    W4A16_PATH_AUTO = 0,     /* choose by N: GEMV for N <= 2, else tensor cores */
+    W4A16_PATH_GEMV = 1,     /* CUDA-core decode kernel (one or two tokens) */
+    W4A16_PATH_TC = 2        /* tcgen05 tensor-core kernel (three tokens and more) */
 } w4a16_path;
 
 /* Human-readable name of a status code.  Never returns NULL. */
