@@ -447,19 +447,31 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
       const int n0 = nt * BN;
       // Issuers that own no slot of this tile (K < kIssuers slots) wrote nothing.
       const int parts = ks_n < C::kIssuers ? ks_n : C::kIssuers;
+      // Drain the accumulator 16 columns at a time, software-pipelined: the
+      // issuer-0 part of chunk c + 1 is in flight while chunk c is converted
+      // and stored; the buffer is handed back to the MMA issuers as soon as
+      // its last columns are in registers.
+      const uint32_t acc0 = lane_base + b * C::kAccCols;
+      uint32_t nxt[16];
+      ptx::tmem_ld_x16(acc0, nxt);
 #pragma unroll 1
       for (int c = 0; c < BN / 16; ++c) {
-        uint32_t v[16];
-        float sum[16];
-        ptx::tmem_ld_x16(lane_base + b * C::kAccCols + 16 * c, v);
         ptx::tmem_wait_ld();
+        float sum[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) sum[j] = __uint_as_float(v[j]);
+        for (int j = 0; j < 16; ++j) sum[j] = __uint_as_float(nxt[j]);
+        if (c + 1 < BN / 16) ptx::tmem_ld_x16(acc0 + 16 * (c + 1), nxt);
         for (int p = 1; p < parts; ++p) {
-          ptx::tmem_ld_x16(lane_base + b * C::kAccCols + p * BN + 16 * c, v);
+          uint32_t v[16];
+          ptx::tmem_ld_x16(acc0 + p * BN + 16 * c, v);
           ptx::tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 16; ++j) sum[j] += __uint_as_float(v[j]);
+        }
+        if (c + 1 == BN / 16) {
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&sh.acc_empty[b]);
         }
         if (m < M) {
 #pragma unroll
@@ -469,9 +481,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
           }
         }
       }
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&sh.acc_empty[b]);
       if (++b == C::kAccBufs) { b = 0; bph ^= 1; }
     }
   }
