@@ -36,7 +36,9 @@
 //                 from the one two steps later).  tcgen05.commit frees
 //                 the A slot, the X stage (once every issuer is done with
 //                 it) and, at the end of a tile, the accumulators.
-//   warps 0..3    epilogue: tcgen05.ld of the issuers' accumulators, their
+//   warps 0..3    epilogue (and 24..27 at BN = 256, each of a lane quarter's
+//                 two warps taking half of the columns): tcgen05.ld of the
+//                 issuers' accumulators, their
 //                 sum in issuer order, one RNE conversion to fp16, stores of
 //                 Y[n][m].
 //
@@ -118,7 +120,12 @@ struct Cfg {
   // (768 threads, more registers each), else a warp of its own after the
   // dequantisers.
   static constexpr int kProducerWarp = kIssuers < 4 ? kFirstIssuerWarp + 3 : kLastDqWarp + 1;
-  static constexpr int kThreads = (kIssuers < 4 ? kLastDqWarp + 1 : kLastDqWarp + 2) * 32;
+  // Epilogue warps: 0..3, plus 4 more after the others at BN = 256, where the
+  // single accumulator keeps the tensor core idle while it is drained; each
+  // epilogue warp of a TMEM lane quarter then drains half of the columns.
+  static constexpr int kEpiWarps = BN == 256 ? 8 : 4;
+  static constexpr int kBaseWarps = kIssuers < 4 ? kLastDqWarp + 1 : kLastDqWarp + 2;
+  static constexpr int kThreads = (kBaseWarps + kEpiWarps - 4) * 32;
   // Parity waits see only the last phase's parity.  They stay exact when
   // every A slot has one consumer (kIssuers | kASlots) and the group
   // filling slot i, whose previous fill (slot i - kDqGroups) waited for the
@@ -199,7 +206,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
     }
     for (int i = 0; i < C::kAccBufs; ++i) {
       ptx::mbar_init(&sh.acc_full[i], C::kIssuers);
-      ptx::mbar_init(&sh.acc_empty[i], 4);
+      ptx::mbar_init(&sh.acc_empty[i], C::kEpiWarps);
     }
     ptx::mbar_init(sh.drain, C::kIssuers);
     *sh.abort_flag = 0;
@@ -432,11 +439,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
       // Nothing may still be writing this CTA's shared memory at exit.
       cp_async_wait<0>();
     }
-  } else if (warp < 4) {
+  } else if (warp < 4 || warp >= C::kBaseWarps) {
     // ------------------------------------------------------------ epilogue
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    // Columns of this warp: all, or one half when two warps share a quarter.
+    constexpr int kCols = BN * 4 / C::kEpiWarps;
+    const int col0 = warp < 4 ? 0 : kCols;
     int b = 0;
     uint32_t bph = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
@@ -444,23 +454,23 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
       if (!wait_bar_warp(&sh.acc_full[b], bph, sh.abort_flag, &g_tc_status)) break;
       ptx::tc_fence_after();
       const int m = mt * kBM + row;
-      const int n0 = nt * BN;
+      const int n0 = nt * BN + col0;
       // Issuers that own no slot of this tile (K < kIssuers slots) wrote nothing.
       const int parts = ks_n < C::kIssuers ? ks_n : C::kIssuers;
       // Drain the accumulator 16 columns at a time, software-pipelined: the
       // issuer-0 part of chunk c + 1 is in flight while chunk c is converted
       // and stored; the buffer is handed back to the MMA issuers as soon as
       // its last columns are in registers.
-      const uint32_t acc0 = lane_base + b * C::kAccCols;
+      const uint32_t acc0 = lane_base + b * C::kAccCols + col0;
       uint32_t nxt[16];
       ptx::tmem_ld_x16(acc0, nxt);
 #pragma unroll 1
-      for (int c = 0; c < BN / 16; ++c) {
+      for (int c = 0; c < kCols / 16; ++c) {
         ptx::tmem_wait_ld();
         float sum[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) sum[j] = __uint_as_float(nxt[j]);
-        if (c + 1 < BN / 16) ptx::tmem_ld_x16(acc0 + 16 * (c + 1), nxt);
+        if (c + 1 < kCols / 16) ptx::tmem_ld_x16(acc0 + 16 * (c + 1), nxt);
         for (int p = 1; p < parts; ++p) {
           uint32_t v[16];
           ptx::tmem_ld_x16(acc0 + p * BN + 16 * c, v);
@@ -468,7 +478,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
 #pragma unroll
           for (int j = 0; j < 16; ++j) sum[j] += __uint_as_float(v[j]);
         }
-        if (c + 1 == BN / 16) {
+        if (c + 1 == kCols / 16) {
           ptx::tc_fence_before();
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&sh.acc_empty[b]);
