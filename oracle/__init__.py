@@ -8,6 +8,10 @@ layer computes, in fp64, on the canonical (unpacked) arrays, written from
 * section 3.1 (low-precision quantisation): weight-only int4 quantisation,
   group_size 128, one scale and one zero per group.  Reading taken:
   w = fp16_RN((q - z) * s), the product exact, one rounding to fp16.
+* the step before it, the group quantiser fp16 W -> (q, s, z) (section 3.1
+  names int4, group 128, a scale and a zero, but no rounding rule): min-max
+  asymmetric with 0 inside the range, every decision in IEEE fp32 (see
+  ``quantize``).
 * section 3.3 item 1: C[m, n] = sum_k A[m, k] B[k, n] with A the weights and n
   the tokens; item 2: the GEMV is the n = 1 case.  Storage taken: x[n][k],
   y[n][m] (token-major), sums in fp64, ascending k.
@@ -61,6 +65,8 @@ def lib():
             L.w4o_gemm_rows.argtypes = [_u8p, _u8p, _u16p, _u16p, _i64, _i64,
                                         _i64, _i64, _i64p, _i64, _f64p]
             L.w4o_gemm_rows.restype = ctypes.c_int
+            L.w4o_quantize.argtypes = [_u16p, _i64, _i64, _i64, _u8p, _u16p, _u8p]
+            L.w4o_quantize.restype = ctypes.c_int
             _lib = L
     return _lib
 
@@ -151,3 +157,28 @@ def gemm_rows(q, zeros, scales, x, rows, group: int = 128) -> np.ndarray:
     if rc:
         raise RuntimeError(f"oracle gemm_rows failed ({rc})")
     return y
+
+
+def quantize(W, group: int = 128):
+    """Group quantiser: W fp16 bit patterns uint16 [M, K] -> (q uint8 [M, K],
+    scales fp16 bits uint16 [M, K/group], zeros uint8 [M, K/group]).
+
+    Per (row, group): lo = min(0, min w), hi = max(0, max w); r = hi - lo
+    raised to 2^-14; s = fp16_RN(r / 15); f = 1 / s; z = clamp(rint(-lo f),
+    0, 15); q = clamp(rint(w f) + z, 0, 15) -- each step one IEEE fp32
+    operation, round to nearest even (reading of "PerfXLLM on Snapdragon 8
+    Gen2", section 3.1, which fixes int4, group 128, scale and zero only)."""
+    W = _c(W, np.uint16)
+    if W.ndim != 2:
+        raise ValueError("W must be [M, K]")
+    M, K = W.shape
+    if group <= 0 or K % group:
+        raise ValueError("K must be a multiple of group")
+    q = np.empty((M, K), dtype=np.uint8)
+    scales = np.empty((M, K // group), dtype=np.uint16)
+    zeros = np.empty((M, K // group), dtype=np.uint8)
+    rc = lib().w4o_quantize(_ptr(W, _u16p), M, K, group, _ptr(q, _u8p), _ptr(scales, _u16p),
+                            _ptr(zeros, _u8p))
+    if rc:
+        raise RuntimeError(f"oracle quantize failed ({rc})")
+    return q, scales, zeros

@@ -211,3 +211,63 @@ int w4o_gemm_rows(const uint8_t* q, const uint8_t* zeros, const uint16_t* scales
 {
     return gemm_rows(q, zeros, scales, x, M, K, N, G, rows, nrows, y);
 }
+
+/* ------------------------------------------------------------ quantiser ---- */
+
+/*
+ * Group quantiser, fp16 W -> (q, s, z): the step before the layer's packing
+ * ("PerfXLLM on Snapdragon 8 Gen2", section 3.1: int4 weights, group_size
+ * 128, one scale and one zero per group).  The page names no rounding rule;
+ * reading taken: min-max asymmetric, with 0 always inside the range, every
+ * decision in IEEE fp32 (round to nearest even) so that a GPU can take the
+ * same decisions:
+ *
+ *   lo = min(0, min w), hi = max(0, max w) over the group (exact in fp32);
+ *   r  = hi - lo, raised to 2^-14 if smaller;
+ *   s  = fp16_RN(r / 15);            f = 1 / float(s);
+ *   z  = clamp(rint(-lo * f), 0, 15);
+ *   q  = clamp(rint(w * f) + z, 0, 15)   for each w of the group.
+ *
+ * Each line is one fp32 operation; this file is compiled without
+ * floating-point contraction.
+ */
+int w4o_quantize(const uint16_t* W, int64_t M, int64_t K, int64_t G,
+                 uint8_t* q, uint16_t* scales, uint8_t* zeros)
+{
+    if (check_shape(M, K, G)) return 1;
+    const int64_t kg = K / G;
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t g = 0; g < kg; ++g) {
+            const uint16_t* w = W + m * K + g * G;
+            float lo = 0.0f, hi = 0.0f;
+            for (int64_t i = 0; i < G; ++i) {
+                const float v = (float)w4o_fp16_to_double(w[i]);
+                if (v < lo) lo = v;
+                if (v > hi) hi = v;
+            }
+            float r = hi - lo;
+            const float r_min = 6.103515625e-05f;          /* 2^-14 */
+            if (!(r >= r_min)) r = r_min;
+            const float s32 = r / 15.0f;
+            const uint16_t s16 = w4o_fp16_from_double((double)s32);
+            const float f = 1.0f / (float)w4o_fp16_to_double(s16);
+            const float zneg = -lo;
+            const float zt = zneg * f;
+            float zf = rintf(zt);
+            if (zf < 0.0f) zf = 0.0f;
+            if (zf > 15.0f) zf = 15.0f;
+            for (int64_t i = 0; i < G; ++i) {
+                const float v = (float)w4o_fp16_to_double(w[i]);
+                const float t = v * f;
+                float qf = rintf(t) + zf;
+                if (qf < 0.0f) qf = 0.0f;
+                if (qf > 15.0f) qf = 15.0f;
+                q[m * K + g * G + i] = (uint8_t)qf;
+            }
+            scales[m * kg + g] = s16;
+            zeros[m * kg + g] = (uint8_t)zf;
+        }
+    }
+    return 0;
+}

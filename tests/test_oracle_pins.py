@@ -252,3 +252,88 @@ def test_synthetic_distributions():
     assert x[:, p.outliers].mean() > 10 * x[:, others].mean()
     again = synth.make_problem(M=512, K=4096, N=4, seed=0, outlier_frac=0.01)
     assert np.array_equal(again.q, p.q) and np.array_equal(again.x, p.x)
+
+
+# ------------------------------------------------------------ quantiser ----
+
+def _quantize_golden():
+    cases = []
+    for line in open(os.path.join(GOLDEN, "quantize_cases.txt")):
+        line = line.strip()
+        if not line.startswith("case "):
+            continue
+        f = dict(kv.split("=") for kv in line[5:].split())
+        runs = [(int(c), int(h, 16)) for c, h in (r.split("x") for r in f["runs"].split(","))]
+        codes = [int(v) for v in f["q"].split(",")]
+        cases.append((runs, codes, int(f["s"], 16), int(f["z"])))
+    return cases
+
+
+def test_quantize_hand_worked_cases():
+    """Hand-derived groups (tests/golden/quantize_cases.txt)."""
+    cases = _quantize_golden()
+    assert len(cases) == 4
+    for runs, codes, s, z in cases:
+        w = np.concatenate([np.full(c, h, dtype=np.uint16) for c, h in runs])[None, :]
+        q, sc, ze = oracle.quantize(w)
+        assert sc[0, 0] == s and ze[0, 0] == z
+        got = np.split(q[0], np.cumsum([c for c, _ in runs])[:-1])
+        for part, code in zip(got, codes):
+            assert np.all(part == code)
+
+
+@pytest.mark.parametrize("group", [64, 128])
+def test_quantize_recovers_values_on_its_grid(group):
+    """Weights already on a grid (k - z) s with s a power of two and both
+    k = 0 and k = 15 present: the quantiser returns exactly (k, s, z)."""
+    rng = np.random.default_rng(11)
+    M, K = 6, 4 * group
+    q0 = rng.integers(0, 16, size=(M, K)).astype(np.uint8)
+    q0[:, ::group] = 0
+    q0[:, 1::group] = 15
+    z0 = rng.integers(0, 16, size=(M, K // group)).astype(np.uint8)
+    e = rng.integers(-9, -2, size=(M, K // group))
+    s0 = np.ldexp(1.0, e)                                   # exact in fp16
+    zf = np.repeat(z0, group, axis=1).astype(np.float64)
+    sf = np.repeat(s0, group, axis=1)
+    w = ((q0.astype(np.float64) - zf) * sf).astype(np.float16).view(np.uint16)
+    q, s, z = oracle.quantize(w, group)
+    assert np.array_equal(q, q0)
+    assert np.array_equal(z, z0)
+    assert np.array_equal(oracle.fp16_to_double(s), s0)
+
+
+def test_quantize_error_bound_and_ranges():
+    """Codes and zeros stay in 0..15, and every weight is reproduced by
+    (q - z) s within half a step plus the scale's own fp16 rounding at the
+    range ends: |w - (q - z) s| <= s / 2 + |r - 15 s|."""
+    rng = np.random.default_rng(12)
+    M, K = 32, 1024
+    wd = rng.normal(0.0, 0.05, size=(M, K))
+    wd[:, ::7] = rng.normal(0.3, 0.1, size=(M, K // 7 + 1))[:, : wd[:, ::7].shape[1]]
+    w = wd.astype(np.float16).view(np.uint16)
+    q, s, z = oracle.quantize(w)
+    assert q.max() <= 15 and z.max() <= 15
+    wv = oracle.fp16_to_double(w).reshape(M, K // 128, 128)
+    sv = oracle.fp16_to_double(s)[..., None]
+    deq = (q.reshape(M, K // 128, 128).astype(np.float64) - z[..., None]) * sv
+    lo = np.minimum(wv.min(axis=2, keepdims=True), 0.0)
+    hi = np.maximum(wv.max(axis=2, keepdims=True), 0.0)
+    bound = 0.5 * sv + np.abs((hi - lo) - 15.0 * sv) + 1e-9
+    assert np.all(np.abs(deq - wv) <= bound)
+
+
+def test_quantize_sign_symmetry_and_scale_invariance():
+    """Negating a group mirrors its codes (q -> 15 - q with z -> 15 - z up to
+    ties), and multiplying it by a power of two scales s and keeps q, z."""
+    rng = np.random.default_rng(13)
+    w = rng.normal(0.0, 0.1, size=(4, 256)).astype(np.float16)
+    q, s, z = oracle.quantize(w.view(np.uint16))
+    q2, s2, z2 = oracle.quantize((w * np.float16(4)).view(np.uint16))
+    assert np.array_equal(q, q2) and np.array_equal(z, z2)
+    assert np.array_equal(oracle.fp16_to_double(s2), 4 * oracle.fp16_to_double(s))
+    qn, sn, zn = oracle.quantize((-w).view(np.uint16))
+    assert np.array_equal(sn, s)
+    deq = lambda qq, ss, zz: (qq.reshape(4, 2, 128).astype(np.float64) - zz[..., None]) * \
+        oracle.fp16_to_double(ss)[..., None]
+    assert np.allclose(deq(qn, sn, zn), -deq(q, s, z), atol=float(oracle.fp16_to_double(s).max()))
