@@ -387,6 +387,8 @@ def main_ours(args):
         return single_shape(args, device, 12288, 4096, 4096)
     if args.workload == "shape":
         return single_shape(args, device, args.M, args.K, args.N, args.path)
+    if args.workload == "quantize":
+        return quantize_workload(args, device, peaks)
 
     calls, x_flat, y_flat = build_decode_step(device, seed=1000 + rank)
     step_bytes = sum(alg_bytes(w.M, w.K, 1) for _, w, _, _ in calls)
@@ -520,6 +522,48 @@ def prefill_measure(device, peaks, args):
     return out
 
 
+def quantize_workload(args, device, peaks):
+    """Group quantiser fp16 W -> (q, s, z) on the four LLaMA-7B projection
+    shapes, 8 rotated weight copies per shape (beyond L2); HBM bytes per call:
+    2 read + 1 written per weight, plus 3 bytes of scale and zero per group."""
+    import torch
+
+    from gemm_w4a16_b200 import w4a16
+
+    for name, M, K in LLAMA7B_LAYER:
+        copies = [torch.randn((M, K), device=device, dtype=torch.float32).mul_(0.05).half()
+                  for _ in range(8)]
+        outs = [(torch.empty((M, K), dtype=torch.uint8, device=device),
+                 torch.empty((M, K // GROUP), dtype=torch.float16, device=device),
+                 torch.empty((M, K // GROUP), dtype=torch.uint8, device=device)) for _ in copies]
+        lib = w4a16.lib()
+        stream = torch.cuda.current_stream().cuda_stream
+
+        def one_pass():
+            for w, (q, s, z) in zip(copies, outs):
+                st = lib.w4a16_quantize(w.data_ptr(), M, K, GROUP, q.data_ptr(), s.data_ptr(), z.data_ptr(),
+                                        stream)
+                if st != 0:
+                    raise RuntimeError(f"w4a16_quantize failed ({st})")
+
+        for _ in range(args.warmup):
+            one_pass()
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            one_pass()
+        e1.record()
+        torch.cuda.synchronize(device)
+        us = e0.elapsed_time(e1) * 1e3 / (args.steps * len(copies))
+        nbytes = 3 * M * K + 3 * M * (K // GROUP)
+        gbps = nbytes / (us * 1e-6) / 1e9
+        print(json.dumps({"workload": f"quantize {name} M={M} K={K}", "us": us, "GBps": gbps,
+                          "frac_hbm": gbps / peaks["hbm_gbs"]}), flush=True)
+        del copies, outs
+    return 0
+
+
 def single_shape(args, device, M, K, N, path=0):
     """One shape, plain launches (used for ncu captures and quick timing)."""
     import torch
@@ -589,7 +633,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["decode", "qkv_n1", "prefill", "sweep", "shape"],
+    ap.add_argument("--workload", choices=["decode", "qkv_n1", "prefill", "sweep", "shape", "quantize"],
                     default="decode")
     ap.add_argument("--M", type=int, default=12288)
     ap.add_argument("--K", type=int, default=4096)

@@ -70,6 +70,16 @@ w4a16_status w4a16_packed_sizes(int M, int K, int group, size_t* wq_bytes,
   return W4A16_OK;
 }
 
+w4a16_status w4a16_quantize(const uint16_t* W, int M, int K, int group, uint8_t* q, uint16_t* scales,
+                            uint8_t* zeros, void* stream) {
+  if (!W || !q || !scales || !zeros) return W4A16_ERR_INVALID_ARG;
+  w4a16_status st = check_shape(M, K, group);
+  if (st != W4A16_OK) return st;
+  if (!aligned16(W) || !aligned16(q) || (reinterpret_cast<uintptr_t>(scales) & 1u))
+    return W4A16_ERR_MISALIGNED;
+  return map_cuda(launch_quantize(W, M, K, q, scales, zeros, static_cast<cudaStream_t>(stream)));
+}
+
 w4a16_status w4a16_pack(const uint8_t* q, const uint16_t* scales, const uint8_t* zeros,
                         int M, int K, int group, void* wq_packed, void* scales_packed,
                         void* zeros_packed, void* stream) {

@@ -108,6 +108,9 @@ cudaError_t launch_gemv(const uint8_t* wq, const uint16_t* scales, const uint8_t
                         const uint16_t* X, uint16_t* Y, int M, int K, int N,
                         cudaStream_t stream);
 
+cudaError_t launch_quantize(const uint16_t* W, int M, int K, uint8_t* q, uint16_t* scales, uint8_t* zeros,
+                            cudaStream_t stream);
+
 cudaError_t launch_pack(const uint8_t* q, const uint16_t* scales, const uint8_t* zeros,
                         int M, int K, uint8_t* wq_p, uint16_t* s_p, uint8_t* z_p,
                         cudaStream_t stream);

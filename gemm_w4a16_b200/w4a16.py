@@ -21,7 +21,7 @@ GROUP = 128
 EXPORTED = (
     "w4a16_status_string", "w4a16_packed_sizes", "w4a16_pack", "w4a16_gemm",
     "w4a16_gemm_ex", "w4a16_select_path", "w4a16_dequant_debug",
-    "w4a16_device_status", "w4a16_selftest_wait_timeout",
+    "w4a16_device_status", "w4a16_selftest_wait_timeout", "w4a16_quantize",
 )
 
 _lib = None
@@ -51,6 +51,8 @@ def lib():
             L.w4a16_status_string.restype = ctypes.c_char_p
             L.w4a16_packed_sizes.argtypes = [_i, _i, _i, _szp, _szp, _szp]
             L.w4a16_packed_sizes.restype = _i
+            L.w4a16_quantize.argtypes = [_vp, _i, _i, _i, _vp, _vp, _vp, _vp]
+            L.w4a16_quantize.restype = _i
             L.w4a16_pack.argtypes = [_vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp]
             L.w4a16_pack.restype = _i
             L.w4a16_gemm.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]
@@ -124,6 +126,22 @@ def empty_packed(M: int, K: int, device, group: int = GROUP) -> PackedWeight:
     a, b, c = packed_sizes(M, K, group)
     mk = lambda n: torch.empty(n, dtype=torch.uint8, device=device)
     return PackedWeight(mk(a), mk(b), mk(c), M, K, group)
+
+
+def quantize(W, group: int = GROUP, stream=None):
+    """fp16 W [M, K] (device) -> canonical (q uint8 [M, K], scales fp16
+    [M, K/G], zeros uint8 [M, K/G]) via w4a16_quantize."""
+    import torch
+
+    if W.dtype != torch.float16 or not W.is_cuda or not W.is_contiguous() or W.dim() != 2:
+        raise ValueError("W must be a contiguous CUDA fp16 [M, K] tensor")
+    M, K = W.shape
+    q = torch.empty((M, K), dtype=torch.uint8, device=W.device)
+    scales = torch.empty((M, K // group), dtype=torch.float16, device=W.device)
+    zeros = torch.empty((M, K // group), dtype=torch.uint8, device=W.device)
+    _check(lib().w4a16_quantize(_ptr(W), M, K, group, _ptr(q), _ptr(scales), _ptr(zeros),
+                                _stream_ptr(stream)), "w4a16_quantize")
+    return q, scales, zeros
 
 
 def pack(q, scales, zeros, group: int = GROUP, out: PackedWeight | None = None,

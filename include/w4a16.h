@@ -84,6 +84,24 @@ W4A16_API w4a16_status w4a16_packed_sizes(int M, int K, int group,
                                 size_t* zeros_bytes);
 
 /*
+ * Group quantiser: fp16 W -> canonical (q, scales, zeros), the step before
+ * w4a16_pack (offline).  "PerfXLLM on Snapdragon 8 Gen2", section 3.1 fixes
+ * 4-bit codes, groups of 128 along K and one scale and one zero per group;
+ * the rounding rule is min-max asymmetric with 0 inside the range, every step
+ * an IEEE fp32 operation (round to nearest even), per (row, group):
+ *     lo = min(0, min w), hi = max(0, max w), r = max(hi - lo, 2^-14),
+ *     s = fp16_RN(r / 15), f = 1 / s, z = clamp(rint(-lo f), 0, 15),
+ *     q = clamp(rint(w f) + z, 0, 15).
+ *   W       device fp16  [M][K], 16-byte aligned, finite values
+ *   q       device uint8 [M][K], 16-byte aligned (output)
+ *   scales  device fp16  [M][K/128], 2-byte aligned (output)
+ *   zeros   device uint8 [M][K/128] (output)
+ * W4A16_ERR_UNSUPPORTED for group != 128 or K % 128 != 0.
+ */
+W4A16_API w4a16_status w4a16_quantize(const uint16_t* W, int M, int K, int group,
+                            uint8_t* q, uint16_t* scales, uint8_t* zeros, void* stream);
+
+/*
  * Canonical -> packed layout (offline; not on the per-token path).
  *   q       device uint8  [M][K], values 0..15 (higher bits are ignored)
  *   scales  device fp16   [M][K/128]

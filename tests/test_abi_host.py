@@ -89,6 +89,12 @@ def test_rejects_bad_arguments_without_launching(L):
     assert L.w4a16_gemm(good, good, good, good, bad, 256, 256, 1, 128, null) == w4a16.ERR_MISALIGNED
     assert L.w4a16_dequant_debug(good, good, good, null, 256, 256, 128, null) == w4a16.ERR_INVALID_ARG
     assert L.w4a16_dequant_debug(good, good, good, bad, 256, 256, 128, null) == w4a16.ERR_MISALIGNED
+    assert L.w4a16_quantize(null, 256, 256, 128, good, good, good, null) == w4a16.ERR_INVALID_ARG
+    assert L.w4a16_quantize(good, 256, 200, 128, good, good, good, null) == w4a16.ERR_UNSUPPORTED
+    assert L.w4a16_quantize(good, 256, 256, 64, good, good, good, null) == w4a16.ERR_UNSUPPORTED
+    assert L.w4a16_quantize(good, 0, 256, 128, good, good, good, null) == w4a16.ERR_INVALID_ARG
+    assert L.w4a16_quantize(bad, 256, 256, 128, good, good, good, null) == w4a16.ERR_MISALIGNED
+    assert L.w4a16_quantize(good, 256, 256, 128, bad, good, good, null) == w4a16.ERR_MISALIGNED
     assert L.w4a16_pack(good, good, good, 256, 256, 100, good, good, good, null) == w4a16.ERR_UNSUPPORTED
     assert L.w4a16_pack(good, good, null, 256, 256, 128, good, good, good, null) == w4a16.ERR_INVALID_ARG
     assert L.w4a16_pack(good, good, good, 256, 256, 128, bad, good, good, null) == w4a16.ERR_MISALIGNED

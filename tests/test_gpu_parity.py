@@ -194,3 +194,48 @@ def test_prefill_with_outlier_channels(M, K, N):
 @pytest.mark.parametrize("M,K", LLAMA3)
 def test_llama3_batched_decode(M, K, N):
     sampled_case(M, K, N, w4a16.PATH_AUTO)
+
+
+# --------------------------------------------------------- group quantiser ----
+
+def _quantize_inputs(M, K, seed):
+    """fp16 weights ~ N(0, 0.05) with special groups: all zero, constant,
+    one-signed, a single large outlier."""
+    rng = np.random.default_rng(seed)
+    w = rng.normal(0.0, 0.05, size=(M, K))
+    if K >= 512 and M >= 4:
+        w[0, 0:128] = 0.0
+        w[1, 128:256] = 0.37
+        w[2, 256:384] = np.abs(w[2, 256:384]) + 0.01
+        w[3, 384:512] = -np.abs(w[3, 384:512])
+        w[M - 1, K - 7] = 6.5
+    return w.astype(np.float16)
+
+
+@pytest.mark.parametrize("M,K", [(256, 256), (200, 384), (1, 128), (37, 1024), (4096, 4096),
+                                 (12288, 4096)])
+def test_quantize_bit_exact(M, K):
+    """Codes, scales and zeros equal the oracle's bit for bit (same fp32
+    decisions on both sides)."""
+    w = _quantize_inputs(M, K, seed=M + K)
+    q_ref, s_ref, z_ref = oracle.quantize(w.view(np.uint16))
+    q, s, z = w4a16.quantize(torch.from_numpy(w).cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(s.cpu().numpy().view(np.uint16), s_ref)
+    assert np.array_equal(z.cpu().numpy(), z_ref)
+
+
+def test_quantize_pack_gemm_pipeline():
+    """fp16 W -> w4a16_quantize -> w4a16_pack -> w4a16_gemm against the oracle
+    layer on the oracle's own quantisation of the same W."""
+    M, K, N = 384, 1024, 5
+    w = _quantize_inputs(M, K, seed=21)
+    x = np.random.default_rng(22).normal(0, 1, size=(N, K)).astype(np.float16)
+    q, s, z = w4a16.quantize(torch.from_numpy(w).cuda())
+    packed = w4a16.pack(q, s, z)
+    for path in (w4a16.PATH_GEMV, w4a16.PATH_TC):
+        y = w4a16.gemm_ex(packed, torch.from_numpy(x).cuda(), path=path)
+        q_ref, s_ref, z_ref = oracle.quantize(w.view(np.uint16))
+        ref = oracle.gemm(q_ref, z_ref, s_ref, x.view(np.uint16))
+        assert_close(to_f64(y), ref, f"quantize+pack+gemm path={PATH_NAMES[path]}")
