@@ -389,6 +389,8 @@ def main_ours(args):
         return single_shape(args, device, args.M, args.K, args.N, args.path)
     if args.workload == "quantize":
         return quantize_workload(args, device, peaks)
+    if args.workload == "qkv_fused":
+        return qkv_fused_workload(args, device, peaks)
 
     calls, x_flat, y_flat = build_decode_step(device, seed=1000 + rank)
     step_bytes = sum(alg_bytes(w.M, w.K, 1) for _, w, _, _ in calls)
@@ -522,6 +524,59 @@ def prefill_measure(device, peaks, args):
     return out
 
 
+def qkv_fused_workload(args, device, peaks):
+    """Fused QKV projection of LLaMA-7B (3 x 4096 rows, K = 4096) at N = 1
+    (8 rotated weight copies, beyond L2) and N = 4096, three arms:
+      plain   w4a16_gemm into one [N][M] buffer (no split, no bias);
+      fused   w4a16_gemm_qkv writing Q, K, V separately with an fp16 bias;
+      unfused w4a16_gemm, then a torch add per projection for the split and
+              the bias (what a caller writes without the fused form; timing
+              comparator only).
+    Each arm is a CUDA graph timed twice, in the order plain, fused, unfused,
+    unfused, fused, plain, and reported as the mean of its two timings, so a
+    clock drift under the power cap falls on every arm alike."""
+    import torch
+
+    from gemm_w4a16_b200 import w4a16
+
+    M, K, splits = 12288, 4096, (4096, 4096, 4096)
+    bounds = [(0, 4096), (4096, 8192), (8192, 12288)]
+    for N, copies_n in ((1, 8), (4096, 1)):
+        problems = [make_device_problem(device, M, K, N, seed=50 + c) for c in range(copies_n)]
+        bias = torch.randn(M, device=device).half()
+        ys = [torch.empty((N, M), dtype=torch.float16, device=device) for _ in problems]
+        outs = [tuple(torch.empty((N, m), dtype=torch.float16, device=device) for m in splits)
+                for _ in problems]
+
+        def plain():
+            for (w, x), y in zip(problems, ys):
+                w4a16.gemm(w, x, Y=y)
+
+        def fused():
+            for (w, x), o in zip(problems, outs):
+                w4a16.gemm_qkv(w, x, splits, bias=bias, out=o)
+
+        def unfused():
+            for (w, x), y, o in zip(problems, ys, outs):
+                w4a16.gemm(w, x, Y=y)
+                for (c0, c1), oi in zip(bounds, o):
+                    torch.add(y[:, c0:c1], bias[c0:c1], out=oi)
+
+        arms = {"plain": plain, "fused_split_bias": fused, "unfused_gemm_then_torch_split_bias": unfused}
+        graphs = {name: capture(fn, device) for name, fn in arms.items()}
+        times = {name: [] for name in arms}
+        for name in list(arms) + list(reversed(list(arms))):
+            times[name].append(time_graph(graphs[name], args.steps, args.warmup, device) * 1e3 / copies_n)
+        for name in arms:
+            us = sum(times[name]) / len(times[name])
+            print(json.dumps({"workload": f"qkv {name} M={M} K={K} N={N}", "us": us,
+                              "us_each": times[name],
+                              "GBps": alg_bytes(M, K, N) / (us * 1e-6) / 1e9,
+                              "TFLOPS": alg_flops(M, K, N) / (us * 1e-6) / 1e12}), flush=True)
+        del graphs, problems, ys, outs
+    return 0
+
+
 def quantize_workload(args, device, peaks):
     """Group quantiser fp16 W -> (q, s, z) on the four LLaMA-7B projection
     shapes, 8 rotated weight copies per shape (beyond L2); HBM bytes per call:
@@ -633,7 +688,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["decode", "qkv_n1", "prefill", "sweep", "shape", "quantize"],
+    ap.add_argument("--workload", choices=["decode", "qkv_n1", "prefill", "sweep", "shape", "quantize",
+                                           "qkv_fused"],
                     default="decode")
     ap.add_argument("--M", type=int, default=12288)
     ap.add_argument("--K", type=int, default=4096)

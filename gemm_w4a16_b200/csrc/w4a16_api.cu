@@ -119,6 +119,36 @@ w4a16_status w4a16_gemm_ex(const void* wq_packed, const void* scales_packed,
   return map_cuda(e);
 }
 
+w4a16_status w4a16_gemm_qkv(const void* wq_packed, const void* scales_packed, const void* zeros_packed,
+                            const uint16_t* X, const uint16_t* bias, int Mq, int Mk, int Mv, int K, int N,
+                            int group, uint16_t* Yq, uint16_t* Yk, uint16_t* Yv, void* stream) {
+  if (!wq_packed || !scales_packed || !zeros_packed || !X || !Yq || !Yk || !Yv) return W4A16_ERR_INVALID_ARG;
+  if (Mq <= 0 || Mk <= 0 || Mv <= 0 || N <= 0) return W4A16_ERR_INVALID_ARG;
+  if ((long long)Mq + Mk + Mv > kMaxM) return W4A16_ERR_UNSUPPORTED;
+  const int M = Mq + Mk + Mv;
+  w4a16_status st = check_shape(M, K, group);
+  if (st != W4A16_OK) return st;
+  if (N > kMaxN) return W4A16_ERR_UNSUPPORTED;
+  if (!aligned16(wq_packed) || !aligned16(scales_packed) || !aligned16(zeros_packed) || !aligned16(X) ||
+      !aligned16(Yq) || !aligned16(Yk) || !aligned16(Yv) || (reinterpret_cast<uintptr_t>(bias) & 1u))
+    return W4A16_ERR_MISALIGNED;
+  OutMap om;
+  om.y0 = Yq;
+  om.y1 = Yk;
+  om.y2 = Yv;
+  om.end0 = Mq;
+  om.end1 = Mq + Mk;
+  om.bias = bias;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint8_t* wq = static_cast<const uint8_t*>(wq_packed);
+  const uint16_t* sp = static_cast<const uint16_t*>(scales_packed);
+  const uint8_t* zp = static_cast<const uint8_t*>(zeros_packed);
+  cudaError_t e = (select_path_impl(M, K, N) == W4A16_PATH_TC)
+                      ? launch_gemm_tc(wq, sp, zp, X, nullptr, M, K, N, s, &om)
+                      : launch_gemv(wq, sp, zp, X, nullptr, M, K, N, s, &om);
+  return map_cuda(e);
+}
+
 w4a16_status w4a16_gemm(const void* wq_packed, const void* scales_packed,
                         const void* zeros_packed, const uint16_t* X, uint16_t* Y,
                         int M, int K, int N, int group, void* stream) {

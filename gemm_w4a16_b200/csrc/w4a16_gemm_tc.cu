@@ -163,11 +163,11 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-template <int BN>
+template <int BN, bool kMap>
 __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __restrict__ wq,
                const uint16_t* __restrict__ s_p, const uint8_t* __restrict__ z_p,
-               uint16_t* __restrict__ Y, int M, int K, int N) {
+               uint16_t* __restrict__ Y, int M, int K, int N, OutMap om) {
   using C = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -451,10 +451,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
     uint32_t bph = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
       const int mt = t % mt_n, nt = t / mt_n;
-      if (!wait_bar_warp(&sh.acc_full[b], bph, sh.abort_flag, &g_tc_status)) break;
-      ptx::tc_fence_after();
       const int m = mt * kBM + row;
       const int n0 = nt * BN + col0;
+      // The fused form's destination and bias of this row, loaded before the
+      // wait so the load overlaps it.
+      RowDst dst = {};
+      if constexpr (kMap) {
+        if (m < M) dst = row_dst(om, M, m);
+      }
+      if (!wait_bar_warp(&sh.acc_full[b], bph, sh.abort_flag, &g_tc_status)) break;
+      ptx::tc_fence_after();
       // Issuers that own no slot of this tile (K < kIssuers slots) wrote nothing.
       const int parts = ks_n < C::kIssuers ? ks_n : C::kIssuers;
       // Drain the accumulator 16 columns at a time, software-pipelined: the
@@ -487,7 +493,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int n = n0 + 16 * c + j;
-            if (n < N) Y[(size_t)n * M + m] = __half_as_ushort(__float2half_rn(sum[j]));
+            if (n < N) {
+              if constexpr (kMap) store_row(dst, om.bias != nullptr, n, sum[j]);
+              else Y[(size_t)n * M + m] = __half_as_ushort(__float2half_rn(sum[j]));
+            }
           }
         }
       }
@@ -546,15 +555,15 @@ int num_sms() {
   return cached[dev];
 }
 
-template <int BN>
+template <int BN, bool kMap>
 cudaError_t launch_bn(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p, const uint16_t* X,
-                      uint16_t* Y, int M, int K, int N, cudaStream_t stream) {
+                      uint16_t* Y, int M, int K, int N, cudaStream_t stream, const OutMap& om) {
   using C = Cfg<BN>;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, kMap>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
@@ -564,7 +573,7 @@ cudaError_t launch_bn(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p
   if (e != cudaSuccess) return e;
   const int tiles = ceil_div(M, kBM) * ceil_div(N, BN);
   const int grid = tiles < num_sms() ? tiles : num_sms();
-  gemm_tc_kernel<BN><<<grid, C::kThreads, C::kSmemBytes, stream>>>(map, wq, s_p, z_p, Y, M, K, N);
+  gemm_tc_kernel<BN, kMap><<<grid, C::kThreads, C::kSmemBytes, stream>>>(map, wq, s_p, z_p, Y, M, K, N, om);
   return cudaGetLastError();
 }
 
@@ -587,14 +596,22 @@ __global__ void wait_timeout_selftest_kernel(long long limit) {
 // shape); the tensor-core kernel from there on.
 int gemv_max_n() { return 2; }
 
+template <bool kMap>
+cudaError_t launch_tc_map(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros, const uint16_t* X,
+                          uint16_t* Y, int M, int K, int N, cudaStream_t stream, const OutMap& om) {
+  if (N <= 16) return launch_bn<16, kMap>(wq, scales, zeros, X, Y, M, K, N, stream, om);
+  if (N <= 32) return launch_bn<32, kMap>(wq, scales, zeros, X, Y, M, K, N, stream, om);
+  if (N <= 64) return launch_bn<64, kMap>(wq, scales, zeros, X, Y, M, K, N, stream, om);
+  if (N <= 128) return launch_bn<128, kMap>(wq, scales, zeros, X, Y, M, K, N, stream, om);
+  return launch_bn<256, kMap>(wq, scales, zeros, X, Y, M, K, N, stream, om);
+}
+
 cudaError_t launch_gemm_tc(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros,
-                           const uint16_t* X, uint16_t* Y, int M, int K, int N, cudaStream_t stream) {
+                           const uint16_t* X, uint16_t* Y, int M, int K, int N, cudaStream_t stream,
+                           const OutMap* om) {
   if (K % kMaxSlotK) return cudaErrorNotSupported;
-  if (N <= 16) return launch_bn<16>(wq, scales, zeros, X, Y, M, K, N, stream);
-  if (N <= 32) return launch_bn<32>(wq, scales, zeros, X, Y, M, K, N, stream);
-  if (N <= 64) return launch_bn<64>(wq, scales, zeros, X, Y, M, K, N, stream);
-  if (N <= 128) return launch_bn<128>(wq, scales, zeros, X, Y, M, K, N, stream);
-  return launch_bn<256>(wq, scales, zeros, X, Y, M, K, N, stream);
+  if (om) return launch_tc_map<true>(wq, scales, zeros, X, nullptr, M, K, N, stream, *om);
+  return launch_tc_map<false>(wq, scales, zeros, X, Y, M, K, N, stream, OutMap{});
 }
 
 cudaError_t launch_wait_timeout_selftest(long long limit_cycles, cudaStream_t stream) {

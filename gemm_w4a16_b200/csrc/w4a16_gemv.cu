@@ -66,11 +66,11 @@ __host__ __device__ inline GvLayout gv_layout(int nt, int gspan, int cl) {
   return L;
 }
 
-template <int NT>
+template <int NT, bool kMap>
 __global__ void __launch_bounds__(kGvThreads)
 gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
             const uint8_t* __restrict__ z_p, const uint16_t* __restrict__ X,
-            uint16_t* __restrict__ Y, int M, int K, int cl) {
+            uint16_t* __restrict__ Y, int M, int K, int cl, OutMap om) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int kg = K / kGroup;
   const int kc_n = K / kChunkK;
@@ -186,6 +186,13 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   __syncthreads();
 
   const int r = threadIdx.x;   // rows for the reduction: threads 0..127
+  // The fused form's destination and bias of row m, loaded before the
+  // reductions so the load overlaps them.
+  RowDst dst = {};
+  if constexpr (kMap) {
+    const int m = b * kRowBlock + r;
+    if (r < kRowBlock && crank == 0 && m < M) dst = row_dst(om, M, m);
+  }
   if (r < kRowBlock) {
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
@@ -224,8 +231,13 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
 
   const int m = b * kRowBlock + r;
   if (m < M) {
+    if constexpr (kMap) {
 #pragma unroll
-    for (int n = 0; n < NT; ++n) Y[(size_t)n * M + m] = __half_as_ushort(__float2half_rn(tot[n]));
+      for (int n = 0; n < NT; ++n) store_row(dst, om.bias != nullptr, n, tot[n]);
+    } else {
+#pragma unroll
+      for (int n = 0; n < NT; ++n) Y[(size_t)n * M + m] = __half_as_ushort(__float2half_rn(tot[n]));
+    }
   }
 }
 
@@ -241,14 +253,14 @@ int sm_count() {
   return cached[dev];
 }
 
-template <int NT>
+template <int NT, bool kMap>
 cudaError_t launch_nt(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p, const uint16_t* X,
-                      uint16_t* Y, int M, int K, int cl, cudaStream_t stream) {
+                      uint16_t* Y, int M, int K, int cl, cudaStream_t stream, const OutMap& om) {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<NT, kMap>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          200 * 1024);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
@@ -267,7 +279,7 @@ cudaError_t launch_nt(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_kernel<NT>, wq, s_p, z_p, X, Y, M, K, cl);
+  return cudaLaunchKernelEx(&cfg, gemv_kernel<NT, kMap>, wq, s_p, z_p, X, Y, M, K, cl, om);
 }
 
 }  // namespace
@@ -304,19 +316,37 @@ int gemv_cluster_size(int M, int K, int sms, int nt) {
 
 cudaError_t launch_gemv(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros,
                         const uint16_t* X, uint16_t* Y, int M, int K, int N,
-                        cudaStream_t stream) {
+                        cudaStream_t stream, const OutMap* om) {
   for (int n0 = 0; n0 < N; n0 += kGemvMaxTokens) {
     const int nt = std::min(kGemvMaxTokens, N - n0);
     const int cl = gemv_cluster_size(M, K, sm_count(), nt);
     if (nt * ceil_div(K / kGroup, cl) * kGroup * 2 > kMaxXSmem) return cudaErrorNotSupported;
     const uint16_t* Xn = X + (size_t)n0 * K;
-    uint16_t* Yn = Y + (size_t)n0 * M;
+    uint16_t* Yn = om ? nullptr : Y + (size_t)n0 * M;
+    // The fused outputs of tokens n0 .. n0 + nt - 1: each segment moves by
+    // n0 of its own rows.
+    OutMap on = {};
+    if (om) {
+      on = *om;
+      on.y0 = om->y0 + (size_t)n0 * om->end0;
+      on.y1 = om->y1 + (size_t)n0 * (om->end1 - om->end0);
+      on.y2 = om->y2 + (size_t)n0 * (M - om->end1);
+    }
     cudaError_t e;
-    switch (nt) {
-      case 1: e = launch_nt<1>(wq, scales, zeros, Xn, Yn, M, K, cl, stream); break;
-      case 2: e = launch_nt<2>(wq, scales, zeros, Xn, Yn, M, K, cl, stream); break;
-      case 3: e = launch_nt<3>(wq, scales, zeros, Xn, Yn, M, K, cl, stream); break;
-      default: e = launch_nt<4>(wq, scales, zeros, Xn, Yn, M, K, cl, stream); break;
+    if (om) {
+      switch (nt) {
+        case 1: e = launch_nt<1, true>(wq, scales, zeros, Xn, Yn, M, K, cl, stream, on); break;
+        case 2: e = launch_nt<2, true>(wq, scales, zeros, Xn, Yn, M, K, cl, stream, on); break;
+        case 3: e = launch_nt<3, true>(wq, scales, zeros, Xn, Yn, M, K, cl, stream, on); break;
+        default: e = launch_nt<4, true>(wq, scales, zeros, Xn, Yn, M, K, cl, stream, on); break;
+      }
+    } else {
+      switch (nt) {
+        case 1: e = launch_nt<1, false>(wq, scales, zeros, Xn, Yn, M, K, cl, stream, on); break;
+        case 2: e = launch_nt<2, false>(wq, scales, zeros, Xn, Yn, M, K, cl, stream, on); break;
+        case 3: e = launch_nt<3, false>(wq, scales, zeros, Xn, Yn, M, K, cl, stream, on); break;
+        default: e = launch_nt<4, false>(wq, scales, zeros, Xn, Yn, M, K, cl, stream, on); break;
+      }
     }
     if (e != cudaSuccess) return e;
   }

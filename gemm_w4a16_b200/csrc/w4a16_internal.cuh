@@ -99,14 +99,61 @@ __device__ __forceinline__ uint32_t zero_code(const uint8_t* zblock, int r) {
   return (zblock[r >> 1] >> ((r & 1) * 4)) & 0xFu;
 }
 
+// --------------------------------------------------------- output map ----
+
+// Where an epilogue puts row m of the result when the caller asked for the
+// fused form (w4a16_gemm_qkv): rows [0, end0), [end0, end1) and [end1, M) go
+// to three token-major outputs of their own widths, each value after adding
+// an optional fp16 bias of its row in fp32 and one RNE rounding to fp16.
+struct OutMap {
+  uint16_t* y0;
+  uint16_t* y1;
+  uint16_t* y2;
+  int end0, end1;
+  const uint16_t* bias;   // [M] or null
+};
+
+// Row m's destination in the fused form, resolved once per row: its element
+// in token 0 of the output it belongs to, that output's row pitch (its
+// width) and the fp32 value of its bias (0 when there is none).
+struct RowDst {
+  uint16_t* y;
+  int ld;
+  float bias;
+};
+
+__device__ __forceinline__ RowDst row_dst(const OutMap& o, int M, int m) {
+  RowDst d;
+  if (m < o.end0) {
+    d.y = o.y0 + m;
+    d.ld = o.end0;
+  } else if (m < o.end1) {
+    d.y = o.y1 + (m - o.end0);
+    d.ld = o.end1 - o.end0;
+  } else {
+    d.y = o.y2 + (m - o.end1);
+    d.ld = M - o.end1;
+  }
+  d.bias = o.bias ? __half2float(__ushort_as_half(o.bias[m])) : 0.0f;
+  return d;
+}
+
+// Token n of row d: the accumulator plus the bias in fp32 (skipped without a
+// bias, so a zero result keeps its sign), rounded once to fp16.
+__device__ __forceinline__ void store_row(const RowDst& d, bool has_bias, int n, float v) {
+  if (has_bias) v = __fadd_rn(v, d.bias);
+  d.y[(size_t)n * d.ld] = __half_as_ushort(__float2half_rn(v));
+}
+
 // ------------------------------------------------------- launch helpers ----
 
 // GEMV (CUDA cores): N in 1..kGemvMaxTokens per launch.
 constexpr int kGemvMaxTokens = 4;
 
+// om: null for the plain [N][M] output Y, else the fused output map (Y unused).
 cudaError_t launch_gemv(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros,
                         const uint16_t* X, uint16_t* Y, int M, int K, int N,
-                        cudaStream_t stream);
+                        cudaStream_t stream, const OutMap* om = nullptr);
 
 cudaError_t launch_quantize(const uint16_t* W, int M, int K, uint8_t* q, uint16_t* scales, uint8_t* zeros,
                             cudaStream_t stream);
@@ -122,7 +169,7 @@ cudaError_t launch_dequant(const uint8_t* wq, const uint16_t* scales, const uint
 // what the kernel handles.
 cudaError_t launch_gemm_tc(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros,
                            const uint16_t* X, uint16_t* Y, int M, int K, int N,
-                           cudaStream_t stream);
+                           cudaStream_t stream, const OutMap* om = nullptr);
 
 // Read-and-clear of the per-kernel-family device status words (1 = a bounded
 // wait ran out).

@@ -21,7 +21,7 @@ GROUP = 128
 EXPORTED = (
     "w4a16_status_string", "w4a16_packed_sizes", "w4a16_pack", "w4a16_gemm",
     "w4a16_gemm_ex", "w4a16_select_path", "w4a16_dequant_debug",
-    "w4a16_device_status", "w4a16_selftest_wait_timeout", "w4a16_quantize",
+    "w4a16_device_status", "w4a16_selftest_wait_timeout", "w4a16_quantize", "w4a16_gemm_qkv",
 )
 
 _lib = None
@@ -57,6 +57,8 @@ def lib():
             L.w4a16_pack.restype = _i
             L.w4a16_gemm.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]
             L.w4a16_gemm.restype = _i
+            L.w4a16_gemm_qkv.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp]
+            L.w4a16_gemm_qkv.restype = _i
             L.w4a16_gemm_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
             L.w4a16_gemm_ex.restype = _i
             L.w4a16_select_path.argtypes = [_i, _i, _i]
@@ -173,6 +175,34 @@ def gemm_ex(w: PackedWeight, X, Y=None, path: int = PATH_AUTO, stream=None):
                                _ptr(Y), w.M, K, N, w.group, path, _stream_ptr(stream)),
            "w4a16_gemm_ex")
     return Y
+
+
+def gemm_qkv(w: PackedWeight, X, splits, bias=None, out=None, stream=None):
+    """(Yq, Yk, Yv) token-major fp16 for a weight whose rows are three stacked
+    projections of widths splits = (Mq, Mk, Mv), each row plus bias[m] (fp16
+    [M] or None), via w4a16_gemm_qkv.  out: three contiguous CUDA fp16 tensors
+    [N, Mq], [N, Mk], [N, Mv] to write, or None to allocate them."""
+    import torch
+
+    N, K = X.shape
+    Mq, Mk, Mv = (int(v) for v in splits)
+    if Mq + Mk + Mv != w.M:
+        raise ValueError("splits must add up to the weight's rows")
+    if K != w.K or X.dtype != torch.float16 or not X.is_cuda or not X.is_contiguous():
+        raise ValueError("X must be a contiguous CUDA fp16 [N, K] tensor")
+    if bias is not None and (bias.dtype != torch.float16 or not bias.is_cuda or bias.numel() != w.M):
+        raise ValueError("bias must be a CUDA fp16 tensor of M values")
+    if out is None:
+        outs = [torch.empty((N, m), dtype=torch.float16, device=X.device) for m in (Mq, Mk, Mv)]
+    else:
+        outs = list(out)
+        if len(outs) != 3 or any(o.dtype != torch.float16 or not o.is_cuda or not o.is_contiguous()
+                                 or tuple(o.shape) != (N, m) for o, m in zip(outs, (Mq, Mk, Mv))):
+            raise ValueError("out must be three contiguous CUDA fp16 tensors [N, Mq], [N, Mk], [N, Mv]")
+    _check(lib().w4a16_gemm_qkv(_ptr(w.wq), _ptr(w.scales), _ptr(w.zeros), _ptr(X), _ptr(bias), Mq, Mk, Mv,
+                                K, N, w.group, _ptr(outs[0]), _ptr(outs[1]), _ptr(outs[2]),
+                                _stream_ptr(stream)), "w4a16_gemm_qkv")
+    return tuple(outs)
 
 
 def gemm(w: PackedWeight, X, Y=None, stream=None):

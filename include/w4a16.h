@@ -127,6 +127,25 @@ W4A16_API w4a16_status w4a16_gemm(const void* wq_packed, const void* scales_pack
                         const void* zeros_packed, const uint16_t* X, uint16_t* Y,
                         int M, int K, int N, int group, void* stream);
 
+/*
+ * The fused-projection form ("PerfXLLM on Snapdragon 8 Gen2", section 3.2:
+ * operator fusion removes intermediate reads and writes, and the three
+ * matrix products that make Q, K and V become one larger product).  The
+ * weight's rows are three projections stacked, M = Mq + Mk + Mv; the result
+ * goes straight to three token-major outputs instead of one [N][M] buffer:
+ *     Yq[n][m]      = fp16_RN(acc[n][m]           + bias[m])           m < Mq
+ *     Yk[n][m]      = fp16_RN(acc[n][Mq + m]      + bias[Mq + m])      m < Mk
+ *     Yv[n][m]      = fp16_RN(acc[n][Mq + Mk + m] + bias[Mq + Mk + m]) m < Mv
+ * with acc the fp32 accumulator of w4a16_gemm and the bias added in fp32
+ * (bias device fp16 [M], or NULL for none).  Mq, Mk, Mv >= 1; other
+ * arguments, alignment (Yq, Yk, Yv 16-byte aligned) and kernel choice as
+ * w4a16_gemm.
+ */
+W4A16_API w4a16_status w4a16_gemm_qkv(const void* wq_packed, const void* scales_packed,
+                            const void* zeros_packed, const uint16_t* X, const uint16_t* bias,
+                            int Mq, int Mk, int Mv, int K, int N, int group,
+                            uint16_t* Yq, uint16_t* Yk, uint16_t* Yv, void* stream);
+
 /* As w4a16_gemm, with the kernel forced (w4a16_path).  W4A16_PATH_AUTO is the
  * same as w4a16_gemm.  Used by tests and the benchmark to time both paths. */
 W4A16_API w4a16_status w4a16_gemm_ex(const void* wq_packed, const void* scales_packed,

@@ -89,6 +89,17 @@ def test_rejects_bad_arguments_without_launching(L):
     assert L.w4a16_gemm(good, good, good, good, bad, 256, 256, 1, 128, null) == w4a16.ERR_MISALIGNED
     assert L.w4a16_dequant_debug(good, good, good, null, 256, 256, 128, null) == w4a16.ERR_INVALID_ARG
     assert L.w4a16_dequant_debug(good, good, good, bad, 256, 256, 128, null) == w4a16.ERR_MISALIGNED
+    q3 = L.w4a16_gemm_qkv
+    assert q3(good, good, good, good, null, 128, 64, 64, 256, 1, 128, good, null, good, null) == \
+        w4a16.ERR_INVALID_ARG
+    assert q3(good, good, good, good, null, 0, 64, 64, 256, 1, 128, good, good, good, null) == \
+        w4a16.ERR_INVALID_ARG
+    assert q3(good, good, good, good, null, 128, 64, 64, 200, 1, 128, good, good, good, null) == \
+        w4a16.ERR_UNSUPPORTED
+    assert q3(good, good, good, good, null, 128, 64, 64, 256, 1, 128, good, bad, good, null) == \
+        w4a16.ERR_MISALIGNED
+    assert q3(good, good, good, good, ctypes.c_void_p(0x10001), 128, 64, 64, 256, 1, 128, good, good, good,
+              null) == w4a16.ERR_MISALIGNED
     assert L.w4a16_quantize(null, 256, 256, 128, good, good, good, null) == w4a16.ERR_INVALID_ARG
     assert L.w4a16_quantize(good, 256, 200, 128, good, good, good, null) == w4a16.ERR_UNSUPPORTED
     assert L.w4a16_quantize(good, 256, 256, 64, good, good, good, null) == w4a16.ERR_UNSUPPORTED

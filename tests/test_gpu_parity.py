@@ -239,3 +239,29 @@ def test_quantize_pack_gemm_pipeline():
         q_ref, s_ref, z_ref = oracle.quantize(w.view(np.uint16))
         ref = oracle.gemm(q_ref, z_ref, s_ref, x.view(np.uint16))
         assert_close(to_f64(y), ref, f"quantize+pack+gemm path={PATH_NAMES[path]}")
+
+
+# ------------------------------------------------- fused QKV split + bias ----
+
+@pytest.mark.parametrize("splits,K,N", [((200, 72, 72), 384, 1), ((200, 72, 72), 384, 2),
+                                        ((200, 72, 72), 384, 5), ((128, 64, 64), 256, 130),
+                                        ((4096, 1024, 1024), 4096, 1), ((4096, 1024, 1024), 4096, 16)])
+def test_gemm_qkv_split_and_bias(splits, K, N):
+    """Three outputs = the plain product's column ranges bit for bit without
+    bias; with an fp16 bias, within tolerance of the oracle's fp64 product
+    plus bias."""
+    M = sum(splits)
+    p = synth.make_problem(M, K, N, seed=M + K + N)
+    w, x = pack_problem(p)
+    y = run(w, x, w4a16.PATH_AUTO)
+    outs = w4a16.gemm_qkv(w, x, splits)
+    c = np.cumsum((0,) + tuple(splits))
+    for i, o in enumerate(outs):
+        assert torch.equal(o.view(torch.int16), y[:, c[i]:c[i + 1]].contiguous().view(torch.int16))
+    bias = (np.random.default_rng(M).normal(0, 1, size=M)).astype(np.float16)
+    # Caller-owned outputs, filled with NaN first: every element is written.
+    outs = tuple(torch.full((N, m), float("nan"), dtype=torch.float16, device="cuda") for m in splits)
+    w4a16.gemm_qkv(w, x, splits, bias=torch.from_numpy(bias).cuda(), out=outs)
+    ref = oracle.gemm(p.q, p.zeros, p.scales, p.x) + bias.astype(np.float64)[None, :]
+    for i, o in enumerate(outs):
+        assert_close(to_f64(o), ref[:, c[i]:c[i + 1]], f"qkv split {i} N={N}")
