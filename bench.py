@@ -42,7 +42,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # gemv_kernel<1> launch on the fused QKV shape, from the ncu capture summarised
 # in profiles/gemv_kernel_qkv_m12288_k4096_n1.md, valid only while the kernel
 # source is unchanged (sha256 prefix of csrc/w4a16_gemv.cu).
-GEMV_TRAFFIC = {"src_sha256_prefix": "6ce6410852d6b000", "qkv_dram_bytes": 26175488,
+GEMV_TRAFFIC = {"src_sha256_prefix": "e34f605c3a3ec7af", "qkv_dram_bytes": 26175488,
                 "qkv_alg_bytes": 26181632}
 
 
@@ -526,54 +526,76 @@ def prefill_measure(device, peaks, args):
 
 def qkv_fused_workload(args, device, peaks):
     """Fused QKV projection of LLaMA-7B (3 x 4096 rows, K = 4096) at N = 1
-    (8 rotated weight copies, beyond L2) and N = 4096, three arms:
-      plain   w4a16_gemm into one [N][M] buffer (no split, no bias);
-      fused   w4a16_gemm_qkv writing Q, K, V separately with an fp16 bias;
-      unfused w4a16_gemm, then a torch add per projection for the split and
-              the bias (what a caller writes without the fused form; timing
-              comparator only).
-    Each arm is a CUDA graph timed twice, in the order plain, fused, unfused,
-    unfused, fused, plain, and reported as the mean of its two timings, so a
-    clock drift under the power cap falls on every arm alike."""
+    (8 rotated weight copies, beyond L2) and N = 4096, four arms:
+      plain           w4a16_gemm into one [N][M] buffer (no split, no bias);
+      fused_split     w4a16_gemm_qkv writing Q, K, V separately, no bias;
+      fused_split_bias  the same with an fp16 bias;
+      unfused         w4a16_gemm, then a torch add per projection for the
+                      split and the bias (what a caller writes without the
+                      fused form; timing comparator only).
+    Each arm is a CUDA graph timed in three passes, the order of the arms
+    alternating (forward, reverse, forward), with the median SM clock of each
+    timing window sampled; reported are the mean time, each pass's time and
+    clock, and the mean of time x clock (cycles), which a clock drift under the
+    power cap does not move."""
     import torch
 
     from gemm_w4a16_b200 import w4a16
 
     M, K, splits = 12288, 4096, (4096, 4096, 4096)
     bounds = [(0, 4096), (4096, 8192), (8192, 12288)]
-    for N, copies_n in ((1, 8), (4096, 1)):
-        problems = [make_device_problem(device, M, K, N, seed=50 + c) for c in range(copies_n)]
-        bias = torch.randn(M, device=device).half()
-        ys = [torch.empty((N, M), dtype=torch.float16, device=device) for _ in problems]
-        outs = [tuple(torch.empty((N, m), dtype=torch.float16, device=device) for m in splits)
-                for _ in problems]
+    sampler = ClockSampler(device.index or 0)
+    sampler.start()
+    try:
+        for N, copies_n in ((1, 8), (4096, 1)):
+            problems = [make_device_problem(device, M, K, N, seed=50 + c) for c in range(copies_n)]
+            bias = torch.randn(M, device=device).half()
+            ys = [torch.empty((N, M), dtype=torch.float16, device=device) for _ in problems]
+            outs = [tuple(torch.empty((N, m), dtype=torch.float16, device=device) for m in splits)
+                    for _ in problems]
 
-        def plain():
-            for (w, x), y in zip(problems, ys):
-                w4a16.gemm(w, x, Y=y)
+            def plain():
+                for (w, x), y in zip(problems, ys):
+                    w4a16.gemm(w, x, Y=y)
 
-        def fused():
-            for (w, x), o in zip(problems, outs):
-                w4a16.gemm_qkv(w, x, splits, bias=bias, out=o)
+            def fused_split():
+                for (w, x), o in zip(problems, outs):
+                    w4a16.gemm_qkv(w, x, splits, out=o)
 
-        def unfused():
-            for (w, x), y, o in zip(problems, ys, outs):
-                w4a16.gemm(w, x, Y=y)
-                for (c0, c1), oi in zip(bounds, o):
-                    torch.add(y[:, c0:c1], bias[c0:c1], out=oi)
+            def fused():
+                for (w, x), o in zip(problems, outs):
+                    w4a16.gemm_qkv(w, x, splits, bias=bias, out=o)
 
-        arms = {"plain": plain, "fused_split_bias": fused, "unfused_gemm_then_torch_split_bias": unfused}
-        graphs = {name: capture(fn, device) for name, fn in arms.items()}
-        times = {name: [] for name in arms}
-        for name in list(arms) + list(reversed(list(arms))):
-            times[name].append(time_graph(graphs[name], args.steps, args.warmup, device) * 1e3 / copies_n)
-        for name in arms:
-            us = sum(times[name]) / len(times[name])
-            print(json.dumps({"workload": f"qkv {name} M={M} K={K} N={N}", "us": us,
-                              "us_each": times[name],
-                              "GBps": alg_bytes(M, K, N) / (us * 1e-6) / 1e9,
-                              "TFLOPS": alg_flops(M, K, N) / (us * 1e-6) / 1e12}), flush=True)
-        del graphs, problems, ys, outs
+            def unfused():
+                for (w, x), y, o in zip(problems, ys, outs):
+                    w4a16.gemm(w, x, Y=y)
+                    for (c0, c1), oi in zip(bounds, o):
+                        torch.add(y[:, c0:c1], bias[c0:c1], out=oi)
+
+            arms = {"plain": plain, "fused_split": fused_split, "fused_split_bias": fused,
+                    "unfused_gemm_then_torch_split_bias": unfused}
+            graphs = {name: capture(fn, device) for name, fn in arms.items()}
+            names = list(arms)
+            runs = {name: [] for name in arms}
+            for order in (names, names[::-1], names):
+                for name in order:
+                    t0 = time.time()
+                    us = time_graph(graphs[name], args.steps, args.warmup, device) * 1e3 / copies_n
+                    t1 = time.time()
+                    runs[name].append((us, sampler.summary(t0, t1)))
+            for name in arms:
+                us = [u for u, _ in runs[name]]
+                mhz = [c["sm_mhz"] for _, c in runs[name]]
+                reasons = sorted({r for _, c in runs[name] for r in c["reasons"]})
+                mean = sum(us) / len(us)
+                kcyc = (sum(u * f for u, f in zip(us, mhz)) / len(us) / 1e3) if None not in mhz else None
+                print(json.dumps({"workload": f"qkv {name} M={M} K={K} N={N}", "us": mean,
+                                  "us_each": us, "sm_mhz_each": mhz, "kcycles": kcyc, "reasons": reasons,
+                                  "GBps": alg_bytes(M, K, N) / (mean * 1e-6) / 1e9,
+                                  "TFLOPS": alg_flops(M, K, N) / (mean * 1e-6) / 1e12}), flush=True)
+            del graphs, problems, ys, outs
+    finally:
+        sampler.stop()
     return 0
 
 
