@@ -12,6 +12,9 @@ layer computes, in fp64, on the canonical (unpacked) arrays, written from
   names int4, group 128, a scale and a zero, but no rounding rule): min-max
   asymmetric with 0 inside the range, every decision in IEEE fp32 (see
   ``quantize``).
+* section 3.2, first fusion (residual addition and normalisation as one
+  operator), the step that produces X: r = fp16_RN(h + d) and
+  x = r * gamma / sqrt(eps + mean(r^2)) per token row (see ``add_rmsnorm``).
 * section 3.3 item 1: C[m, n] = sum_k A[m, k] B[k, n] with A the weights and n
   the tokens; item 2: the GEMV is the n = 1 case.  Storage taken: x[n][k],
   y[n][m] (token-major), sums in fp64, ascending k.
@@ -67,6 +70,8 @@ def lib():
             L.w4o_gemm_rows.restype = ctypes.c_int
             L.w4o_quantize.argtypes = [_u16p, _i64, _i64, _i64, _u8p, _u16p, _u8p]
             L.w4o_quantize.restype = ctypes.c_int
+            L.w4o_add_rmsnorm.argtypes = [_u16p, _u16p, _u16p, ctypes.c_double, _i64, _i64, _u16p, _f64p]
+            L.w4o_add_rmsnorm.restype = ctypes.c_int
             _lib = L
     return _lib
 
@@ -182,3 +187,32 @@ def quantize(W, group: int = 128):
     if rc:
         raise RuntimeError(f"oracle quantize failed ({rc})")
     return q, scales, zeros
+
+
+def add_rmsnorm(h, gamma, eps: float, d=None):
+    """Residual add and RMS normalisation per token row (reading of "PerfXLLM
+    on Snapdragon 8 Gen2", section 3.2, first fusion): r = fp16_RN(h + d)
+    (d None: r = h) and x = r * gamma / sqrt(eps + mean_k r^2).
+
+    h, d: fp16 bit patterns uint16 [N, K]; gamma: uint16 [K].  Returns
+    (r uint16 [N, K] fp16 bits, x float64 [N, K] unrounded)."""
+    h = _c(h, np.uint16)
+    if h.ndim != 2:
+        raise ValueError("h must be [N, K]")
+    N, K = h.shape
+    gamma = _c(gamma, np.uint16).reshape(-1)
+    if gamma.size != K:
+        raise ValueError("gamma must hold K values")
+    dp = None
+    if d is not None:
+        d = _c(d, np.uint16)
+        if d.shape != h.shape:
+            raise ValueError("d must match h")
+        dp = _ptr(d, _u16p)
+    r = np.empty((N, K), dtype=np.uint16)
+    x = np.empty((N, K), dtype=np.float64)
+    rc = lib().w4o_add_rmsnorm(_ptr(h, _u16p), dp, _ptr(gamma, _u16p), float(eps), N, K,
+                               _ptr(r, _u16p), _ptr(x, _f64p))
+    if rc:
+        raise RuntimeError(f"oracle add_rmsnorm failed ({rc})")
+    return r, x

@@ -271,3 +271,42 @@ int w4o_quantize(const uint16_t* W, int64_t M, int64_t K, int64_t G,
     }
     return 0;
 }
+
+/* ------------------------------------------------ residual add + norm ---- */
+
+/*
+ * Residual add and RMS normalisation, the operator that produces the
+ * layer's input X.  "PerfXLLM on Snapdragon 8 Gen2", section 3.2, first
+ * fusion: the residual connection's addition and the normalisation become
+ * one operator, so their intermediate does not travel through global memory.
+ * The page names the two operations only; reading taken, per token row n of
+ * K channels:
+ *
+ *   r[k] = fp16_RN(h[k] + d[k])        (d absent: r[k] = h[k]), the new residual
+ *   x[k] = r[k] * gamma[k] / sqrt(eps + (1/K) * sum_j r[j]^2)
+ *
+ * h, d and gamma are fp16.  The sum of two fp16 values is exact in double, so
+ * r has one rounding.  The sum of squares runs in fp64 in ascending k; x is
+ * returned in fp64, unrounded.
+ */
+int w4o_add_rmsnorm(const uint16_t* h, const uint16_t* d, const uint16_t* gamma, double eps,
+                    int64_t N, int64_t K, uint16_t* r_out, double* x_out)
+{
+    if (N < 0 || K <= 0 || !(eps >= 0.0)) return 1;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        uint16_t* r = r_out + n * K;
+        double ss = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            double v = w4o_fp16_to_double(h[n * K + k]);
+            if (d) v += w4o_fp16_to_double(d[n * K + k]);
+            r[k] = w4o_fp16_from_double(v);
+            const double rv = w4o_fp16_to_double(r[k]);
+            ss += rv * rv;
+        }
+        const double rms = sqrt(ss / (double)K + eps);
+        for (int64_t k = 0; k < K; ++k)
+            x_out[n * K + k] = w4o_fp16_to_double(r[k]) * w4o_fp16_to_double(gamma[k]) / rms;
+    }
+    return 0;
+}

@@ -337,3 +337,90 @@ def test_quantize_sign_symmetry_and_scale_invariance():
     deq = lambda qq, ss, zz: (qq.reshape(4, 2, 128).astype(np.float64) - zz[..., None]) * \
         oracle.fp16_to_double(ss)[..., None]
     assert np.allclose(deq(qn, sn, zn), -deq(q, s, z), atol=float(oracle.fp16_to_double(s).max()))
+
+
+# ------------------------------------------------ residual add + RMS norm ----
+
+def _bits(vals):
+    return np.asarray(vals, dtype=np.float16).view(np.uint16)
+
+
+def test_add_rmsnorm_closed_form_3_4():
+    """r = (1 + 2, 4 + 0) = (3, 4): the mean of squares is 12.5, so
+    x = (3, 4) / sqrt(12.5) = (3 sqrt2 / 5, 4 sqrt2 / 5); gamma = (2, 1/2)
+    scales channel by channel (swapped channels would give other values)."""
+    h, d = _bits([[1.0, 4.0]]), _bits([[2.0, 0.0]])
+    r, x = oracle.add_rmsnorm(h, _bits([1.0, 1.0]), 0.0, d=d)
+    assert r.tolist() == _bits([[3.0, 4.0]]).tolist()
+    s2 = np.sqrt(2.0)
+    np.testing.assert_allclose(x[0], [3 * s2 / 5, 4 * s2 / 5], rtol=1e-15, atol=0)
+    _, x = oracle.add_rmsnorm(h, _bits([2.0, 0.5]), 0.0, d=d)
+    np.testing.assert_allclose(x[0], [6 * s2 / 5, 2 * s2 / 5], rtol=1e-15, atol=0)
+
+
+def test_add_rmsnorm_residual_rounds_to_nearest_even():
+    """In [2048, 4096) fp16 values are 2 apart.  2048 + 1 = 2049 is halfway
+    between 2048 and 2050 and goes to the even significand, 2048; 2048 + 3 =
+    2051 goes to 2052; 2048 + 0.5 to 2048; -2048 - 1 to -2048.  Without d the
+    residual is h bit for bit, a negative zero and a subnormal included."""
+    h, d = _bits([[2048, 2048, 2048, -2048]]), _bits([[1, 3, 0.5, -1]])
+    r, _ = oracle.add_rmsnorm(h, _bits([1] * 4), 0.0, d=d)
+    assert r[0].tolist() == [0x6800, 0x6802, 0x6800, 0xE800]
+    h2 = np.array([[0x8000, 0x3C00, 0x0001, 0x7BFF]], dtype=np.uint16)
+    r2, _ = oracle.add_rmsnorm(h2, _bits([1] * 4), 0.0)
+    assert np.array_equal(r2, h2)
+
+
+def test_add_rmsnorm_normalises_the_rounded_residual():
+    """h = (2048, 1), d = (1, 0): r = (2048, 1) after rounding (not the exact
+    2049), so x0 = 2048 / sqrt((2048^2 + 1) / 2); the unrounded sum would be
+    off by about 5e-4 relative."""
+    _, x = oracle.add_rmsnorm(_bits([[2048, 1]]), _bits([1, 1]), 0.0, d=_bits([[1, 0]]))
+    rms = np.sqrt((2048.0 ** 2 + 1.0) / 2.0)
+    np.testing.assert_allclose(x[0], [2048.0 / rms, 1.0 / rms], rtol=1e-14, atol=0)
+
+
+@pytest.mark.parametrize("K", [1, 7, 4096])
+def test_add_rmsnorm_constant_row_is_sign_times_gamma(K):
+    """A row holding one value c has mean(r^2) = c^2, so with eps = 0,
+    x = gamma * c / |c| for every K (a sum in place of the mean would give
+    gamma / sqrt(K))."""
+    rng = np.random.default_rng(K)
+    gamma = rng.normal(1, 0.2, K).astype(np.float16)
+    for c in (0.75, -3.0, 2.0 ** -10):
+        h = np.full((1, K), c, dtype=np.float16).view(np.uint16)
+        _, x = oracle.add_rmsnorm(h, gamma.view(np.uint16), 0.0)
+        np.testing.assert_allclose(x[0], np.sign(c) * gamma.astype(np.float64), rtol=1e-15, atol=0)
+
+
+def test_add_rmsnorm_eps_inside_the_root():
+    """c = 2^-10 and eps = 3 * 2^-20: sqrt(c^2 + eps) = sqrt(4 * 2^-20) = 2^-9,
+    so x = gamma / 2 exactly; a zero row with eps > 0 gives x = 0."""
+    K = 16
+    gamma = _bits(np.linspace(0.5, 2.0, K))
+    h = np.full((1, K), 2.0 ** -10, dtype=np.float16).view(np.uint16)
+    _, x = oracle.add_rmsnorm(h, gamma, 3 * 2.0 ** -20)
+    np.testing.assert_array_equal(x[0], _f16(gamma).astype(np.float64) / 2)
+    _, x0 = oracle.add_rmsnorm(np.zeros((2, K), np.uint16), gamma, 2.0 ** -20)
+    assert np.all(x0 == 0)
+
+
+def test_add_rmsnorm_scale_invariance_and_row_independence():
+    """With eps = 0, scaling h and d by 8 scales r by 8 exactly (fp16 values
+    are multiples of 2^-24, so no sum rounds in the subnormal range) and
+    leaves x unchanged; a row's result does not depend on the other rows."""
+    rng = np.random.default_rng(3)
+    N, K = 4, 4096
+    h = rng.normal(0, 1, (N, K)).astype(np.float16)
+    d = rng.normal(0, 1, (N, K)).astype(np.float16)
+    gamma = rng.normal(1, 0.1, K).astype(np.float16).view(np.uint16)
+    r, x = oracle.add_rmsnorm(h.view(np.uint16), gamma, 0.0, d=d.view(np.uint16))
+    r8, x8 = oracle.add_rmsnorm((h * np.float16(8)).view(np.uint16), gamma, 0.0,
+                                d=(d * np.float16(8)).view(np.uint16))
+    assert np.array_equal(r8, (_f16(r) * np.float16(8)).view(np.uint16))
+    np.testing.assert_allclose(x8, x, rtol=1e-13, atol=0)
+    h2 = h.copy()
+    h2[0] = rng.normal(0, 5, K).astype(np.float16)
+    r2, x2 = oracle.add_rmsnorm(h2.view(np.uint16), gamma, 0.0, d=d.view(np.uint16))
+    assert np.array_equal(r2[1:], r[1:]) and np.array_equal(x2[1:], x[1:])
+    assert not np.array_equal(x2[0], x[0])
