@@ -14,7 +14,8 @@ every rank runs its own copy of the step (weak scaling), no collective on the
 data path; time is the max over ranks.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-    python bench.py --workload qkv_n1|prefill|sweep ...   (secondary workloads)
+    python bench.py --workload qkv_n1|prefill|sweep|quantize|qkv_fused|add_rmsnorm ...
+                                                          (secondary workloads)
 """
 from __future__ import annotations
 
@@ -391,6 +392,8 @@ def main_ours(args):
         return quantize_workload(args, device, peaks)
     if args.workload == "qkv_fused":
         return qkv_fused_workload(args, device, peaks)
+    if args.workload == "add_rmsnorm":
+        return add_rmsnorm_workload(args, device, peaks)
 
     calls, x_flat, y_flat = build_decode_step(device, seed=1000 + rank)
     step_bytes = sum(alg_bytes(w.M, w.K, 1) for _, w, _, _ in calls)
@@ -641,6 +644,42 @@ def quantize_workload(args, device, peaks):
     return 0
 
 
+def add_rmsnorm_workload(args, device, peaks):
+    """Residual add + RMS normalisation at LLaMA-7B width (K = 4096): N = 1
+    (one decode token; 64 rotated row buffers per graph) and N = 16384 (four
+    4096-token prefill batches; 512 MB of h, d, r and X per call, beyond L2).
+    HBM bytes per call: h and d read, r and X written, 2 bytes each per
+    channel, plus gamma once.  Each size one CUDA graph of w4a16_add_rmsnorm
+    calls."""
+    import torch
+
+    from gemm_w4a16_b200 import w4a16
+
+    K = 4096
+    gen = torch.Generator(device=device)
+    gen.manual_seed(7)
+    gamma = (1.0 + 0.1 * torch.randn(K, device=device, generator=gen)).half()
+    for N, copies_n in ((1, 64), (16384, 1)):
+        sets = []
+        for _ in range(copies_n):
+            h = torch.randn((N, K), device=device, generator=gen).half()
+            d = torch.randn((N, K), device=device, generator=gen).half()
+            sets.append((h, d, torch.empty_like(h), torch.empty_like(h)))
+
+        def fn():
+            for h, d, r, X in sets:
+                w4a16.add_rmsnorm(h, gamma, eps=1e-6, d=d, r_out=r, X=X)
+
+        g = capture(fn, device)
+        us = time_graph(g, args.steps, args.warmup, device) * 1e3 / copies_n
+        nbytes = 8 * N * K + 2 * K
+        gbps = nbytes / (us * 1e-6) / 1e9
+        print(json.dumps({"workload": f"add_rmsnorm N={N} K={K}", "us": us, "GBps": gbps,
+                          "frac_hbm": gbps / peaks["hbm_gbs"], "launches_per_graph": copies_n}), flush=True)
+        del g, sets
+    return 0
+
+
 def single_shape(args, device, M, K, N, path=0):
     """One shape, plain launches (used for ncu captures and quick timing)."""
     import torch
@@ -711,7 +750,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["decode", "qkv_n1", "prefill", "sweep", "shape", "quantize",
-                                           "qkv_fused"],
+                                           "qkv_fused", "add_rmsnorm"],
                     default="decode")
     ap.add_argument("--M", type=int, default=12288)
     ap.add_argument("--K", type=int, default=4096)

@@ -23,6 +23,12 @@ constexpr int kMaxN = 1 << 20;
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Whether the byte ranges [a, a + n) and [b, b + n) share a byte.
+bool overlap(const void* a, const void* b, size_t n) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + n && y < x + n;
+}
+
 w4a16_status check_shape(int M, int K, int group) {
   if (M <= 0 || K <= 0) return W4A16_ERR_INVALID_ARG;
   if (group != kGroup || K % kGroup != 0) return W4A16_ERR_UNSUPPORTED;
@@ -78,6 +84,25 @@ w4a16_status w4a16_quantize(const uint16_t* W, int M, int K, int group, uint8_t*
   if (!aligned16(W) || !aligned16(q) || (reinterpret_cast<uintptr_t>(scales) & 1u))
     return W4A16_ERR_MISALIGNED;
   return map_cuda(launch_quantize(W, M, K, q, scales, zeros, static_cast<cudaStream_t>(stream)));
+}
+
+w4a16_status w4a16_add_rmsnorm(const uint16_t* h, const uint16_t* d, const uint16_t* gamma, float eps,
+                               int N, int K, uint16_t* r_out, uint16_t* X, void* stream) {
+  if (!h || !gamma || !X) return W4A16_ERR_INVALID_ARG;
+  if (N <= 0 || K <= 0 || !(eps >= 0.0f) || !(eps <= 3.4028234663852886e38f)) return W4A16_ERR_INVALID_ARG;
+  if (K % 8 != 0 || K > kMaxNormK || N > kMaxN) return W4A16_ERR_UNSUPPORTED;
+  if (!aligned16(h) || (d && !aligned16(d)) || !aligned16(gamma) || (r_out && !aligned16(r_out)) ||
+      !aligned16(X))
+    return W4A16_ERR_MISALIGNED;
+  const size_t bytes = (size_t)N * K * 2;
+  // r_out may be h or d itself; X shares no byte with the other rows' data.
+  if (overlap(X, h, bytes) || (d && overlap(X, d, bytes)) || (r_out && overlap(X, r_out, bytes)) ||
+      overlap(X, gamma, (size_t)K * 2))
+    return W4A16_ERR_INVALID_ARG;
+  if (r_out && ((r_out != h && overlap(r_out, h, bytes)) || (d && r_out != d && overlap(r_out, d, bytes)) ||
+                overlap(r_out, gamma, (size_t)K * 2)))
+    return W4A16_ERR_INVALID_ARG;
+  return map_cuda(launch_add_rmsnorm(h, d, gamma, eps, N, K, r_out, X, static_cast<cudaStream_t>(stream)));
 }
 
 w4a16_status w4a16_pack(const uint8_t* q, const uint16_t* scales, const uint8_t* zeros,

@@ -155,6 +155,12 @@ cudaError_t launch_gemv(const uint8_t* wq, const uint16_t* scales, const uint8_t
                         const uint16_t* X, uint16_t* Y, int M, int K, int N,
                         cudaStream_t stream, const OutMap* om = nullptr);
 
+// Residual add + RMS normalisation: one CTA per token row, K a multiple of 8
+// and at most kMaxNormK (the row's residual is held in shared memory).
+constexpr int kMaxNormK = 1 << 16;
+cudaError_t launch_add_rmsnorm(const uint16_t* h, const uint16_t* d, const uint16_t* gamma, float eps,
+                               int N, int K, uint16_t* r_out, uint16_t* X, cudaStream_t stream);
+
 cudaError_t launch_quantize(const uint16_t* W, int M, int K, uint8_t* q, uint16_t* scales, uint8_t* zeros,
                             cudaStream_t stream);
 

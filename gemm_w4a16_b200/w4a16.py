@@ -22,6 +22,7 @@ EXPORTED = (
     "w4a16_status_string", "w4a16_packed_sizes", "w4a16_pack", "w4a16_gemm",
     "w4a16_gemm_ex", "w4a16_select_path", "w4a16_dequant_debug",
     "w4a16_device_status", "w4a16_selftest_wait_timeout", "w4a16_quantize", "w4a16_gemm_qkv",
+    "w4a16_add_rmsnorm",
 )
 
 _lib = None
@@ -53,6 +54,8 @@ def lib():
             L.w4a16_packed_sizes.restype = _i
             L.w4a16_quantize.argtypes = [_vp, _i, _i, _i, _vp, _vp, _vp, _vp]
             L.w4a16_quantize.restype = _i
+            L.w4a16_add_rmsnorm.argtypes = [_vp, _vp, _vp, ctypes.c_float, _i, _i, _vp, _vp, _vp]
+            L.w4a16_add_rmsnorm.restype = _i
             L.w4a16_pack.argtypes = [_vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp]
             L.w4a16_pack.restype = _i
             L.w4a16_gemm.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]
@@ -144,6 +147,32 @@ def quantize(W, group: int = GROUP, stream=None):
     _check(lib().w4a16_quantize(_ptr(W), M, K, group, _ptr(q), _ptr(scales), _ptr(zeros),
                                 _stream_ptr(stream)), "w4a16_quantize")
     return q, scales, zeros
+
+
+def add_rmsnorm(h, gamma, eps: float = 1e-6, d=None, r_out=None, X=None, stream=None):
+    """Residual add + RMS normalisation via w4a16_add_rmsnorm: r = h + d
+    (fp16, written to r_out when given; r_out may be h or d) and
+    X = r * gamma / sqrt(eps + mean(r^2)) per token row.  h, d, r_out, X:
+    contiguous CUDA fp16 [N, K]; gamma [K].  Returns (r_out, X)."""
+    import torch
+
+    def _ok(t, shape):
+        return (t.dtype == torch.float16 and t.is_cuda and t.is_contiguous()
+                and tuple(t.shape) == tuple(shape))
+
+    if h.dim() != 2 or not _ok(h, h.shape):
+        raise ValueError("h must be a contiguous CUDA fp16 [N, K] tensor")
+    N, K = h.shape
+    if not _ok(gamma, (K,)):
+        raise ValueError("gamma must be a contiguous CUDA fp16 tensor of K values")
+    for name, t in (("d", d), ("r_out", r_out), ("X", X)):
+        if t is not None and not _ok(t, (N, K)):
+            raise ValueError(f"{name} must be a contiguous CUDA fp16 [N, K] tensor")
+    if X is None:
+        X = torch.empty((N, K), dtype=torch.float16, device=h.device)
+    _check(lib().w4a16_add_rmsnorm(_ptr(h), _ptr(d), _ptr(gamma), float(eps), N, K, _ptr(r_out), _ptr(X),
+                                   _stream_ptr(stream)), "w4a16_add_rmsnorm")
+    return r_out, X
 
 
 def pack(q, scales, zeros, group: int = GROUP, out: PackedWeight | None = None,

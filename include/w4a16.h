@@ -102,6 +102,30 @@ W4A16_API w4a16_status w4a16_quantize(const uint16_t* W, int M, int K, int group
                             uint8_t* q, uint16_t* scales, uint8_t* zeros, void* stream);
 
 /*
+ * Residual add + RMS normalisation: the operator that produces X for the
+ * projections.  "PerfXLLM on Snapdragon 8 Gen2", section 3.2, first fusion:
+ * the residual connection's addition and the normalisation are one operator,
+ * so their intermediate does not travel through global memory.  Per token row
+ * n (reading of the page, which names the two operations only):
+ *     r[n][k] = fp16_RN(h[n][k] + d[n][k])                 (d == NULL: r = h)
+ *     X[n][k] = fp16_RN((r[n][k] * inv) * gamma[k]),  inv = 1 / sqrt(eps + (1/K) sum_k r[n][k]^2)
+ * with the mean, the root and the products in fp32 and one rounding of X.
+ *   h      device fp16 [N][K], the residual stream
+ *   d      device fp16 [N][K] added to it, or NULL
+ *   gamma  device fp16 [K], the normalisation weight
+ *   eps    finite, >= 0
+ *   r_out  device fp16 [N][K], the new residual, or NULL not to write it; may be
+ *          h or d itself (updated in place), must not partly overlap either
+ *   X      device fp16 [N][K]; must not overlap h, d, gamma or r_out
+ * Every pointer 16-byte aligned; N >= 1; K a multiple of 8, at most 65536.
+ * W4A16_ERR_INVALID_ARG for null h, gamma or X, N or K <= 0, a negative or
+ * non-finite eps, or overlapping buffers; W4A16_ERR_UNSUPPORTED for K % 8 != 0
+ * or K > 65536.
+ */
+W4A16_API w4a16_status w4a16_add_rmsnorm(const uint16_t* h, const uint16_t* d, const uint16_t* gamma,
+                               float eps, int N, int K, uint16_t* r_out, uint16_t* X, void* stream);
+
+/*
  * Canonical -> packed layout (offline; not on the per-token path).
  *   q       device uint8  [M][K], values 0..15 (higher bits are ignored)
  *   scales  device fp16   [M][K/128]

@@ -118,6 +118,38 @@ def test_rejects_bad_arguments_without_launching(L):
     assert L.w4a16_selftest_wait_timeout(1 << 40, null) == w4a16.ERR_INVALID_ARG
 
 
+def test_add_rmsnorm_rejects_bad_arguments_without_launching(L):
+    """Each call breaks one rule and must fail on the host (none may reach a
+    launch: the addresses are not memory).  N = 2, K = 64: 256 bytes a row
+    block; the fake buffers sit 64 KB apart."""
+    p = lambda a: ctypes.c_void_p(a)
+    h, d, g, r, x, null = 0x10000, 0x20000, 0x30000, 0x40000, 0x50000, 0
+    f = L.w4a16_add_rmsnorm
+
+    def call(h=h, d=d, g=g, eps=1e-6, N=2, K=64, r=r, x=x):
+        return f(p(h), p(d), p(g), eps, N, K, p(r), p(x), p(null))
+
+    assert call(h=null) == w4a16.ERR_INVALID_ARG
+    assert call(g=null) == w4a16.ERR_INVALID_ARG
+    assert call(x=null) == w4a16.ERR_INVALID_ARG
+    assert call(N=0) == w4a16.ERR_INVALID_ARG
+    assert call(K=0) == w4a16.ERR_INVALID_ARG
+    assert call(eps=-1.0) == w4a16.ERR_INVALID_ARG
+    assert call(eps=float("nan")) == w4a16.ERR_INVALID_ARG
+    assert call(eps=float("inf")) == w4a16.ERR_INVALID_ARG
+    assert call(K=60) == w4a16.ERR_UNSUPPORTED
+    assert call(K=65536 + 8) == w4a16.ERR_UNSUPPORTED
+    for name in ("h", "d", "g", "r", "x"):
+        assert call(**{name: {"h": h, "d": d, "g": g, "r": r, "x": x}[name] + 8}) == w4a16.ERR_MISALIGNED
+    assert call(x=h + 128) == w4a16.ERR_INVALID_ARG          # X inside h
+    assert call(x=d + 240) == w4a16.ERR_INVALID_ARG          # X overlaps d's last bytes
+    assert call(x=g) == w4a16.ERR_INVALID_ARG                # X on gamma
+    assert call(x=r + 16) == w4a16.ERR_INVALID_ARG           # X inside r_out
+    assert call(r=h + 16) == w4a16.ERR_INVALID_ARG           # r_out partly over h
+    assert call(r=d - 16) == w4a16.ERR_INVALID_ARG           # r_out partly over d
+    assert call(r=g) == w4a16.ERR_INVALID_ARG                # r_out on gamma
+
+
 def test_select_path_is_monotone_in_n(L):
     assert w4a16.select_path(0, 4096, 1) == -1
     assert w4a16.select_path(4096, 100, 1) == -1

@@ -265,3 +265,120 @@ def test_gemm_qkv_split_and_bias(splits, K, N):
     ref = oracle.gemm(p.q, p.zeros, p.scales, p.x) + bias.astype(np.float64)[None, :]
     for i, o in enumerate(outs):
         assert_close(to_f64(o), ref[:, c[i]:c[i + 1]], f"qkv split {i} N={N}")
+
+
+# ------------------------------------------ residual add + RMS normalisation ----
+
+NORM_EPS = 1e-6
+
+
+def _norm_inputs(N, K, seed, outliers=0):
+    """h, d ~ N(0, 1) fp16 (the residual stream and the block output added to
+    it), gamma ~ N(1, 0.1); `outliers` fixed channels of h scaled by 50 in
+    fp32 before the fp16 rounding."""
+    rng = np.random.default_rng(seed)
+    h = rng.normal(0, 1, (N, K))
+    if outliers:
+        h[:, rng.choice(K, size=outliers, replace=False)] *= 50.0
+    d = rng.normal(0, 1, (N, K))
+    gamma = rng.normal(1, 0.1, K)
+    return h.astype(np.float16), d.astype(np.float16), gamma.astype(np.float16)
+
+
+def _assert_norm_close(X, x_ref, what):
+    """Per element |X - x| <= 2^-10 |x| + 2^-24: one fp16 rounding (2^-11
+    relative, 2^-25 absolute for subnormals) on top of fp32 arithmetic whose
+    relative error stays below 1e-5 (a sum of non-negative squares over at
+    most 256 sequential terms per thread plus 8 reduction steps, then the
+    mean, the root and two products), and the C9 tensor bar."""
+    y = to_f64(X)
+    bound = np.abs(x_ref) * 2.0 ** -10 + 2.0 ** -24
+    bad = np.abs(y - x_ref) > bound
+    assert not bad.any(), f"{what}: {int(bad.sum())} elements beyond the bound"
+    assert_close(y, x_ref, what)
+
+
+@pytest.mark.parametrize("N,K", [(1, 8), (1, 4096), (3, 4096), (7, 24), (5, 5120), (2, 65536),
+                                 (64, 8192), (33, 11008)])
+def test_add_rmsnorm_matches_oracle(N, K):
+    h, d, gamma = _norm_inputs(N, K, seed=N + K)
+    th, td, tg = (torch.from_numpy(a).cuda() for a in (h, d, gamma))
+    r = torch.empty_like(th)
+    _, X = w4a16.add_rmsnorm(th, tg, eps=NORM_EPS, d=td, r_out=r)
+    _, X2 = w4a16.add_rmsnorm(th, tg, eps=NORM_EPS, d=td)
+    torch.cuda.synchronize()
+    r_ref, x_ref = oracle.add_rmsnorm(h.view(np.uint16), gamma.view(np.uint16), NORM_EPS, d=d.view(np.uint16))
+    assert np.array_equal(r.cpu().numpy().view(np.uint16), r_ref)
+    _assert_norm_close(X, x_ref, f"add_rmsnorm N={N} K={K}")
+    assert torch.equal(X.view(torch.int16), X2.view(torch.int16))      # deterministic
+
+
+def test_add_rmsnorm_without_d_and_in_place():
+    N, K = 6, 4096
+    h, d, gamma = _norm_inputs(N, K, seed=11)
+    tg = torch.from_numpy(gamma).cuda()
+    # No d: X from h alone, nothing else written.
+    _, X = w4a16.add_rmsnorm(torch.from_numpy(h).cuda(), tg, eps=NORM_EPS)
+    _, x_ref = oracle.add_rmsnorm(h.view(np.uint16), gamma.view(np.uint16), NORM_EPS)
+    _assert_norm_close(X, x_ref, "add_rmsnorm without d")
+    r_ref, x_ref = oracle.add_rmsnorm(h.view(np.uint16), gamma.view(np.uint16), NORM_EPS, d=d.view(np.uint16))
+    # The residual updated in place, over h and over d.
+    for target in ("h", "d"):
+        th, td = torch.from_numpy(h).cuda(), torch.from_numpy(d).cuda()
+        dst = th if target == "h" else td
+        _, X = w4a16.add_rmsnorm(th, tg, eps=NORM_EPS, d=td, r_out=dst)
+        torch.cuda.synchronize()
+        assert np.array_equal(dst.cpu().numpy().view(np.uint16), r_ref), target
+        _assert_norm_close(X, x_ref, f"add_rmsnorm in place over {target}")
+
+
+def test_add_rmsnorm_zero_rows_outliers_and_guard_bands():
+    N, K, pad = 16, 4096, 64
+    h, d, gamma = _norm_inputs(N, K, seed=12, outliers=40)
+    h[3] = 0
+    d[3] = 0
+    th, td, tg = (torch.from_numpy(a).cuda() for a in (h, d, gamma))
+    buf = torch.full((N * K + 2 * pad,), 12345, dtype=torch.int16, device="cuda")
+    X = buf[pad:pad + N * K].view(torch.float16).view(N, K)
+    w4a16.add_rmsnorm(th, tg, eps=NORM_EPS, d=td, X=X)
+    torch.cuda.synchronize()
+    assert torch.all(buf[:pad] == 12345) and torch.all(buf[-pad:] == 12345)
+    assert torch.count_nonzero(X[3]).item() == 0
+    _, x_ref = oracle.add_rmsnorm(h.view(np.uint16), gamma.view(np.uint16), NORM_EPS, d=d.view(np.uint16))
+    _assert_norm_close(X, x_ref, "add_rmsnorm with outlier channels")
+
+
+def test_add_rmsnorm_full_size_sampled_rows():
+    """16384 token rows of LLaMA-7B width (4096), the benchmarked size; sampled
+    rows against the oracle (each row is normalised on its own)."""
+    N, K = 16384, 4096
+    h, d, gamma = _norm_inputs(N, K, seed=13, outliers=40)
+    th, td, tg = (torch.from_numpy(a).cuda() for a in (h, d, gamma))
+    r = torch.empty_like(th)
+    _, X = w4a16.add_rmsnorm(th, tg, eps=NORM_EPS, d=td, r_out=r)
+    torch.cuda.synchronize()
+    rows = sample_rows(N, 256, seed=13)
+    r_ref, x_ref = oracle.add_rmsnorm(h[rows].view(np.uint16), gamma.view(np.uint16), NORM_EPS,
+                                      d=d[rows].view(np.uint16))
+    ti = torch.from_numpy(rows).cuda()
+    assert np.array_equal(r[ti].cpu().numpy().view(np.uint16), r_ref)
+    _assert_norm_close(X[ti], x_ref, "add_rmsnorm full size (sampled rows)")
+
+
+def test_add_rmsnorm_then_fused_qkv():
+    """The layer's first two steps chained on the GPU: X from the residual add
+    and normalisation, then the fused QKV projection; against the oracle's
+    chain, whose X is rounded to fp16 by the oracle itself."""
+    N, K, splits = 5, 4096, (4096, 1024, 1024)
+    M = sum(splits)
+    h, d, gamma = _norm_inputs(N, K, seed=14)
+    p = synth.make_problem(M, K, N, seed=14)
+    w, _ = pack_problem(p)
+    _, X = w4a16.add_rmsnorm(*(torch.from_numpy(a).cuda() for a in (h, gamma)), eps=NORM_EPS,
+                             d=torch.from_numpy(d).cuda())
+    outs = w4a16.gemm_qkv(w, X, splits)
+    _, x_ref = oracle.add_rmsnorm(h.view(np.uint16), gamma.view(np.uint16), NORM_EPS, d=d.view(np.uint16))
+    y_ref = oracle.gemm(p.q, p.zeros, p.scales, oracle.fp16_from_double(x_ref))
+    c = np.cumsum((0,) + splits)
+    for i, o in enumerate(outs):
+        assert_close(to_f64(o), y_ref[:, c[i]:c[i + 1]], f"add_rmsnorm -> qkv split {i}")
