@@ -1,6 +1,7 @@
 // C-ABI entry points of libw4a16: host-side argument checks, the N-based
-// dispatcher between the CUDA-core GEMV and the tcgen05 GEMM, and status
-// mapping.  "PerfXLLM on Snapdragon 8 Gen2", section 3.3: prefill (tokens > 1)
+// dispatcher between the CUDA-core GEMV and the tcgen05 GEMM (for the plain
+// product and its fused QKV form), the quantiser, packing and residual
+// add + normalisation launches, and status mapping.  "PerfXLLM on Snapdragon 8 Gen2", section 3.3: prefill (tokens > 1)
 // is a GEMM and decode (tokens = 1) a GEMV; few tokens make the GEMM
 // memory-bound and many make it compute-bound, and each regime gets its own
 // tiling.  Here each regime gets its own kernel.
