@@ -15,6 +15,8 @@ layer computes, in fp64, on the canonical (unpacked) arrays, written from
 * section 3.2, first fusion (residual addition and normalisation as one
   operator), the step that produces X: r = fp16_RN(h + d) and
   x = r * gamma / sqrt(eps + mean(r^2)) per token row (see ``add_rmsnorm``).
+* the gate/up projection's epilogue, SiLU(gate) * up (an extension of the
+  fusion principle of section 3.2; see ``gate_up``).
 * section 3.3 item 1: C[m, n] = sum_k A[m, k] B[k, n] with A the weights and n
   the tokens; item 2: the GEMV is the n = 1 case.  Storage taken: x[n][k],
   y[n][m] (token-major), sums in fp64, ascending k.
@@ -216,3 +218,28 @@ def add_rmsnorm(h, gamma, eps: float, d=None):
     if rc:
         raise RuntimeError(f"oracle add_rmsnorm failed ({rc})")
     return r, x
+
+
+def silu_mul(y, Mi: int) -> np.ndarray:
+    """H[n][i] = silu(g) * u with g = y[n][i], u = y[n][Mi + i] and
+    silu(g) = g / (1 + exp(-g)), all in fp64 (y: [N, 2 Mi] float64, e.g. the
+    accumulators of ``gemm`` on a weight whose rows are the gate projection's
+    Mi rows followed by the up projection's Mi rows)."""
+    y = np.asarray(y, dtype=np.float64)
+    if y.ndim != 2 or y.shape[1] != 2 * Mi or Mi <= 0:
+        raise ValueError("y must be [N, 2 Mi]")
+    g, u = y[:, :Mi], y[:, Mi:]
+    with np.errstate(over="ignore"):
+        return g / (1.0 + np.exp(-g)) * u
+
+
+def gate_up(q, zeros, scales, x, Mi: int, group: int = 128) -> np.ndarray:
+    """The gate/up layer's output SiLU(X W_gate^T) * (X W_up^T) in fp64, for a
+    canonical weight of 2 Mi rows: rows [0, Mi) the gate projection, rows
+    [Mi, 2 Mi) the up projection (reading of "PerfXLLM on Snapdragon 8 Gen2",
+    section 3.2: fusion removes the intermediate's round trip through global
+    memory; the page names no such fusion for the feed-forward block, the
+    principle is extended to it).  Returns [N, Mi]."""
+    if np.asarray(q).shape[0] != 2 * Mi:
+        raise ValueError("the weight must have 2 Mi rows")
+    return silu_mul(gemm(q, zeros, scales, x, group), Mi)

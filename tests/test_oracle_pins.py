@@ -424,3 +424,81 @@ def test_add_rmsnorm_scale_invariance_and_row_independence():
     r2, x2 = oracle.add_rmsnorm(h2.view(np.uint16), gamma, 0.0, d=d.view(np.uint16))
     assert np.array_equal(r2[1:], r[1:]) and np.array_equal(x2[1:], x[1:])
     assert not np.array_equal(x2[0], x[0])
+
+
+# ------------------------------------------------ gate/up: SiLU(gate) * up ----
+
+# The logistic function at 1, 2 and -1: e/(1+e), e^2/(1+e^2), 1/(1+e).
+SIGMA_1 = 0.7310585786300049
+SIGMA_2 = 0.8807970779778823
+SIGMA_M1 = 0.2689414213699951
+
+
+def _one_hot_problem(g_vals, u_vals, K=128):
+    """s = 1, z = 8 and X = e_0, so the product's row m is q[m][0] - 8 exactly:
+    the gate rows hold g_vals, the up rows u_vals."""
+    Mi = len(g_vals)
+    q = np.full((2 * Mi, K), 8, dtype=np.uint8)
+    q[:Mi, 0] = 8 + np.asarray(g_vals)
+    q[Mi:, 0] = 8 + np.asarray(u_vals)
+    zeros = np.full((2 * Mi, K // 128), 8, dtype=np.uint8)
+    scales = np.full((2 * Mi, K // 128), 0x3C00, dtype=np.uint16)       # 1.0
+    x = np.zeros((1, K), dtype=np.float16)
+    x[0, 0] = 1.0
+    return q, zeros, scales, x.view(np.uint16), Mi
+
+
+def test_gate_up_textbook_logistic_values():
+    """silu(g) = g * sigma(g): g = 0, 1, 2, -1 against the logistic function's
+    textbook values, each times its own u (row i pairs with row Mi + i)."""
+    g, u = [0, 1, 2, -1], [3, 2, 1, 5]
+    q, z, s, x, Mi = _one_hot_problem(g, u)
+    h = oracle.gate_up(q, z, s, x, Mi)
+    expect = [0.0, 1 * SIGMA_1 * 2, 2 * SIGMA_2 * 1, -1 * SIGMA_M1 * 5]
+    np.testing.assert_allclose(h[0], expect, rtol=1e-15, atol=0)
+
+
+def test_gate_up_order_of_gate_and_up_matters():
+    """(g, u) = (1, 2) gives 2 sigma(1) = 1.462...; the swapped reading
+    silu(u) * g would give 2 sigma(2) = 1.761..."""
+    q, z, s, x, Mi = _one_hot_problem([1], [2])
+    h = oracle.gate_up(q, z, s, x, Mi)[0, 0]
+    assert abs(h - 2 * SIGMA_1) < 1e-15
+    assert abs(h - 2 * SIGMA_2) > 0.2
+
+
+def test_gate_up_odd_symmetry_and_extremes():
+    """silu(g) - silu(-g) = g (sigma(g) + sigma(-g) = 1) for every g; far
+    negative g gives 0 (exp overflows to infinity, no NaN), far positive g
+    gives g."""
+    rng = np.random.default_rng(21)
+    g = rng.normal(0, 4, 64)
+    y = np.concatenate([np.stack([g, -g]), np.ones((2, 64))], axis=1)
+    h = oracle.silu_mul(y, 64)
+    np.testing.assert_allclose(h[0] - h[1], g, rtol=0, atol=1e-13)
+    ext = oracle.silu_mul(np.array([[-1024.0, 40.0, 3.0, 2.0]]), 2)
+    assert np.all(np.isfinite(ext)) and ext[0, 0] == 0.0
+    assert ext[0, 1] == 80.0                 # 40 * (1 + e^-40)^-1 rounds to 40 in fp64
+
+
+def test_gate_up_large_negative_accumulator_through_the_product():
+    """All gate codes 0 (w = -8) and X = 1 in every channel: g = -1024 exactly,
+    so SiLU(g) * u underflows to zero without a NaN."""
+    K = 128
+    q = np.zeros((2, K), dtype=np.uint8)
+    q[1] = 9                                                            # u = K * 1
+    zeros = np.full((2, 1), 8, dtype=np.uint8)
+    scales = np.full((2, 1), 0x3C00, dtype=np.uint16)
+    x = np.ones((1, K), dtype=np.float16).view(np.uint16)
+    y = oracle.gemm(q, zeros, scales, x)
+    assert y[0, 0] == -1024.0 and y[0, 1] == 128.0
+    h = oracle.gate_up(q, zeros, scales, x, 1)
+    assert h.shape == (1, 1) and h[0, 0] == 0.0
+
+
+def test_gate_up_rejects_bad_shapes():
+    with pytest.raises(ValueError):
+        oracle.silu_mul(np.zeros((1, 5)), 2)
+    q, z, s, x, Mi = _one_hot_problem([1, 2], [3, 4])
+    with pytest.raises(ValueError):
+        oracle.gate_up(q, z, s, x, 3)
