@@ -24,10 +24,29 @@ constexpr int kMaxN = 1 << 20;
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Whether the byte ranges [a, a + n) and [b, b + n) share a byte.
-bool overlap(const void* a, const void* b, size_t n) {
+// Whether the byte ranges [a, a + na) and [b, b + nb) share a byte (a null
+// pointer or an empty range shares none).
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b || !na || !nb) return false;
   const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
-  return x < y + n && y < x + n;
+  return x < y + nb && y < x + na;
+}
+
+// Byte sizes of the packed buffers of an M x K weight (group 128).
+struct PackedBytes {
+  size_t wq, scales, zeros;
+};
+
+PackedBytes packed_bytes(int M, int K) {
+  const size_t mp = (size_t)ceil_div(M, kRowBlock) * kRowBlock;
+  const size_t kg = (size_t)K / kGroup;
+  return {mp * (size_t)K / 2, mp * kg * 2, mp * kg / 2};
+}
+
+// Whether the output range [y, y + ny) overlaps the packed weight.
+bool overlaps_weight(const void* y, size_t ny, const void* wq, const void* sp, const void* zp,
+                     const PackedBytes& pb) {
+  return overlap(y, ny, wq, pb.wq) || overlap(y, ny, sp, pb.scales) || overlap(y, ny, zp, pb.zeros);
 }
 
 w4a16_status check_shape(int M, int K, int group) {
@@ -69,11 +88,10 @@ w4a16_status w4a16_packed_sizes(int M, int K, int group, size_t* wq_bytes,
   if (!wq_bytes || !scales_bytes || !zeros_bytes) return W4A16_ERR_INVALID_ARG;
   w4a16_status st = check_shape(M, K, group);
   if (st != W4A16_OK) return st;
-  const size_t mp = (size_t)ceil_div(M, kRowBlock) * kRowBlock;
-  const size_t kg = (size_t)K / kGroup;
-  *wq_bytes = mp * (size_t)K / 2;
-  *scales_bytes = mp * kg * 2;
-  *zeros_bytes = mp * kg / 2;
+  const PackedBytes pb = packed_bytes(M, K);
+  *wq_bytes = pb.wq;
+  *scales_bytes = pb.scales;
+  *zeros_bytes = pb.zeros;
   return W4A16_OK;
 }
 
@@ -84,6 +102,10 @@ w4a16_status w4a16_quantize(const uint16_t* W, int M, int K, int group, uint8_t*
   if (st != W4A16_OK) return st;
   if (!aligned16(W) || !aligned16(q) || (reinterpret_cast<uintptr_t>(scales) & 1u))
     return W4A16_ERR_MISALIGNED;
+  const size_t mk = (size_t)M * K, mg = (size_t)M * (K / kGroup);
+  if (overlap(q, mk, W, mk * 2) || overlap(scales, mg * 2, W, mk * 2) || overlap(zeros, mg, W, mk * 2) ||
+      overlap(q, mk, scales, mg * 2) || overlap(q, mk, zeros, mg) || overlap(scales, mg * 2, zeros, mg))
+    return W4A16_ERR_INVALID_ARG;
   return map_cuda(launch_quantize(W, M, K, q, scales, zeros, static_cast<cudaStream_t>(stream)));
 }
 
@@ -97,11 +119,12 @@ w4a16_status w4a16_add_rmsnorm(const uint16_t* h, const uint16_t* d, const uint1
     return W4A16_ERR_MISALIGNED;
   const size_t bytes = (size_t)N * K * 2;
   // r_out may be h or d itself; X shares no byte with the other rows' data.
-  if (overlap(X, h, bytes) || (d && overlap(X, d, bytes)) || (r_out && overlap(X, r_out, bytes)) ||
-      overlap(X, gamma, (size_t)K * 2))
+  const size_t gbytes = (size_t)K * 2;
+  if (overlap(X, bytes, h, bytes) || overlap(X, bytes, d, bytes) || overlap(X, bytes, r_out, bytes) ||
+      overlap(X, bytes, gamma, gbytes))
     return W4A16_ERR_INVALID_ARG;
-  if (r_out && ((r_out != h && overlap(r_out, h, bytes)) || (d && r_out != d && overlap(r_out, d, bytes)) ||
-                overlap(r_out, gamma, (size_t)K * 2)))
+  if (r_out && ((r_out != h && overlap(r_out, bytes, h, bytes)) ||
+                (r_out != d && overlap(r_out, bytes, d, bytes)) || overlap(r_out, bytes, gamma, gbytes)))
     return W4A16_ERR_INVALID_ARG;
   return map_cuda(launch_add_rmsnorm(h, d, gamma, eps, N, K, r_out, X, static_cast<cudaStream_t>(stream)));
 }
@@ -116,6 +139,19 @@ w4a16_status w4a16_pack(const uint8_t* q, const uint16_t* scales, const uint8_t*
   if (!aligned16(wq_packed) || !aligned16(scales_packed) || !aligned16(zeros_packed) ||
       (reinterpret_cast<uintptr_t>(scales) & 1u))
     return W4A16_ERR_MISALIGNED;
+  {
+    const PackedBytes pb = packed_bytes(M, K);
+    const size_t mk = (size_t)M * K, mg = (size_t)M * (K / kGroup);
+    const void* outs[3] = {wq_packed, scales_packed, zeros_packed};
+    const size_t out_n[3] = {pb.wq, pb.scales, pb.zeros};
+    for (int i = 0; i < 3; ++i) {
+      if (overlap(outs[i], out_n[i], q, mk) || overlap(outs[i], out_n[i], scales, mg * 2) ||
+          overlap(outs[i], out_n[i], zeros, mg))
+        return W4A16_ERR_INVALID_ARG;
+      for (int j = i + 1; j < 3; ++j)
+        if (overlap(outs[i], out_n[i], outs[j], out_n[j])) return W4A16_ERR_INVALID_ARG;
+    }
+  }
   return map_cuda(launch_pack(q, scales, zeros, M, K, static_cast<uint8_t*>(wq_packed),
                               static_cast<uint16_t*>(scales_packed),
                               static_cast<uint8_t*>(zeros_packed),
@@ -135,6 +171,12 @@ w4a16_status w4a16_gemm_ex(const void* wq_packed, const void* scales_packed,
   if (!aligned16(wq_packed) || !aligned16(scales_packed) || !aligned16(zeros_packed) ||
       !aligned16(X) || !aligned16(Y))
     return W4A16_ERR_MISALIGNED;
+  {
+    const size_t ny = (size_t)N * M * 2;
+    if (overlap(Y, ny, X, (size_t)N * K * 2) ||
+        overlaps_weight(Y, ny, wq_packed, scales_packed, zeros_packed, packed_bytes(M, K)))
+      return W4A16_ERR_INVALID_ARG;
+  }
   if (path == W4A16_PATH_AUTO) path = select_path_impl(M, K, N);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const uint8_t* wq = static_cast<const uint8_t*>(wq_packed);
@@ -158,6 +200,18 @@ w4a16_status w4a16_gemm_qkv(const void* wq_packed, const void* scales_packed, co
   if (!aligned16(wq_packed) || !aligned16(scales_packed) || !aligned16(zeros_packed) || !aligned16(X) ||
       !aligned16(Yq) || !aligned16(Yk) || !aligned16(Yv) || (reinterpret_cast<uintptr_t>(bias) & 1u))
     return W4A16_ERR_MISALIGNED;
+  {
+    const PackedBytes pb = packed_bytes(M, K);
+    const void* outs[3] = {Yq, Yk, Yv};
+    const size_t out_n[3] = {(size_t)N * Mq * 2, (size_t)N * Mk * 2, (size_t)N * Mv * 2};
+    for (int i = 0; i < 3; ++i) {
+      if (overlap(outs[i], out_n[i], X, (size_t)N * K * 2) || overlap(outs[i], out_n[i], bias, (size_t)M * 2) ||
+          overlaps_weight(outs[i], out_n[i], wq_packed, scales_packed, zeros_packed, pb))
+        return W4A16_ERR_INVALID_ARG;
+      for (int j = i + 1; j < 3; ++j)
+        if (overlap(outs[i], out_n[i], outs[j], out_n[j])) return W4A16_ERR_INVALID_ARG;
+    }
+  }
   OutMap om;
   om.y0 = Yq;
   om.y1 = Yk;
@@ -191,6 +245,8 @@ w4a16_status w4a16_dequant_debug(const void* wq_packed, const void* scales_packe
   if (!aligned16(wq_packed) || !aligned16(scales_packed) || !aligned16(zeros_packed) ||
       !aligned16(W_out))
     return W4A16_ERR_MISALIGNED;
+  if (overlaps_weight(W_out, (size_t)M * K * 2, wq_packed, scales_packed, zeros_packed, packed_bytes(M, K)))
+    return W4A16_ERR_INVALID_ARG;
   return map_cuda(launch_dequant(static_cast<const uint8_t*>(wq_packed),
                                  static_cast<const uint16_t*>(scales_packed),
                                  static_cast<const uint8_t*>(zeros_packed), W_out, M, K,

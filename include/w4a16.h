@@ -20,6 +20,9 @@
  *   - Argument checks run on the host before any launch and return an error
  *     code without touching the GPU.  Launch failures are reported as
  *     W4A16_ERR_CUDA.  Nothing is thrown and nothing exits.
+ *   - An output buffer may not share a byte with an input or with another
+ *     output of the same call (W4A16_ERR_INVALID_ARG), except where a call
+ *     allows in-place use (the residual of w4a16_add_rmsnorm).
  *   - Calls are asynchronous on `stream` (0 = the legacy default stream).
  */
 #ifndef W4A16_H

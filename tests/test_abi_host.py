@@ -150,6 +150,43 @@ def test_add_rmsnorm_rejects_bad_arguments_without_launching(L):
     assert call(r=g) == w4a16.ERR_INVALID_ARG                # r_out on gamma
 
 
+def test_overlapping_buffers_rejected_without_launching(L):
+    """Outputs may not overlap inputs or each other.  M = K = 256, N = 2:
+    packed codes 32 KB, scales 1 KB, zeros 256 B, X and Y 1 KB; every fake
+    buffer sits 1 MB from the next, so the one overlap planted per call is the
+    only one (and no call reaches a launch)."""
+    p = lambda a: ctypes.c_void_p(a)
+    wq, sc, zp, x, y, bias, yq, yk, yv = (k << 20 for k in range(1, 10))
+    null = p(0)
+    ex = lambda Y: L.w4a16_gemm_ex(p(wq), p(sc), p(zp), p(x), p(Y), 256, 256, 2, 128, 0, null)
+    assert ex(x) == w4a16.ERR_INVALID_ARG                    # Y on X
+    assert ex(wq + 0x1000) == w4a16.ERR_INVALID_ARG          # Y inside the packed codes
+    assert ex(zp + 0x80) == w4a16.ERR_INVALID_ARG            # Y over the zeros
+    assert L.w4a16_gemm(p(wq), p(sc), p(zp), p(x), p(sc + 0x100), 256, 256, 2, 128, null) == \
+        w4a16.ERR_INVALID_ARG                                # Y over the scales
+
+    def qkv(Yq=yq, Yk=yk, Yv=yv, B=bias):                    # Mq = 128, Mk = Mv = 64
+        return L.w4a16_gemm_qkv(p(wq), p(sc), p(zp), p(x), p(B), 128, 64, 64, 256, 2, 128,
+                                p(Yq), p(Yk), p(Yv), null)
+
+    assert qkv(Yk=yq + 256) == w4a16.ERR_INVALID_ARG         # Yk inside Yq (512 B)
+    assert qkv(Yv=x + 16) == w4a16.ERR_INVALID_ARG           # Yv over X
+    assert qkv(Yq=bias + 256) == w4a16.ERR_INVALID_ARG       # Yq over the bias (512 B)
+    assert qkv(Yv=wq + 0x2000) == w4a16.ERR_INVALID_ARG      # Yv inside the packed codes
+    # quantiser: W 128 KB, q 64 KB, scales 1 KB, zeros 512 B
+    assert L.w4a16_quantize(p(wq), 256, 256, 128, p(wq + 0x10000), p(sc), p(zp), null) == \
+        w4a16.ERR_INVALID_ARG                                # q inside W
+    assert L.w4a16_quantize(p(wq), 256, 256, 128, p(x), p(x + 0x1000), p(zp), null) == \
+        w4a16.ERR_INVALID_ARG                                # scales inside q
+    # pack: inputs q 64 KB, scales 1 KB, zeros 512 B; outputs 32 KB, 1 KB, 256 B
+    assert L.w4a16_pack(p(x), p(sc), p(zp), 256, 256, 128, p(x + 0x100), p(yq), p(yk), null) == \
+        w4a16.ERR_INVALID_ARG                                # packed codes over q
+    assert L.w4a16_pack(p(x), p(sc), p(zp), 256, 256, 128, p(yq), p(yq + 0x400), p(yk), null) == \
+        w4a16.ERR_INVALID_ARG                                # packed scales inside packed codes
+    assert L.w4a16_dequant_debug(p(wq), p(sc), p(zp), p(sc), 256, 256, 128, null) == \
+        w4a16.ERR_INVALID_ARG                                # W_out on the scales
+
+
 def test_select_path_is_monotone_in_n(L):
     assert w4a16.select_path(0, 4096, 1) == -1
     assert w4a16.select_path(4096, 100, 1) == -1
