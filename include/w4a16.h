@@ -164,7 +164,7 @@ W4A16_API w4a16_status w4a16_gemm(const void* wq_packed, const void* scales_pack
  *     Yk[n][m]      = fp16_RN(acc[n][Mq + m]      + bias[Mq + m])      m < Mk
  *     Yv[n][m]      = fp16_RN(acc[n][Mq + Mk + m] + bias[Mq + Mk + m]) m < Mv
  * with acc the fp32 accumulator of w4a16_gemm and the bias added in fp32
- * (bias device fp16 [M], or NULL for none).  Mq, Mk, Mv >= 1; other
+ * (bias device fp16 [M], 2-byte aligned, or NULL for none).  Mq, Mk, Mv >= 1; other
  * arguments, alignment (Yq, Yk, Yv 16-byte aligned) and kernel choice as
  * w4a16_gemm.
  */
