@@ -4,10 +4,16 @@
 Default workload (one "step"): a LLaMA-7B-shaped decode step at N = 1 token --
 32 layers x {fused QKV 12288x4096, O 4096x4096, fused gate/up 22016x4096,
 down 4096x11008}, 128 distinct packed weight sets resident in HBM (3.37 GB, far
-beyond the 126 MB L2, so no flush is needed), each projection one w4a16_gemm
-call, the step captured once in a CUDA graph.  The metric is algorithmic HBM
-bytes per second (packed int4 weights + 2.5 B per group of metadata + fp16 X
-and Y), reported against the measured HBM copy bandwidth.
+beyond the 126 MB L2, so no flush is needed), each projection one
+w4a16_gemm_ws call (the split tensor-core decode kernel, weights streamed
+early under programmatic dependent launch), the step captured once in a CUDA
+graph.  The metric is algorithmic HBM bytes per second (packed int4 weights +
+2.5 B per group of metadata + fp16 X and Y), reported against the measured HBM
+copy bandwidth.  The same JSON line carries, each with its own clock summary
+and median / p10 / p90 over its repeats: every projection alone, the two
+prefill GEMMs (TFLOP/s), the fused-QKV N sweep on every kernel, the
+LLaMA-3-8B batched-decode shapes, and the CPU oracle at all cores and at one
+thread.
 
 One JSON line on stdout (rank 0).  Multi-GPU runs (torchrun) are replicas:
 every rank runs its own copy of the step (weak scaling), no collective on the
@@ -39,12 +45,13 @@ LLAMA7B_LAYER = [("qkv", 12288, 4096), ("o", 4096, 4096), ("gate_up", 22016, 409
 N_LAYERS = 32
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one
-# gemv_kernel<1> launch on the fused QKV shape, from the ncu capture summarised
-# in profiles/gemv_kernel_qkv_m12288_k4096_n1.md, valid only while the kernel
-# source is unchanged (sha256 prefix of csrc/w4a16_gemv.cu).
-GEMV_TRAFFIC = {"src_sha256_prefix": "e34f605c3a3ec7af", "qkv_dram_bytes": 26175488,
-                "qkv_alg_bytes": 26181632}
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one decode
+# launch of the split tensor-core kernel on the fused QKV shape at N = 1, from
+# an ncu capture of this repository's kernel; it holds only while the kernel
+# source is the one captured (sha256 prefix of csrc/w4a16_gemv_tc.cu), and
+# the bench reports null otherwise.
+DECODE_TRAFFIC = {"src_sha256_prefix": "", "qkv_dram_bytes": 0, "qkv_alg_bytes": 26181632}
+NOMINAL_DENSE_FP16_TFLOPS = 2250.0   # B200 dense fp16/bf16 tensor rate, NVIDIA's figure
 
 
 def alg_bytes(M, K, N):
@@ -56,20 +63,21 @@ def alg_flops(M, K, N):
     return 2 * M * N * K
 
 
-def gemv_traffic_per_launch(alg_bytes_per_launch):
+def decode_traffic_per_launch(alg_bytes_per_launch):
     """ncu DRAM bytes per decode launch, scaled from the QKV capture by the
     algorithmic bytes (every shape streams its weights once), or None when
     the kernel source changed since the capture."""
     import hashlib
 
-    src = os.path.join(ROOT, "gemm_w4a16_b200", "csrc", "w4a16_gemv.cu")
+    src = os.path.join(ROOT, "gemm_w4a16_b200", "csrc", "w4a16_gemv_tc.cu")
     try:
         h = hashlib.sha256(open(src, "rb").read()).hexdigest()
     except OSError:
         return None
-    if not h.startswith(GEMV_TRAFFIC["src_sha256_prefix"]):
+    pre = DECODE_TRAFFIC["src_sha256_prefix"]
+    if not pre or not h.startswith(pre):
         return None
-    return GEMV_TRAFFIC["qkv_dram_bytes"] / GEMV_TRAFFIC["qkv_alg_bytes"] * alg_bytes_per_launch
+    return DECODE_TRAFFIC["qkv_dram_bytes"] / DECODE_TRAFFIC["qkv_alg_bytes"] * alg_bytes_per_launch
 
 
 def load_peaks():
@@ -228,6 +236,14 @@ def run_calls(calls, path=0):
             w4a16.gemm(w, x, Y=y)
 
 
+def run_calls_ws(calls, ws, flags=0, path=0):
+    """Each call through w4a16_gemm_ws on one shared workspace."""
+    from gemm_w4a16_b200 import w4a16
+
+    for _, w, x, y in calls:
+        w4a16.gemm_ws(w, x, Y=y, path=path, workspace=ws, flags=flags)
+
+
 def capture(fn, device):
     import torch
 
@@ -244,8 +260,10 @@ def capture(fn, device):
     return g
 
 
-def time_graph(g, steps, warmup, device, pre=None, post=None):
-    """ms per step of graph replays, CUDA events on the replay stream."""
+def time_steps(g, steps, warmup, device, pre=None, post=None):
+    """Replays of graph g: W untimed, then exactly `steps` timed with a CUDA
+    event recorded on the replay stream before the first and after every
+    replay.  Returns (total ms of the bracketed region, per-replay ms)."""
     import torch
 
     stream = torch.cuda.current_stream(device)
@@ -256,18 +274,33 @@ def time_graph(g, steps, warmup, device, pre=None, post=None):
         if post:
             post()
     torch.cuda.synchronize(device)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(steps):
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    ev[0].record(stream)
+    for i in range(steps):
         if pre:
             pre()
         g.replay()
         if post:
             post()
-    e1.record(stream)
+        ev[i + 1].record(stream)
     torch.cuda.synchronize(device)
-    return e0.elapsed_time(e1) / steps
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+    return ev[0].elapsed_time(ev[steps]), per
+
+
+def time_graph(g, steps, warmup, device, pre=None, post=None):
+    """Mean ms per replay of graph g over `steps` timed replays."""
+    total, _ = time_steps(g, steps, warmup, device, pre, post)
+    return total / steps
+
+
+def pct(values, scale=1.0):
+    """median, p10 and p90 of a list (times scale)."""
+    import numpy as np
+
+    v = np.asarray(values, dtype=np.float64) * scale
+    return {"median": float(np.median(v)), "p10": float(np.percentile(v, 10)),
+            "p90": float(np.percentile(v, 90)), "n": int(v.size)}
 
 
 # ------------------------------------------------------- CPU (oracle) leg --
@@ -298,12 +331,15 @@ def _oracle_pass(layer):
     return nbytes
 
 
-def oracle_decode_sample(target_s=12.0, max_layers=N_LAYERS, seed=0):
-    """Time the CPU oracle, as it stands, over whole synthetic layers of the
-    decode step until about target_s seconds of work; returns GB/s."""
+def oracle_decode_sample(target_s=12.0, max_layers=N_LAYERS, seed=0, threads=None, rows=None):
+    """Time the CPU oracle, as it stands, over synthetic layers of the decode
+    step (whole layers, or their first `rows` output rows) until about
+    target_s seconds of work, on `threads` host threads (default: all);
+    returns GB/s of algorithmic bytes."""
     import oracle
 
-    layer = _oracle_layer(seed=seed)
+    oracle.set_threads(threads or os.cpu_count() or 1)
+    layer = _oracle_layer(rows=rows, seed=seed)
     nbytes = 0
     layers = 0
     t0 = time.perf_counter()
@@ -313,9 +349,10 @@ def oracle_decode_sample(target_s=12.0, max_layers=N_LAYERS, seed=0):
         if time.perf_counter() - t0 >= target_s:
             break
     dt = time.perf_counter() - t0
+    what = "full layer(s)" if rows is None else f"layer(s) of the first {rows} rows"
     return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": oracle.get_threads(),
             "kind": "oracle",
-            "sample": f"{layers} full layer(s) of the 4 LLaMA-7B projections at N=1 "
+            "sample": f"{layers} {what} of the 4 LLaMA-7B projections at N=1 "
                       f"({layers * 4} oracle products, {nbytes / 1e6:.0f} MB algorithmic, "
                       f"{dt:.1f} s)"}
 
@@ -395,39 +432,31 @@ def main_ours(args):
     if args.workload == "add_rmsnorm":
         return add_rmsnorm_workload(args, device, peaks)
 
-    calls, x_flat, y_flat = build_decode_step(device, seed=1000 + rank)
-    step_bytes = sum(alg_bytes(w.M, w.K, 1) for _, w, _, _ in calls)
-    launches_per_step = len(calls)      # one kernel launch per projection at N = 1
-    g = capture(lambda: run_calls(calls), device)
-
-    # Device-resident timing (the headline value).
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
+
+    calls, x_flat, y_flat = build_decode_step(device, seed=1000 + rank)
+    step_bytes = sum(alg_bytes(w.M, w.K, 1) for _, w, _, _ in calls)
+    ws = w4a16.Workspace(device, max(w4a16.workspace_size(w.M, w.K, 1) for _, w, _, _ in calls))
+    flags = w4a16.FLAG_EARLY_WEIGHTS
+    launches_per_step = len(calls)      # one kernel launch per projection at N = 1
+    g = capture(lambda: run_calls_ws(calls, ws, flags), device)
+
+    # Device-resident timing (the headline value).
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize(device)
     t_wall0 = time.time()
-    ms = time_graph(g, args.steps, args.warmup, device)
+    total_ms, per_step = time_steps(g, args.steps, args.warmup, device)
     t_wall1 = time.time()
-    time.sleep(0.2)
-    sampler.stop()
+    ms = total_ms / args.steps
     ms_max = max_over_ranks(ms, dist, device)
     total_bytes = sum_over_ranks(step_bytes * args.steps, dist, device)
     value = total_bytes / (ms_max * args.steps * 1e-3) / 1e9
+    clocks = sampler.summary(t_wall0, t_wall1)
 
-    # Per-shape achieved bandwidth: each projection type alone, 32 distinct
-    # weight sets per graph so every launch reads its weights from HBM.
-    per_shape = {}
-    for name, M, K in LLAMA7B_LAYER:
-        sub = [c for c in calls if c[0] == name]
-        gs = capture(lambda sub=sub: run_calls(sub), device)
-        ms_s = time_graph(gs, max(10, args.steps // 4), 3, device) / len(sub)
-        b = alg_bytes(M, K, 1)
-        per_shape[name] = {"M": M, "K": K, "N": 1, "us": ms_s * 1e3,
-                           "GBps": b / (ms_s * 1e-3) / 1e9,
-                           "frac_hbm": b / (ms_s * 1e-3) / 1e9 / peaks["hbm_gbs"]}
-        del gs
+    per_shape = per_shape_measure(calls, ws, flags, device, peaks, sampler)
 
     # End to end: H2D of every call's X from pinned host memory, the graph,
     # D2H of every Y, all on the stream, inside the event-timed region.
@@ -440,27 +469,32 @@ def main_ours(args):
                         post=lambda: y_host.copy_(y_flat, non_blocking=True))
     ms_e2e_max = max_over_ranks(ms_e2e, dist, device)
     e2e_value = sum_over_ranks(step_bytes, dist, device) / (ms_e2e_max * 1e-3) / 1e9
+    del g, calls, x_flat, y_flat
+    torch.cuda.empty_cache()
 
-    prefill = None
-    if w4a16.select_path(12288, 4096, 4096) == w4a16.PATH_TC and not args.no_prefill:
-        prefill = prefill_measure(device, peaks, args)
+    extra = {}
+    if not args.no_extra:
+        extra["prefill"] = prefill_measure(device, peaks, sampler)
+        extra["n_sweep"] = n_sweep_measure(device, peaks, sampler)
+        extra["llama3"] = llama3_measure(device, peaks, sampler)
 
     res = None
     if rank == 0 and world == 1 and not args.no_cpu:
         res = oracle_decode_sample(target_s=args.cpu_seconds)
+        res["single_thread"] = oracle_decode_sample(target_s=args.cpu_seconds, threads=1, rows=512)
+    sampler.stop()
 
     if dist is not None:
-        del g
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
         return 0
 
-    clocks = sampler.summary(t_wall0, t_wall1)
     achieved = step_bytes / (ms * 1e-3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "ms_per_step_pct": pct(per_step),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f16", "accumulate": "f32", "data": "synthetic",
         "config": {"workload": "llama7b_decode_step_n1",
@@ -468,26 +502,50 @@ def main_ours(args):
                                   "down 4096x11008}, N=1, group 128, 128 distinct weight sets",
                    "bytes_per_step": step_bytes, "global_batch": 1, "seq_len": 1,
                    "l2": "inputs 3.37 GB per step > 126 MB L2 (no flush needed)",
-                   "launch": "cuda_graph", "parallelism": f"replicas{world}"},
-        "roofline": {"bound": "hbm", "kernel": "gemv_kernel<1>", "achieved": achieved,
+                   "launch": "cuda_graph, programmatic dependent launch (early weights)",
+                   "api": "w4a16_gemm_ws (auto path: split tensor-core decode kernel)",
+                   "parallelism": f"replicas{world}"},
+        "roofline": {"bound": "hbm", "kernel": "gemv_tc_kernel", "achieved": achieved,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks_src,
-                     "traffic": gemv_traffic_per_launch(step_bytes / len(calls)),
-                     "traffic_note": "bytes per launch, scaled from the QKV ncu capture"},
+                     "traffic": decode_traffic_per_launch(step_bytes / launches_per_step),
+                     "traffic_note": "DRAM bytes per launch, scaled from the QKV ncu capture"},
         "per_shape": per_shape,
         "e2e": {"value": e2e_value, "unit": "GB/s",
-                "h2d_bytes_per_step": int(x_flat.numel() * 2),
-                "d2h_bytes_per_step": int(y_flat.numel() * 2), "ms_per_step": ms_e2e_max,
-                "api": "w4a16_gemm (128 calls captured in a CUDA graph) + pinned H2D/D2H"},
+                "h2d_bytes_per_step": int(x_host.numel() * 2),
+                "d2h_bytes_per_step": int(y_host.numel() * 2), "ms_per_step": ms_e2e_max,
+                "api": "w4a16_gemm_ws (128 calls captured in a CUDA graph) + pinned H2D/D2H by torch copy_"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
-    if prefill:
-        line["prefill"] = prefill
+    line.update(extra)
     if res:
         line["cpu_baseline"] = res
     print(json.dumps(line), flush=True)
     return 0
+
+
+def per_shape_measure(calls, ws, flags, device, peaks, sampler, reps=60):
+    """Each projection type alone: its 32 distinct weight sets in one graph
+    (so every launch reads its weights from HBM); per-call microseconds as
+    median / p10 / p90 over the replays."""
+    from gemm_w4a16_b200 import w4a16  # noqa: F401
+
+    out = {}
+    for name, M, K in LLAMA7B_LAYER:
+        sub = [c for c in calls if c[0] == name]
+        gs = capture(lambda sub=sub: run_calls_ws(sub, ws, flags), device)
+        t0 = time.time()
+        _, per = time_steps(gs, reps, 5, device)
+        t1 = time.time()
+        us = pct(per, 1e3 / len(sub))
+        b = alg_bytes(M, K, 1)
+        out[name] = {"M": M, "K": K, "N": 1, "us": us["median"], "us_pct": us,
+                     "GBps": b / (us["median"] * 1e-6) / 1e9,
+                     "frac_hbm": b / (us["median"] * 1e-6) / 1e9 / peaks["hbm_gbs"],
+                     "clocks": sampler.summary(t0, t1)}
+        del gs
+    return out
 
 
 def make_device_problem(device, M, K, N, seed, outlier_frac=0.0):
@@ -508,23 +566,125 @@ def make_device_problem(device, M, K, N, seed, outlier_frac=0.0):
     return w, x
 
 
-def prefill_measure(device, peaks, args):
+def prefill_measure(device, peaks, sampler, reps=50, copies=3):
+    """The two prefill GEMMs of the benchmark configuration (1 % outlier
+    channels in X), TFLOP/s.  `copies` distinct (W, X, Y) sets per graph
+    (> 250 MB, beyond L2) so no call finds its inputs cached; per-call
+    microseconds as median / p10 / p90 over the replays, against the measured
+    bf16 peak (fp16 runs at the same rate) and NVIDIA's dense fp16 figure."""
     import torch
 
     from gemm_w4a16_b200 import w4a16
 
     out = {}
     for name, M, K, N in (("qkv_n4096", 12288, 4096, 4096), ("down_n2048", 4096, 11008, 2048)):
-        w, x = make_device_problem(device, M, K, N, seed=7, outlier_frac=0.01)
-        y = torch.empty((N, M), dtype=torch.float16, device=device)
-        g = capture(lambda: w4a16.gemm(w, x, Y=y), device)
-        ms = time_graph(g, 20, 5, device)
-        tf = alg_flops(M, K, N) / (ms * 1e-3) / 1e12
-        out[name] = {"M": M, "K": K, "N": N, "us": ms * 1e3, "TFLOPS": tf,
-                     "frac_tensor": tf / peaks["bf16_tflops"],
-                     "peak": peaks["bf16_tflops"], "peak_kind": "bf16 burst (fp16 same rate)"}
-        del g, w, x, y
+        sets = []
+        for c in range(copies):
+            w, x = make_device_problem(device, M, K, N, seed=7 + c, outlier_frac=0.01)
+            sets.append((w, x, torch.empty((N, M), dtype=torch.float16, device=device)))
+        g = capture(lambda: [w4a16.gemm(w, x, Y=y) for w, x, y in sets], device)
+        t0 = time.time()
+        _, per = time_steps(g, reps, 5, device)
+        t1 = time.time()
+        us = pct(per, 1e3 / copies)
+        tf = alg_flops(M, K, N) / (us["median"] * 1e-6) / 1e12
+        out[name] = {"M": M, "K": K, "N": N, "us": us["median"], "us_pct": us, "TFLOPS": tf,
+                     "path": w4a16.select_path(M, K, N),
+                     "frac_tensor": tf / peaks["bf16_tflops"], "peak": peaks["bf16_tflops"],
+                     "peak_kind": "measured bf16 burst (cuBLAS; fp16 same rate)",
+                     "frac_nominal_dense_fp16": tf / NOMINAL_DENSE_FP16_TFLOPS,
+                     "clocks": sampler.summary(t0, t1)}
+        del g, sets
+        torch.cuda.empty_cache()
     return out
+
+
+SWEEP_N = (1, 2, 4, 8, 16, 32, 64, 128, 256, 512, 1024, 2048, 4096)
+
+
+def n_sweep_measure(device, peaks, sampler, copies=16, reps=20):
+    """N sweep on the fused QKV shape (M = 12288, K = 4096), every kernel that
+    takes the N (CUDA-core GEMV up to 64 tokens, split tensor-core decode up
+    to 16, tensor-core tiles always), 16 rotated weight copies (420 MB,
+    beyond L2).  Rows: [N, path, median us, roofline fraction, chosen]."""
+    import torch
+
+    from gemm_w4a16_b200 import synth, w4a16
+
+    M, K = 12288, 4096
+    ws_copies = [make_device_problem(device, M, K, 1, seed=100 + i)[0] for i in range(copies)]
+    rows = []
+    t0 = time.time()
+    for N in SWEEP_N:
+        gen = torch.Generator(device=device)
+        gen.manual_seed(N)
+        x = synth.make_activations_torch(N, K, gen, device)
+        y = torch.empty((N, M), dtype=torch.float16, device=device)
+        wsp = w4a16.Workspace(device, w4a16.workspace_size(M, K, min(N, w4a16.GEMV_TC_MAX_TOKENS)))
+        chosen = w4a16.select_path_ws(M, K, N)
+        paths = [w4a16.PATH_TC]
+        if N <= 64:
+            paths.insert(0, w4a16.PATH_GEMV)
+        if N <= w4a16.GEMV_TC_MAX_TOKENS:
+            paths.append(w4a16.PATH_GEMV_TC)
+        for path in paths:
+            flags = w4a16.FLAG_EARLY_WEIGHTS if path == w4a16.PATH_GEMV_TC else 0
+            g = capture(lambda path=path, flags=flags: [w4a16.gemm_ws(w, x, Y=y, path=path, workspace=wsp,
+                                                                     flags=flags) for w in ws_copies], device)
+            _, per = time_steps(g, reps, 3, device)
+            us = pct(per, 1e3 / copies)["median"]
+            gbs = alg_bytes(M, K, N) / (us * 1e-6) / 1e9
+            tfs = alg_flops(M, K, N) / (us * 1e-6) / 1e12
+            rows.append([N, {1: "gemv", 2: "tc", 3: "gemv_tc"}[path], round(us, 2),
+                         round(max(gbs / peaks["hbm_gbs"], tfs / peaks["bf16_tflops"]), 3),
+                         path == chosen])
+            del g
+    t1 = time.time()
+    del ws_copies
+    torch.cuda.empty_cache()
+    return {"M": M, "K": K, "columns": ["N", "path", "us", "roof_frac", "auto_choice"], "rows": rows,
+            "clocks": sampler.summary(t0, t1)}
+
+
+LLAMA3_SHAPES = [("qkv", 6144, 4096), ("o", 4096, 4096), ("gate_up", 28672, 4096), ("down", 4096, 14336),
+                 ("lm_head", 128256, 4096)]
+
+
+def llama3_measure(device, peaks, sampler, reps=20):
+    """LLaMA-3-8B batched decode, N in {1, 16, 64}, the automatic path of the
+    workspace entry point (early weights); rotated copies totalling at least
+    400 MB per shape (beyond L2).  Rows: [shape, N, path, median us, GB/s,
+    roofline fraction]."""
+    import torch
+
+    from gemm_w4a16_b200 import synth, w4a16
+
+    rows = []
+    t0 = time.time()
+    for name, M, K in LLAMA3_SHAPES:
+        copies = max(2, min(16, -(-400_000_000 // alg_bytes(M, K, 1))))
+        wts = [make_device_problem(device, M, K, 1, seed=300 + i)[0] for i in range(copies)]
+        for N in (1, 16, 64):
+            gen = torch.Generator(device=device)
+            gen.manual_seed(N)
+            x = synth.make_activations_torch(N, K, gen, device)
+            y = torch.empty((N, M), dtype=torch.float16, device=device)
+            wsp = w4a16.Workspace(device, w4a16.workspace_size(M, K, N))
+            g = capture(lambda: [w4a16.gemm_ws(w, x, Y=y, workspace=wsp, flags=w4a16.FLAG_EARLY_WEIGHTS)
+                                 for w in wts], device)
+            _, per = time_steps(g, reps, 3, device)
+            us = pct(per, 1e3 / copies)["median"]
+            gbs = alg_bytes(M, K, N) / (us * 1e-6) / 1e9
+            tfs = alg_flops(M, K, N) / (us * 1e-6) / 1e12
+            rows.append([name, N, {1: "gemv", 2: "tc", 3: "gemv_tc"}[w4a16.select_path_ws(M, K, N)],
+                         round(us, 2), round(gbs, 1),
+                         round(max(gbs / peaks["hbm_gbs"], tfs / peaks["bf16_tflops"]), 3)])
+            del g
+        del wts
+        torch.cuda.empty_cache()
+    t1 = time.time()
+    return {"columns": ["shape", "N", "path", "us", "GBps", "roof_frac"], "rows": rows,
+            "clocks": sampler.summary(t0, t1)}
 
 
 def qkv_fused_workload(args, device, peaks):
@@ -758,7 +918,8 @@ def main(argv=None):
     ap.add_argument("--path", type=int, default=0, help="0 auto, 1 GEMV, 2 tensor cores")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the prefill, N-sweep and LLaMA-3 measurements")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -62,9 +62,110 @@ w4a16_status map_cuda(cudaError_t e) {
   return W4A16_ERR_CUDA;
 }
 
-int select_path_impl(int M, int K, int N) {
+// with_ws: a workspace is available, which opens the split decode kernel.
+int select_path_impl(int M, int K, int N, bool with_ws) {
   if (M <= 0 || K <= 0 || N <= 0 || K % kGroup) return -1;
+  if (with_ws && N <= kGemvTcMaxTokens) return W4A16_PATH_GEMV_TC;
   return N <= gemv_max_n() ? W4A16_PATH_GEMV : W4A16_PATH_TC;
+}
+
+size_t workspace_for(int path, int M, int K, int N) {
+  return path == W4A16_PATH_GEMV_TC ? gemv_tc_workspace_bytes(M, K, N) : 0;
+}
+
+// Checks shared by the plain and the workspace entry points, then the launch
+// on the chosen path.  ws may be null (ws_bytes 0).
+w4a16_status gemm_impl(const void* wq_packed, const void* scales_packed, const void* zeros_packed,
+                       const uint16_t* X, uint16_t* Y, int M, int K, int N, int group, int path, void* ws,
+                       size_t ws_bytes, unsigned flags, void* stream) {
+  if (!wq_packed || !scales_packed || !zeros_packed || !X || !Y) return W4A16_ERR_INVALID_ARG;
+  if (N <= 0 || path < W4A16_PATH_AUTO || path > W4A16_PATH_GEMV_TC) return W4A16_ERR_INVALID_ARG;
+  if (flags & ~W4A16_FLAG_EARLY_WEIGHTS) return W4A16_ERR_INVALID_ARG;
+  if (!ws && ws_bytes) return W4A16_ERR_INVALID_ARG;
+  w4a16_status st = check_shape(M, K, group);
+  if (st != W4A16_OK) return st;
+  if (N > kMaxN) return W4A16_ERR_UNSUPPORTED;
+  if (!aligned16(wq_packed) || !aligned16(scales_packed) || !aligned16(zeros_packed) ||
+      !aligned16(X) || !aligned16(Y) || (ws && !aligned16(ws)))
+    return W4A16_ERR_MISALIGNED;
+  if (path == W4A16_PATH_AUTO) path = select_path_impl(M, K, N, ws != nullptr);
+  if (path == W4A16_PATH_GEMV_TC && N > kGemvTcMaxTokens) return W4A16_ERR_UNSUPPORTED;
+  const size_t need = workspace_for(path, M, K, N);
+  if (need > ws_bytes) return W4A16_ERR_INVALID_ARG;
+  {
+    const PackedBytes pb = packed_bytes(M, K);
+    const size_t ny = (size_t)N * M * 2, nx = (size_t)N * K * 2;
+    if (overlap(Y, ny, X, nx) || overlaps_weight(Y, ny, wq_packed, scales_packed, zeros_packed, pb))
+      return W4A16_ERR_INVALID_ARG;
+    if (need && (overlap(ws, need, X, nx) || overlap(ws, need, Y, ny) ||
+                 overlaps_weight(ws, need, wq_packed, scales_packed, zeros_packed, pb)))
+      return W4A16_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint8_t* wq = static_cast<const uint8_t*>(wq_packed);
+  const uint16_t* sp = static_cast<const uint16_t*>(scales_packed);
+  const uint8_t* zp = static_cast<const uint8_t*>(zeros_packed);
+  cudaError_t e;
+  if (path == W4A16_PATH_GEMV_TC)
+    e = launch_gemv_tc(wq, sp, zp, X, Y, M, K, N, ws, (flags & W4A16_FLAG_EARLY_WEIGHTS) != 0, s);
+  else if (path == W4A16_PATH_TC)
+    e = launch_gemm_tc(wq, sp, zp, X, Y, M, K, N, s);
+  else
+    e = launch_gemv(wq, sp, zp, X, Y, M, K, N, s);
+  return map_cuda(e);
+}
+
+w4a16_status gemm_qkv_impl(const void* wq_packed, const void* scales_packed, const void* zeros_packed,
+                           const uint16_t* X, const uint16_t* bias, int Mq, int Mk, int Mv, int K, int N,
+                           int group, uint16_t* Yq, uint16_t* Yk, uint16_t* Yv, void* ws, size_t ws_bytes,
+                           unsigned flags, void* stream) {
+  if (!wq_packed || !scales_packed || !zeros_packed || !X || !Yq || !Yk || !Yv) return W4A16_ERR_INVALID_ARG;
+  if (Mq <= 0 || Mk <= 0 || Mv <= 0 || N <= 0) return W4A16_ERR_INVALID_ARG;
+  if (flags & ~W4A16_FLAG_EARLY_WEIGHTS) return W4A16_ERR_INVALID_ARG;
+  if (!ws && ws_bytes) return W4A16_ERR_INVALID_ARG;
+  if ((long long)Mq + Mk + Mv > kMaxM) return W4A16_ERR_UNSUPPORTED;
+  const int M = Mq + Mk + Mv;
+  w4a16_status st = check_shape(M, K, group);
+  if (st != W4A16_OK) return st;
+  if (N > kMaxN) return W4A16_ERR_UNSUPPORTED;
+  if (!aligned16(wq_packed) || !aligned16(scales_packed) || !aligned16(zeros_packed) || !aligned16(X) ||
+      !aligned16(Yq) || !aligned16(Yk) || !aligned16(Yv) || (reinterpret_cast<uintptr_t>(bias) & 1u) ||
+      (ws && !aligned16(ws)))
+    return W4A16_ERR_MISALIGNED;
+  const int path = select_path_impl(M, K, N, ws != nullptr);
+  const size_t need = workspace_for(path, M, K, N);
+  if (need > ws_bytes) return W4A16_ERR_INVALID_ARG;
+  {
+    const PackedBytes pb = packed_bytes(M, K);
+    const void* outs[4] = {Yq, Yk, Yv, need ? ws : nullptr};
+    const size_t out_n[4] = {(size_t)N * Mq * 2, (size_t)N * Mk * 2, (size_t)N * Mv * 2, need};
+    for (int i = 0; i < 4; ++i) {
+      if (overlap(outs[i], out_n[i], X, (size_t)N * K * 2) || overlap(outs[i], out_n[i], bias, (size_t)M * 2) ||
+          overlaps_weight(outs[i], out_n[i], wq_packed, scales_packed, zeros_packed, pb))
+        return W4A16_ERR_INVALID_ARG;
+      for (int j = i + 1; j < 4; ++j)
+        if (overlap(outs[i], out_n[i], outs[j], out_n[j])) return W4A16_ERR_INVALID_ARG;
+    }
+  }
+  OutMap om;
+  om.y0 = Yq;
+  om.y1 = Yk;
+  om.y2 = Yv;
+  om.end0 = Mq;
+  om.end1 = Mq + Mk;
+  om.bias = bias;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint8_t* wq = static_cast<const uint8_t*>(wq_packed);
+  const uint16_t* sp = static_cast<const uint16_t*>(scales_packed);
+  const uint8_t* zp = static_cast<const uint8_t*>(zeros_packed);
+  cudaError_t e;
+  if (path == W4A16_PATH_GEMV_TC)
+    e = launch_gemv_tc(wq, sp, zp, X, nullptr, M, K, N, ws, (flags & W4A16_FLAG_EARLY_WEIGHTS) != 0, s, &om);
+  else if (path == W4A16_PATH_TC)
+    e = launch_gemm_tc(wq, sp, zp, X, nullptr, M, K, N, s, &om);
+  else
+    e = launch_gemv(wq, sp, zp, X, nullptr, M, K, N, s, &om);
+  return map_cuda(e);
 }
 
 }  // namespace
@@ -158,75 +259,45 @@ w4a16_status w4a16_pack(const uint8_t* q, const uint16_t* scales, const uint8_t*
                               static_cast<cudaStream_t>(stream)));
 }
 
-int w4a16_select_path(int M, int K, int N) { return select_path_impl(M, K, N); }
+int w4a16_select_path(int M, int K, int N) { return select_path_impl(M, K, N, false); }
+
+int w4a16_select_path_ws(int M, int K, int N) { return select_path_impl(M, K, N, true); }
 
 w4a16_status w4a16_gemm_ex(const void* wq_packed, const void* scales_packed,
                            const void* zeros_packed, const uint16_t* X, uint16_t* Y,
                            int M, int K, int N, int group, int path, void* stream) {
-  if (!wq_packed || !scales_packed || !zeros_packed || !X || !Y) return W4A16_ERR_INVALID_ARG;
-  if (N <= 0 || path < W4A16_PATH_AUTO || path > W4A16_PATH_TC) return W4A16_ERR_INVALID_ARG;
+  return gemm_impl(wq_packed, scales_packed, zeros_packed, X, Y, M, K, N, group, path, nullptr, 0, 0u, stream);
+}
+
+w4a16_status w4a16_gemm_ws(const void* wq_packed, const void* scales_packed, const void* zeros_packed,
+                           const uint16_t* X, uint16_t* Y, int M, int K, int N, int group, int path,
+                           void* workspace, size_t workspace_bytes, unsigned flags, void* stream) {
+  return gemm_impl(wq_packed, scales_packed, zeros_packed, X, Y, M, K, N, group, path, workspace,
+                   workspace_bytes, flags, stream);
+}
+
+w4a16_status w4a16_gemm_workspace_size(int M, int K, int N, int group, size_t* bytes) {
+  if (!bytes || N <= 0) return W4A16_ERR_INVALID_ARG;
   w4a16_status st = check_shape(M, K, group);
   if (st != W4A16_OK) return st;
   if (N > kMaxN) return W4A16_ERR_UNSUPPORTED;
-  if (!aligned16(wq_packed) || !aligned16(scales_packed) || !aligned16(zeros_packed) ||
-      !aligned16(X) || !aligned16(Y))
-    return W4A16_ERR_MISALIGNED;
-  {
-    const size_t ny = (size_t)N * M * 2;
-    if (overlap(Y, ny, X, (size_t)N * K * 2) ||
-        overlaps_weight(Y, ny, wq_packed, scales_packed, zeros_packed, packed_bytes(M, K)))
-      return W4A16_ERR_INVALID_ARG;
-  }
-  if (path == W4A16_PATH_AUTO) path = select_path_impl(M, K, N);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const uint8_t* wq = static_cast<const uint8_t*>(wq_packed);
-  const uint16_t* sp = static_cast<const uint16_t*>(scales_packed);
-  const uint8_t* zp = static_cast<const uint8_t*>(zeros_packed);
-  cudaError_t e = (path == W4A16_PATH_TC) ? launch_gemm_tc(wq, sp, zp, X, Y, M, K, N, s)
-                                          : launch_gemv(wq, sp, zp, X, Y, M, K, N, s);
-  return map_cuda(e);
+  *bytes = workspace_for(select_path_impl(M, K, N, true), M, K, N);
+  return W4A16_OK;
 }
 
 w4a16_status w4a16_gemm_qkv(const void* wq_packed, const void* scales_packed, const void* zeros_packed,
                             const uint16_t* X, const uint16_t* bias, int Mq, int Mk, int Mv, int K, int N,
                             int group, uint16_t* Yq, uint16_t* Yk, uint16_t* Yv, void* stream) {
-  if (!wq_packed || !scales_packed || !zeros_packed || !X || !Yq || !Yk || !Yv) return W4A16_ERR_INVALID_ARG;
-  if (Mq <= 0 || Mk <= 0 || Mv <= 0 || N <= 0) return W4A16_ERR_INVALID_ARG;
-  if ((long long)Mq + Mk + Mv > kMaxM) return W4A16_ERR_UNSUPPORTED;
-  const int M = Mq + Mk + Mv;
-  w4a16_status st = check_shape(M, K, group);
-  if (st != W4A16_OK) return st;
-  if (N > kMaxN) return W4A16_ERR_UNSUPPORTED;
-  if (!aligned16(wq_packed) || !aligned16(scales_packed) || !aligned16(zeros_packed) || !aligned16(X) ||
-      !aligned16(Yq) || !aligned16(Yk) || !aligned16(Yv) || (reinterpret_cast<uintptr_t>(bias) & 1u))
-    return W4A16_ERR_MISALIGNED;
-  {
-    const PackedBytes pb = packed_bytes(M, K);
-    const void* outs[3] = {Yq, Yk, Yv};
-    const size_t out_n[3] = {(size_t)N * Mq * 2, (size_t)N * Mk * 2, (size_t)N * Mv * 2};
-    for (int i = 0; i < 3; ++i) {
-      if (overlap(outs[i], out_n[i], X, (size_t)N * K * 2) || overlap(outs[i], out_n[i], bias, (size_t)M * 2) ||
-          overlaps_weight(outs[i], out_n[i], wq_packed, scales_packed, zeros_packed, pb))
-        return W4A16_ERR_INVALID_ARG;
-      for (int j = i + 1; j < 3; ++j)
-        if (overlap(outs[i], out_n[i], outs[j], out_n[j])) return W4A16_ERR_INVALID_ARG;
-    }
-  }
-  OutMap om;
-  om.y0 = Yq;
-  om.y1 = Yk;
-  om.y2 = Yv;
-  om.end0 = Mq;
-  om.end1 = Mq + Mk;
-  om.bias = bias;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const uint8_t* wq = static_cast<const uint8_t*>(wq_packed);
-  const uint16_t* sp = static_cast<const uint16_t*>(scales_packed);
-  const uint8_t* zp = static_cast<const uint8_t*>(zeros_packed);
-  cudaError_t e = (select_path_impl(M, K, N) == W4A16_PATH_TC)
-                      ? launch_gemm_tc(wq, sp, zp, X, nullptr, M, K, N, s, &om)
-                      : launch_gemv(wq, sp, zp, X, nullptr, M, K, N, s, &om);
-  return map_cuda(e);
+  return gemm_qkv_impl(wq_packed, scales_packed, zeros_packed, X, bias, Mq, Mk, Mv, K, N, group, Yq, Yk, Yv,
+                       nullptr, 0, 0u, stream);
+}
+
+w4a16_status w4a16_gemm_qkv_ws(const void* wq_packed, const void* scales_packed, const void* zeros_packed,
+                               const uint16_t* X, const uint16_t* bias, int Mq, int Mk, int Mv, int K, int N,
+                               int group, uint16_t* Yq, uint16_t* Yk, uint16_t* Yv, void* workspace,
+                               size_t workspace_bytes, unsigned flags, void* stream) {
+  return gemm_qkv_impl(wq_packed, scales_packed, zeros_packed, X, bias, Mq, Mk, Mv, K, N, group, Yq, Yk, Yv,
+                       workspace, workspace_bytes, flags, stream);
 }
 
 w4a16_status w4a16_gemm(const void* wq_packed, const void* scales_packed,
@@ -256,11 +327,12 @@ w4a16_status w4a16_dequant_debug(const void* wq_packed, const void* scales_packe
 w4a16_status w4a16_device_status(void* stream, int* status) {
   if (!status) return W4A16_ERR_INVALID_ARG;
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
-  int a = 0, b = 0;
+  int a = 0, b = 0, c = 0;
   if (e == cudaSuccess) e = read_and_clear_tc_status(&a);
   if (e == cudaSuccess) e = read_and_clear_gemv_status(&b);
+  if (e == cudaSuccess) e = read_and_clear_gvtc_status(&c);
   if (e != cudaSuccess) return map_cuda(e);
-  *status = (a || b) ? W4A16_ERR_TIMEOUT : W4A16_OK;
+  *status = (a || b || c) ? W4A16_ERR_TIMEOUT : W4A16_OK;
   return W4A16_OK;
 }
 

@@ -50,11 +50,6 @@
 #include "w4a16_internal.cuh"
 #include "sm100_ptx.cuh"
 
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
-#include <mutex>
-
 namespace w4a16 {
 
 __device__ int g_tc_status = 0;
@@ -514,62 +509,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
 
 // ------------------------------------------------------------------ host --
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-// X [N][K] fp16 viewed as a 3D tensor (64 k, N rows, K/64 slabs): the box
-// (64, BN, slabs) lands as `slabs` K-major 128-byte-swizzled tiles of BN x 64,
-// the layout the MMA's B descriptor describes.  Zero fill past N and K.
-cudaError_t make_x_map(CUtensorMap* map, const uint16_t* X, int N, int K, int BN, int slabs) {
-  auto fn = encode_fn();
-  if (!fn) return cudaErrorNotSupported;
-  cuuint64_t dims[3] = {64, (cuuint64_t)N, (cuuint64_t)(K / 64)};
-  cuuint64_t strides[2] = {(cuuint64_t)K * 2, 128};
-  cuuint32_t box[3] = {64, (cuuint32_t)BN, (cuuint32_t)slabs};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<uint16_t*>(X), dims, strides, box,
-                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
-
-int num_sms() {
-  static int cached[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (!cached[dev]) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    cached[dev] = n;
-  }
-  return cached[dev];
-}
-
 template <int BN, bool kMap>
 cudaError_t launch_bn(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p, const uint16_t* X,
                       uint16_t* Y, int M, int K, int N, cudaStream_t stream, const OutMap& om) {
   using C = Cfg<BN>;
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, kMap>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::atomic<unsigned long long> smem_set{0};
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(gemm_tc_kernel<BN, kMap>), C::kSmemBytes,
+                                    smem_set);
+  if (e != cudaSuccess) return e;
   CUtensorMap map;
-  cudaError_t e = make_x_map(&map, X, N, K, BN, C::kXSlabs);
+  e = make_x_map(&map, X, N, K, BN, C::kXSlabs);
   if (e != cudaSuccess) return e;
   const int tiles = ceil_div(M, kBM) * ceil_div(N, BN);
   const int grid = tiles < num_sms() ? tiles : num_sms();

@@ -241,30 +241,12 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   }
 }
 
-int sm_count() {
-  static int cached[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (!cached[dev]) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    cached[dev] = n;
-  }
-  return cached[dev];
-}
-
 template <int NT, bool kMap>
 cudaError_t launch_nt(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p, const uint16_t* X,
                       uint16_t* Y, int M, int K, int cl, cudaStream_t stream, const OutMap& om) {
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<NT, kMap>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         200 * 1024);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::atomic<unsigned long long> smem_set{0};
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(gemv_kernel<NT, kMap>), 200 * 1024, smem_set);
+  if (e != cudaSuccess) return e;
   const int blocks = ceil_div(M, kRowBlock);
   const GvLayout L = gv_layout(NT, ceil_div(K / kGroup, cl), cl);
   cudaLaunchConfig_t cfg = {};
@@ -319,7 +301,7 @@ cudaError_t launch_gemv(const uint8_t* wq, const uint16_t* scales, const uint8_t
                         cudaStream_t stream, const OutMap* om) {
   for (int n0 = 0; n0 < N; n0 += kGemvMaxTokens) {
     const int nt = std::min(kGemvMaxTokens, N - n0);
-    const int cl = gemv_cluster_size(M, K, sm_count(), nt);
+    const int cl = gemv_cluster_size(M, K, num_sms(), nt);
     if (nt * ceil_div(K / kGroup, cl) * kGroup * 2 > kMaxXSmem) return cudaErrorNotSupported;
     const uint16_t* Xn = X + (size_t)n0 * K;
     uint16_t* Yn = om ? nullptr : Y + (size_t)n0 * M;

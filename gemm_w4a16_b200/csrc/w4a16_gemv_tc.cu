@@ -1,0 +1,467 @@
+// Decode GEMV / few-token product on the tensor cores, with the weight
+// stream split evenly over every SM (sm_100a).
+//
+// "PerfXLLM on Snapdragon 8 Gen2", section 3.3 item 2: with one token (or a
+// few) the product is a GEMV, bound by memory; the goal is to keep the weight
+// stream at memory speed and hide the arithmetic, tiling the weight along
+// both its rows and K so that every compute unit has a share.  On sm_100a:
+//
+//  * Unit = (128-row block b, quantisation group g): 8 KB of codes, 256 B of
+//    scales and 64 B of zeros, each contiguous in its packed array, units in
+//    block-major order.  CTA c of G takes units [c U / G, (c + 1) U / G) of
+//    the U = blocks x groups units, so every SM streams the same bytes for
+//    any M and K (a block may be split between consecutive CTAs).
+//  * One producer thread copies each unit (three bulk copies) and its
+//    activation tile (one TMA copy of BN tokens x 128 k, 128-byte swizzle,
+//    the K-major layout the MMA reads; tokens past N zero-filled) into a
+//    ring of shared-memory stages.
+//  * Dequantiser groups of four warps (thread = weight row) take the units in
+//    turn: exact in-register dequant (dequant_word), tcgen05.st of the row's
+//    128 fp16 weights into a TMEM A slot.  Issuer warps take the units in
+//    turn and run eight tcgen05.mma kind::f16 (M = 128, N = BN, K = 16) from
+//    the A slot and the X tile into their own fp32 accumulator in TMEM (one
+//    issuing thread completes a small-N MMA only every few tens of cycles,
+//    so several issue side by side).
+//  * Epilogue warps (one per TMEM lane quarter): at the end of each of the
+//    CTA's blocks, tcgen05.ld of the issuers' accumulators, summed in issuer
+//    order.  A block the CTA covers entirely is rounded once to fp16 and
+//    written.  Otherwise the fp32 partial goes to the caller's workspace; the
+//    last CTA to finish the block's lane quarter (an atomic counter per block
+//    and quarter) adds the partials of all of the block's CTAs in CTA order,
+//    rounds once and writes Y, then resets the counter.  Deterministic, no
+//    floating-point atomics, and no CTA ever waits for another.
+//  * Footprint: about 100 KB of shared memory, 256 TMEM columns and at most
+//    32 K registers, so two CTAs fit on an SM.  With programmatic dependent
+//    launch the next call's CTAs then start streaming their weights while
+//    this call's CTAs finish; X, Y and the workspace are touched only after
+//    the grid dependency wait.
+//  * Every mbarrier wait is bounded: on expiry the kernel records a timeout
+//    in a device status word, stops, drains its copies and MMAs, frees TMEM
+//    and returns.
+#include "w4a16_internal.cuh"
+#include "sm100_ptx.cuh"
+
+namespace w4a16 {
+
+__device__ int g_gvtc_status = 0;
+
+namespace {
+
+constexpr int kUnitCodes = kRowBlock * kGroup / 2;    // 8192 B of codes per unit
+constexpr int kUnitS = kRowBlock * 2;                 // 256 B of scales
+constexpr int kUnitZ = kRowBlock / 2;                 // 64 B of zeros
+constexpr int kUnitW = kUnitCodes + kUnitS + kUnitZ;  // one weight stage
+constexpr int kACols = kGroup / 2;                    // TMEM columns of one unit's A (fp16 pairs)
+
+// True when n = t a + u b for some t >= 1, u >= 0.
+__host__ __device__ constexpr bool reachable(int n, int a, int b) {
+  for (int t = 1; t * a <= n; ++t)
+    if ((n - t * a) % b == 0) return true;
+  return false;
+}
+
+template <int BN_, int DQ, int ISS, int ASLOTS, int ACCB, int STAGES>
+struct GtCfg {
+  static constexpr int BN = BN_;
+  static constexpr int kDq = DQ;            // dequantiser groups of four warps
+  static constexpr int kIss = ISS;          // MMA issuer warps, one accumulator each
+  static constexpr int kASlots = ASLOTS;    // TMEM A slots, one unit each
+  static constexpr int kAccBufs = ACCB;     // accumulator sets
+  static constexpr int kStages = STAGES;    // shared-memory stages, one unit each
+  static constexpr int kXBytes = BN * kGroup * 2;
+  static constexpr int kAccCols = kIss * BN;
+  static constexpr int kACol0 = kAccBufs * kAccCols;
+  static constexpr int kTmemCols = 256;
+  static constexpr uint32_t kIdesc = ptx::idesc_f16_f32(kRowBlock, BN);
+  // Warps: 0..3 epilogue, 4..4+kIss-1 issuers, then the producer, then the
+  // dequantiser groups.
+  static constexpr int kFirstIss = 4;
+  static constexpr int kProducer = kFirstIss + kIss;
+  static constexpr int kFirstDq = kProducer + 1;
+  static constexpr int kThreads = (kFirstDq + 4 * kDq) * 32;
+  // Shared memory: X ring (1024-byte aligned tiles), weight ring, barriers.
+  static constexpr int kXOff = 0;
+  static constexpr int kWOff = kStages * kXBytes;
+  static constexpr int kBarOff = kWOff + kStages * kUnitW;
+  static constexpr int kNumBars = 3 * kStages + 2 * kASlots + 2 * kAccBufs + 1;
+  static constexpr int kSmemBytes = kBarOff + 8 * kNumBars + 16 + 1024;
+
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 64, "MMA N");
+  static_assert(kACol0 + kASlots * kACols <= kTmemCols, "TMEM budget");
+  static_assert(kSmemBytes <= 113 * 1024, "two CTAs per SM");
+  static_assert(kXBytes % 1024 == 0, "swizzled X tiles stay 1024-byte aligned");
+  // A parity wait cannot tell a phase from the one two steps later.  The
+  // waits below stay exact when each waiter already knows the phase before
+  // the one it waits for is complete:
+  //  - stage barriers: every dequantiser group and every issuer sees each
+  //    stage it uses, in order (kDq | kStages, kIss | kStages);
+  //  - an A slot's "empty" barrier: the fill before the previous one was
+  //    freed, which a group knows from its own earlier wait plus the in-order
+  //    commits of one issuer (kASlots = t kDq + u kIss, t >= 1);
+  //  - an A slot's "full" barrier: the fill before the one awaited is known
+  //    to be done from the issuer's own earlier waits and the in-order fills
+  //    of one group (kASlots = t kIss + u kDq, t >= 1).
+  static_assert(kStages % kDq == 0 && kStages % kIss == 0, "stage ring");
+  static_assert(reachable(kASlots, kDq, kIss) && reachable(kASlots, kIss, kDq), "A-slot phases");
+};
+
+// Units [start(c), start(c + 1)) belong to CTA c.
+__host__ __device__ __forceinline__ long long unit_start(long long U, int G, int c) {
+  return U * c / G;
+}
+
+// The CTA whose range holds unit u.
+__host__ __device__ __forceinline__ int cta_of(long long U, int G, long long u) {
+  return (int)(((u + 1) * G - 1) / U);
+}
+
+template <class C, bool kMap>
+__global__ void __launch_bounds__(C::kThreads, 2)
+gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __restrict__ wq,
+               const uint16_t* __restrict__ s_p, const uint8_t* __restrict__ z_p, uint16_t* __restrict__ Y,
+               int M, int K, int N, uint32_t* __restrict__ ws_cnt, float* __restrict__ ws_part, OutMap om) {
+  constexpr int BN = C::BN;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* wfull = bars;
+  uint64_t* xfull = wfull + S;
+  uint64_t* empty = xfull + S;
+  uint64_t* a_full = empty + S;
+  uint64_t* a_empty = a_full + C::kASlots;
+  uint64_t* acc_full = a_empty + C::kASlots;
+  uint64_t* acc_empty = acc_full + C::kAccBufs;
+  uint64_t* drain = acc_empty + C::kAccBufs;
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_ptr + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int kg = K / kGroup;
+  const int nb = ceil_div(M, kRowBlock);
+  const long long U = (long long)nb * kg;
+  const int G = (int)gridDim.x;
+  const int c = (int)blockIdx.x;
+  const int u0 = (int)unit_start(U, G, c);
+  const int u1 = (int)unit_start(U, G, c + 1);
+  const int L = u1 - u0;                      // units of this CTA (>= 1: G <= U)
+  const int b_first = u0 / kg;
+  const int nblk = (u1 - 1) / kg - b_first + 1;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      ptx::mbar_init(&wfull[i], 1);
+      ptx::mbar_init(&xfull[i], 1);
+      ptx::mbar_init(&empty[i], 5);           // the 4 warps of one group + one issuer's commit
+    }
+    for (int i = 0; i < C::kASlots; ++i) {
+      ptx::mbar_init(&a_full[i], 4);
+      ptx::mbar_init(&a_empty[i], 1);
+    }
+    for (int i = 0; i < C::kAccBufs; ++i) {
+      ptx::mbar_init(&acc_full[i], C::kIss);
+      ptx::mbar_init(&acc_empty[i], 4);
+    }
+    ptx::mbar_init(drain, C::kIss);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&tmap_x);
+  }
+  if (warp == C::kFirstIss) {
+    ptx::tmem_alloc(tmem_ptr, C::kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  ptx::griddep_launch_dependents();
+  const uint32_t tmem = *tmem_ptr;
+
+  if (warp == C::kProducer) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint8_t* wsrc = wq + (size_t)u0 * kUnitCodes;
+      const uint8_t* ssrc = reinterpret_cast<const uint8_t*>(s_p) + (size_t)u0 * kUnitS;
+      const uint8_t* zsrc = z_p + (size_t)u0 * kUnitZ;
+      auto issue_w = [&](int i) {
+        uint8_t* dst = smem + C::kWOff + (i % S) * kUnitW;
+        uint64_t* bar = &wfull[i % S];
+        ptx::mbar_arrive_expect_tx(bar, kUnitW);
+        ptx::bulk_load(dst, wsrc + (size_t)i * kUnitCodes, kUnitCodes, bar);
+        ptx::bulk_load(dst + kUnitCodes, ssrc + (size_t)i * kUnitS, kUnitS, bar);
+        ptx::bulk_load(dst + kUnitCodes + kUnitS, zsrc + (size_t)i * kUnitZ, kUnitZ, bar);
+      };
+      auto issue_x = [&](int i) {
+        uint64_t* bar = &xfull[i % S];
+        ptx::mbar_arrive_expect_tx(bar, C::kXBytes);
+        ptx::tma_load_3d(smem + C::kXOff + (i % S) * C::kXBytes, &tmap_x, bar, 0, 0, 2 * ((u0 + i) % kg));
+      };
+      // The weights do not depend on the kernels before this one in the
+      // stream: the first stages' weights are requested before the grid
+      // dependency wait, the activations only after it.
+      const int pre = L < S ? L : S;
+      for (int i = 0; i < pre; ++i) issue_w(i);
+      ptx::griddep_wait();
+      for (int i = 0; i < pre; ++i) issue_x(i);
+      int issued = pre;
+      for (int i = pre; i < L; ++i) {
+        if (!wait_bar(&empty[i % S], (uint32_t)(((i / S) & 1) ^ 1), abort_flag, &g_gvtc_status)) break;
+        issue_w(i);
+        issue_x(i);
+        issued = i + 1;
+      }
+      // Drain: every copy issued into this CTA's shared memory has landed.
+      for (int i = issued - S > 0 ? issued - S : 0; i < issued; ++i) {
+        wait_bar(&wfull[i % S], (uint32_t)((i / S) & 1), abort_flag, &g_gvtc_status, false);
+        wait_bar(&xfull[i % S], (uint32_t)((i / S) & 1), abort_flag, &g_gvtc_status, false);
+      }
+    }
+  } else if (warp >= C::kFirstIss && warp < C::kFirstIss + C::kIss) {
+    // --------------------------------------------------------- MMA issuers
+    // Issuer ii takes the CTA's units i = ii, ii + kIss, ...; per block it
+    // accumulates its units into its own BN columns of the block's
+    // accumulator set, and arrives (commit, or a plain arrive when it had
+    // no unit there) on the set's "full" barrier.
+    const int ii = warp - C::kFirstIss;
+    if (lane == 0) {
+      const uint64_t desc0 = ptx::smem_desc_sw128(ptx::smem_addr(smem + C::kXOff));
+      bool ok = true;
+      for (int bi = 0; ok && bi < nblk; ++bi) {
+        const int b = b_first + bi;
+        const int i0 = (b * kg > u0 ? b * kg : u0) - u0;
+        const int i1 = ((b + 1) * kg < u1 ? (b + 1) * kg : u1) - u0;
+        const int buf = bi % C::kAccBufs;
+        if (!wait_bar(&acc_empty[buf], (uint32_t)(((bi / C::kAccBufs) & 1) ^ 1), abort_flag, &g_gvtc_status))
+          break;
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem + buf * C::kAccCols + ii * BN;
+        bool first = true;
+        for (int i = i0 + ((ii - i0 % C::kIss) + C::kIss) % C::kIss; i < i1; i += C::kIss) {
+          const int st = i % S;
+          const int a = i % C::kASlots;
+          if (!wait_bar(&xfull[st], (uint32_t)((i / S) & 1), abort_flag, &g_gvtc_status) ||
+              !wait_bar(&a_full[a], (uint32_t)((i / C::kASlots) & 1), abort_flag, &g_gvtc_status)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint64_t desc = desc0 + (uint64_t)((st * C::kXBytes) >> 4);
+          ptx::mma_ts_f16_slot<8>(d_tmem, tmem + C::kACol0 + a * kACols, desc, C::kIdesc, first ? 0u : 1u,
+                                  &a_empty[a], (BN * 128) >> 4);
+          ptx::mma_commit(&empty[st]);
+          first = false;
+        }
+        if (!ok) break;
+        if (first) ptx::mbar_arrive(&acc_full[buf]);
+        else ptx::mma_commit(&acc_full[buf]);
+      }
+      // Drain: all MMAs issued by this thread have completed.
+      ptx::mma_commit(drain);
+      wait_bar(drain, 0, abort_flag, &g_gvtc_status, false);
+    }
+  } else if (warp >= C::kFirstDq) {
+    // -------------------------------------------------------- dequantisers
+    // Group gi takes units i = gi, gi + kDq, ...; thread = row of the block.
+    const int gi = (warp - C::kFirstDq) >> 2;
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t a_lane = tmem + ((uint32_t)(quad * 32) << 16) + C::kACol0;
+    const uint32_t wring = ptx::smem_addr(smem + C::kWOff);
+    for (int i = gi; i < L; i += C::kDq) {
+      const int st = i % S;
+      if (!wait_bar_warp(&wfull[st], (uint32_t)((i / S) & 1), abort_flag, &g_gvtc_status)) break;
+      const uint32_t base = wring + st * kUnitW;
+      const uint4 v0 = ptx::lds_v4(base + 0 * 2048 + row * 16);
+      const uint4 v1 = ptx::lds_v4(base + 1 * 2048 + row * 16);
+      const uint4 v2 = ptx::lds_v4(base + 2 * 2048 + row * 16);
+      const uint4 v3 = ptx::lds_v4(base + 3 * 2048 + row * 16);
+      const uint32_t sv = ptx::lds_u16(base + kUnitCodes + row * 2);
+      const uint32_t zb = ptx::lds_u8(base + kUnitCodes + kUnitS + (row >> 1));
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&empty[st]);
+      const GroupConsts gc = make_group_consts((zb >> ((row & 1) * 4)) & 0xFu, (uint16_t)sv);
+      const int a = i % C::kASlots;
+      const uint32_t dst = a_lane + a * kACols;
+      uint32_t h[16];
+      dequant_word(v0.x, gc, &h[0]);
+      dequant_word(v0.y, gc, &h[4]);
+      dequant_word(v0.z, gc, &h[8]);
+      dequant_word(v0.w, gc, &h[12]);
+      if (!wait_bar_warp(&a_empty[a], (uint32_t)(((i / C::kASlots) & 1) ^ 1), abort_flag, &g_gvtc_status)) break;
+      ptx::tc_fence_after();
+      ptx::tmem_st_x16(dst, h);
+      dequant_word(v1.x, gc, &h[0]);
+      dequant_word(v1.y, gc, &h[4]);
+      dequant_word(v1.z, gc, &h[8]);
+      dequant_word(v1.w, gc, &h[12]);
+      ptx::tmem_st_x16(dst + 16, h);
+      dequant_word(v2.x, gc, &h[0]);
+      dequant_word(v2.y, gc, &h[4]);
+      dequant_word(v2.z, gc, &h[8]);
+      dequant_word(v2.w, gc, &h[12]);
+      ptx::tmem_st_x16(dst + 32, h);
+      dequant_word(v3.x, gc, &h[0]);
+      dequant_word(v3.y, gc, &h[4]);
+      dequant_word(v3.z, gc, &h[8]);
+      dequant_word(v3.w, gc, &h[12]);
+      ptx::tmem_st_x16(dst + 48, h);
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&a_full[a]);
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ epilogue
+    const int quad = warp;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    // Outputs and the workspace may still be in use by the kernel before
+    // this one until the grid dependency is resolved.
+    ptx::griddep_wait();
+    for (int bi = 0; bi < nblk; ++bi) {
+      const int b = b_first + bi;
+      const int i0 = (b * kg > u0 ? b * kg : u0) - u0;
+      const int i1 = ((b + 1) * kg < u1 ? (b + 1) * kg : u1) - u0;
+      const int span = i1 - i0;
+      const int buf = bi % C::kAccBufs;
+      const int m = b * kRowBlock + row;
+      RowDst rd = {};
+      if constexpr (kMap) {
+        if (m < M) rd = row_dst(om, M, m);
+      }
+      if (!wait_bar_warp(&acc_full[buf], (uint32_t)((bi / C::kAccBufs) & 1), abort_flag, &g_gvtc_status)) break;
+      ptx::tc_fence_after();
+      float acc[BN];
+      bool have = false;
+#pragma unroll
+      for (int p = 0; p < C::kIss; ++p) {
+        // Issuer p owns a unit of this block iff one of i0 .. i1 - 1 is p mod kIss.
+        if (span < C::kIss && ((p - i0 % C::kIss) + C::kIss) % C::kIss >= span) continue;
+#pragma unroll
+        for (int h = 0; h < BN / 16; ++h) {
+          uint32_t v[16];
+          ptx::tmem_ld_x16(lane_base + buf * C::kAccCols + p * BN + h * 16, v);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) acc[h * 16 + j] = have ? acc[h * 16 + j] + __uint_as_float(v[j])
+                                                              : __uint_as_float(v[j]);
+        }
+        have = true;
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&acc_empty[buf]);
+
+      bool write = span == kg;
+      if (!write) {
+        // Partial of a split block: this CTA's fp32 share to the workspace;
+        // the last of the block's CTAs (per lane quarter) sums them all.
+        const int slot = bi == 0 ? 0 : 1;
+        float* part = ws_part + (size_t)(c * 2 + slot) * N * kRowBlock + row;
+#pragma unroll
+        for (int n = 0; n < BN; ++n)
+          if (n < N) part[(size_t)n * kRowBlock] = acc[n];
+        __threadfence();
+        __syncwarp();
+        uint32_t old = 0;
+        if (lane == 0) old = ptx::atom_add_acq_rel_gpu(&ws_cnt[b * 4 + quad], 1u);
+        old = __shfl_sync(0xffffffffu, old, 0);
+        const int cf = cta_of(U, G, (long long)b * kg);
+        const int cl = cta_of(U, G, (long long)(b + 1) * kg - 1);
+        if (old == (uint32_t)(cl - cf)) {
+          __threadfence();
+#pragma unroll
+          for (int n = 0; n < BN; ++n) acc[n] = 0.f;
+          for (int cc = cf; cc <= cl; ++cc) {
+            const int sl = (long long)b == unit_start(U, G, cc) / kg ? 0 : 1;
+            const float* pp = ws_part + (size_t)(cc * 2 + sl) * N * kRowBlock + row;
+#pragma unroll
+            for (int n = 0; n < BN; ++n)
+              if (n < N) acc[n] += __ldcg(pp + (size_t)n * kRowBlock);
+          }
+          if (lane == 0) ws_cnt[b * 4 + quad] = 0u;
+          write = true;
+        }
+      }
+      if (write && m < M) {
+#pragma unroll
+        for (int n = 0; n < BN; ++n) {
+          if (n < N) {
+            if constexpr (kMap) store_row(rd, om.bias != nullptr, n, acc[n]);
+            else Y[(size_t)n * M + m] = __half_as_ushort(__float2half_rn(acc[n]));
+          }
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == C::kFirstIss) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// Few tokens: three dequantiser groups, three issuers, one accumulator set.
+using Cfg16 = GtCfg<16, 3, 3, 3, 1, 6>;
+
+int grid_for(int M, int K) {
+  const long long U = (long long)ceil_div(M, kRowBlock) * (K / kGroup);
+  const int sms = num_sms();
+  return (int)(U < sms ? U : sms);
+}
+
+template <class C, bool kMap>
+cudaError_t launch_cfg(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p, const uint16_t* X,
+                       uint16_t* Y, int M, int K, int N, void* ws, bool pdl, cudaStream_t stream,
+                       const OutMap& om) {
+  static std::atomic<unsigned long long> smem_set{0};
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(gemv_tc_kernel<C, kMap>), C::kSmemBytes,
+                                    smem_set);
+  if (e != cudaSuccess) return e;
+  CUtensorMap map;
+  e = make_x_map(&map, X, N, K, C::BN, 2);
+  if (e != cudaSuccess) return e;
+  uint32_t* cnt = static_cast<uint32_t*>(ws);
+  float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + gemv_tc_counter_bytes(M));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid_for(M, K), 1, 1);
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, gemv_tc_kernel<C, kMap>, map, wq, s_p, z_p, Y, M, K, N, cnt, part, om);
+}
+
+}  // namespace
+
+size_t gemv_tc_counter_bytes(int M) {
+  return ((size_t)ceil_div(M, kRowBlock) * 4 * sizeof(uint32_t) + 255) / 256 * 256;
+}
+
+size_t gemv_tc_workspace_bytes(int M, int K, int N) {
+  return gemv_tc_counter_bytes(M) + (size_t)grid_for(M, K) * 2 * N * kRowBlock * sizeof(float);
+}
+
+cudaError_t launch_gemv_tc(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros, const uint16_t* X,
+                           uint16_t* Y, int M, int K, int N, void* workspace, bool pdl, cudaStream_t stream,
+                           const OutMap* om) {
+  if (N > kGemvTcMaxTokens) return cudaErrorNotSupported;
+  if (om) return launch_cfg<Cfg16, true>(wq, scales, zeros, X, nullptr, M, K, N, workspace, pdl, stream, *om);
+  return launch_cfg<Cfg16, false>(wq, scales, zeros, X, Y, M, K, N, workspace, pdl, stream, OutMap{});
+}
+
+cudaError_t read_and_clear_gvtc_status(int* v) {
+  cudaError_t e = cudaMemcpyFromSymbol(v, g_gvtc_status, sizeof(int));
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_gvtc_status, &zero, sizeof(int));
+}
+
+}  // namespace w4a16

@@ -5,9 +5,12 @@
 // a warp reads 32 consecutive rows' chunks as 512 contiguous bytes.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
+
+#include <atomic>
 
 #include "../../include/w4a16.h"
 
@@ -147,6 +150,27 @@ __device__ __forceinline__ void store_row(const RowDst& d, bool has_bias, int n,
 
 // ------------------------------------------------------- launch helpers ----
 
+// SM count of the current device (cached per device; 148 if it cannot be read).
+int num_sms();
+
+// Tensor map of X [N][K] fp16 for the tensor-core kernels: boxes of 64 k x
+// box_rows tokens x `slabs` 64-k slabs, 128-byte swizzle, zero fill past N.
+cudaError_t make_x_map(CUtensorMap* map, const uint16_t* X, int N, int K, int box_rows, int slabs);
+
+// Raise a kernel's dynamic shared-memory limit on the current device, once
+// per device (bit `dev` of `done`).  Two threads racing on the first call
+// both set the same value, which is harmless.
+inline cudaError_t ensure_smem_limit(const void* fn, int bytes, std::atomic<unsigned long long>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+  return e;
+}
+
 // GEMV (CUDA cores): N in 1..kGemvMaxTokens per launch.
 constexpr int kGemvMaxTokens = 4;
 
@@ -177,10 +201,24 @@ cudaError_t launch_gemm_tc(const uint8_t* wq, const uint16_t* scales, const uint
                            const uint16_t* X, uint16_t* Y, int M, int K, int N,
                            cudaStream_t stream, const OutMap* om = nullptr);
 
+// Decode GEMV / few-token product on the tensor cores, split along the
+// weight stream over every SM (N in 1..kGemvTcMaxTokens).  The caller's
+// workspace holds one counter per (row block, lane quarter), zero between
+// calls, then the fp32 partials of the blocks split between CTAs.  With pdl
+// the launch may overlap the previous kernel in the stream: the weights are
+// read before the grid dependency wait, X, Y and the workspace after it.
+constexpr int kGemvTcMaxTokens = 16;
+size_t gemv_tc_counter_bytes(int M);
+size_t gemv_tc_workspace_bytes(int M, int K, int N);
+cudaError_t launch_gemv_tc(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros, const uint16_t* X,
+                           uint16_t* Y, int M, int K, int N, void* workspace, bool pdl, cudaStream_t stream,
+                           const OutMap* om = nullptr);
+
 // Read-and-clear of the per-kernel-family device status words (1 = a bounded
 // wait ran out).
 cudaError_t read_and_clear_tc_status(int* v);
 cudaError_t read_and_clear_gemv_status(int* v);
+cudaError_t read_and_clear_gvtc_status(int* v);
 
 // Diagnostic: a kernel whose bounded wait must run out (see
 // w4a16_selftest_wait_timeout).

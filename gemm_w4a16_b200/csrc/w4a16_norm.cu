@@ -131,17 +131,9 @@ cudaError_t launch_add_rmsnorm(const uint16_t* h, const uint16_t* d, const uint1
                                int N, int K, uint16_t* r_out, uint16_t* X, cudaStream_t stream) {
   const size_t smem = (size_t)K * 2;
   if (smem > 48 * 1024) {
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static std::atomic<unsigned long long> smem_set{0};
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(add_rmsnorm_kernel), kMaxNormK * 2, smem_set);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorNotSupported;
-    if (!attr_set[dev]) {
-      e = cudaFuncSetAttribute(add_rmsnorm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               kMaxNormK * 2);
-      if (e != cudaSuccess) return e;
-      attr_set[dev] = true;
-    }
   }
   add_rmsnorm_kernel<<<(unsigned)N, kNormThreads, smem, stream>>>(h, d, gamma, eps, K, r_out, X);
   return cudaGetLastError();

@@ -15,14 +15,17 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libw4a16.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_CUDA, ERR_TIMEOUT = range(6)
-PATH_AUTO, PATH_GEMV, PATH_TC = 0, 1, 2
+PATH_AUTO, PATH_GEMV, PATH_TC, PATH_GEMV_TC = 0, 1, 2, 3
+FLAG_EARLY_WEIGHTS = 1
+GEMV_TC_MAX_TOKENS = 16
 GROUP = 128
 
 EXPORTED = (
     "w4a16_status_string", "w4a16_packed_sizes", "w4a16_pack", "w4a16_gemm",
     "w4a16_gemm_ex", "w4a16_select_path", "w4a16_dequant_debug",
     "w4a16_device_status", "w4a16_selftest_wait_timeout", "w4a16_quantize", "w4a16_gemm_qkv",
-    "w4a16_add_rmsnorm",
+    "w4a16_add_rmsnorm", "w4a16_gemm_workspace_size", "w4a16_gemm_ws", "w4a16_gemm_qkv_ws",
+    "w4a16_select_path_ws",
 )
 
 _lib = None
@@ -30,6 +33,8 @@ _lock = threading.Lock()
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
 _szp = ctypes.POINTER(ctypes.c_size_t)
+_sz = ctypes.c_size_t
+_u = ctypes.c_uint
 
 
 class W4A16Error(RuntimeError):
@@ -66,6 +71,15 @@ def lib():
             L.w4a16_gemm_ex.restype = _i
             L.w4a16_select_path.argtypes = [_i, _i, _i]
             L.w4a16_select_path.restype = _i
+            L.w4a16_select_path_ws.argtypes = [_i, _i, _i]
+            L.w4a16_select_path_ws.restype = _i
+            L.w4a16_gemm_workspace_size.argtypes = [_i, _i, _i, _i, _szp]
+            L.w4a16_gemm_workspace_size.restype = _i
+            L.w4a16_gemm_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _sz, _u, _vp]
+            L.w4a16_gemm_ws.restype = _i
+            L.w4a16_gemm_qkv_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp,
+                                            _vp, _sz, _u, _vp]
+            L.w4a16_gemm_qkv_ws.restype = _i
             L.w4a16_dequant_debug.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _vp]
             L.w4a16_dequant_debug.restype = _i
             L.w4a16_device_status.argtypes = [_vp, ctypes.POINTER(_i)]
@@ -107,6 +121,59 @@ def packed_sizes(M: int, K: int, group: int = GROUP):
 
 def select_path(M: int, K: int, N: int) -> int:
     return int(lib().w4a16_select_path(M, K, N))
+
+
+def select_path_ws(M: int, K: int, N: int) -> int:
+    """The path w4a16_gemm_ws takes when given a workspace."""
+    return int(lib().w4a16_select_path_ws(M, K, N))
+
+
+def workspace_size(M: int, K: int, N: int, group: int = GROUP) -> int:
+    """Bytes of workspace w4a16_gemm_ws needs for these sizes on the current
+    device (0 when its automatic choice needs none)."""
+    n = ctypes.c_size_t()
+    _check(lib().w4a16_gemm_workspace_size(M, K, N, group, ctypes.byref(n)), "w4a16_gemm_workspace_size")
+    return n.value
+
+
+class Workspace:
+    """A zero-filled device buffer for the workspace entry points.  The
+    kernels leave it zero-filled after every completed call, so one buffer
+    serves any number of calls in one stream; `ensure` grows it (outside
+    CUDA-graph capture) to the size a call needs."""
+
+    def __init__(self, device=None, nbytes: int = 0):
+        import torch
+
+        self.device = torch.device("cuda") if device is None else torch.device(device)
+        self.buf = torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=self.device)
+
+    @property
+    def nbytes(self) -> int:
+        return self.buf.numel()
+
+    def ensure(self, nbytes: int) -> "Workspace":
+        import torch
+
+        if nbytes > self.buf.numel():
+            self.buf = torch.zeros(nbytes, dtype=torch.uint8, device=self.device)
+        return self
+
+    def clear(self) -> None:
+        """Zero-fill again (needed only after a call that timed out)."""
+        self.buf.zero_()
+
+
+_default_ws = {}
+
+
+def default_workspace(device, stream) -> Workspace:
+    """One workspace per (device, stream): calls in one stream never overlap."""
+    key = (device.index, stream.cuda_stream)
+    ws = _default_ws.get(key)
+    if ws is None:
+        ws = _default_ws[key] = Workspace(device)
+    return ws
 
 
 @dataclass
@@ -206,11 +273,8 @@ def gemm_ex(w: PackedWeight, X, Y=None, path: int = PATH_AUTO, stream=None):
     return Y
 
 
-def gemm_qkv(w: PackedWeight, X, splits, bias=None, out=None, stream=None):
-    """(Yq, Yk, Yv) token-major fp16 for a weight whose rows are three stacked
-    projections of widths splits = (Mq, Mk, Mv), each row plus bias[m] (fp16
-    [M] or None), via w4a16_gemm_qkv.  out: three contiguous CUDA fp16 tensors
-    [N, Mq], [N, Mk], [N, Mv] to write, or None to allocate them."""
+def _qkv_outs(w: PackedWeight, X, splits, bias, out):
+    """Checked (Yq, Yk, Yv) for the fused QKV form: `out`, or new tensors."""
     import torch
 
     N, K = X.shape
@@ -219,18 +283,67 @@ def gemm_qkv(w: PackedWeight, X, splits, bias=None, out=None, stream=None):
         raise ValueError("splits must add up to the weight's rows")
     if K != w.K or X.dtype != torch.float16 or not X.is_cuda or not X.is_contiguous():
         raise ValueError("X must be a contiguous CUDA fp16 [N, K] tensor")
-    if bias is not None and (bias.dtype != torch.float16 or not bias.is_cuda or bias.numel() != w.M):
-        raise ValueError("bias must be a CUDA fp16 tensor of M values")
+    if bias is not None and (bias.dtype != torch.float16 or not bias.is_cuda or bias.numel() != w.M
+                             or not bias.is_contiguous()):
+        raise ValueError("bias must be a contiguous CUDA fp16 tensor of M values")
     if out is None:
-        outs = [torch.empty((N, m), dtype=torch.float16, device=X.device) for m in (Mq, Mk, Mv)]
-    else:
-        outs = list(out)
-        if len(outs) != 3 or any(o.dtype != torch.float16 or not o.is_cuda or not o.is_contiguous()
-                                 or tuple(o.shape) != (N, m) for o, m in zip(outs, (Mq, Mk, Mv))):
-            raise ValueError("out must be three contiguous CUDA fp16 tensors [N, Mq], [N, Mk], [N, Mv]")
+        return [torch.empty((N, m), dtype=torch.float16, device=X.device) for m in (Mq, Mk, Mv)]
+    outs = list(out)
+    if len(outs) != 3 or any(o.dtype != torch.float16 or not o.is_cuda or not o.is_contiguous()
+                             or tuple(o.shape) != (N, m) for o, m in zip(outs, (Mq, Mk, Mv))):
+        raise ValueError("out must be three contiguous CUDA fp16 tensors [N, Mq], [N, Mk], [N, Mv]")
+    return outs
+
+
+def gemm_qkv(w: PackedWeight, X, splits, bias=None, out=None, stream=None):
+    """(Yq, Yk, Yv) token-major fp16 for a weight whose rows are three stacked
+    projections of widths splits = (Mq, Mk, Mv), each row plus bias[m] (fp16
+    [M] or None), via w4a16_gemm_qkv.  out: three contiguous CUDA fp16 tensors
+    [N, Mq], [N, Mk], [N, Mv] to write, or None to allocate them."""
+    N, K = X.shape
+    outs = _qkv_outs(w, X, splits, bias, out)
+    Mq, Mk, Mv = (int(v) for v in splits)
     _check(lib().w4a16_gemm_qkv(_ptr(w.wq), _ptr(w.scales), _ptr(w.zeros), _ptr(X), _ptr(bias), Mq, Mk, Mv,
                                 K, N, w.group, _ptr(outs[0]), _ptr(outs[1]), _ptr(outs[2]),
                                 _stream_ptr(stream)), "w4a16_gemm_qkv")
+    return tuple(outs)
+
+
+def gemm_ws(w: PackedWeight, X, Y=None, path: int = PATH_AUTO, workspace: Workspace | None = None,
+            flags: int = 0, stream=None):
+    """Y [N, M] fp16 = X [N, K] fp16 . dequant(W)^T via w4a16_gemm_ws, with a
+    workspace (the caller's, or one kept per device and stream)."""
+    import torch
+
+    N, K = X.shape
+    if K != w.K or X.dtype != torch.float16 or not X.is_cuda or not X.is_contiguous():
+        raise ValueError("X must be a contiguous CUDA fp16 [N, K] tensor")
+    if Y is None:
+        Y = torch.empty((N, w.M), dtype=torch.float16, device=X.device)
+    st = torch.cuda.current_stream(X.device) if stream is None else stream
+    ws = workspace if workspace is not None else default_workspace(X.device, st)
+    need = workspace_size(w.M, K, N, w.group) if path in (PATH_AUTO, PATH_GEMV_TC) else 0
+    ws.ensure(need)
+    _check(lib().w4a16_gemm_ws(_ptr(w.wq), _ptr(w.scales), _ptr(w.zeros), _ptr(X), _ptr(Y), w.M, K, N,
+                               w.group, path, _ptr(ws.buf), ws.nbytes, int(flags), _vp(st.cuda_stream)),
+           "w4a16_gemm_ws")
+    return Y
+
+
+def gemm_qkv_ws(w: PackedWeight, X, splits, bias=None, out=None, workspace: Workspace | None = None,
+                flags: int = 0, stream=None):
+    """gemm_qkv through w4a16_gemm_qkv_ws (with a workspace)."""
+    import torch
+
+    N, K = X.shape
+    outs = _qkv_outs(w, X, splits, bias, out)
+    st = torch.cuda.current_stream(X.device) if stream is None else stream
+    ws = workspace if workspace is not None else default_workspace(X.device, st)
+    ws.ensure(workspace_size(w.M, K, N, w.group))
+    Mq, Mk, Mv = (int(v) for v in splits)
+    _check(lib().w4a16_gemm_qkv_ws(_ptr(w.wq), _ptr(w.scales), _ptr(w.zeros), _ptr(X), _ptr(bias), Mq, Mk, Mv,
+                                   K, N, w.group, _ptr(outs[0]), _ptr(outs[1]), _ptr(outs[2]), _ptr(ws.buf),
+                                   ws.nbytes, int(flags), _vp(st.cuda_stream)), "w4a16_gemm_qkv_ws")
     return tuple(outs)
 
 

@@ -50,12 +50,23 @@ typedef enum {
     W4A16_ERR_TIMEOUT = 5       /* a bounded device-side wait ran out */
 } w4a16_status;
 
-/* Kernel selection for w4a16_gemm_ex. */
+/* Kernel selection for w4a16_gemm_ex and w4a16_gemm_ws. */
 typedef enum {
-    W4A16_PATH_AUTO = 0,     /* choose by N: GEMV for N <= 2, else tensor cores */
-    W4A16_PATH_GEMV = 1,     /* CUDA-core decode kernel (one or two tokens) */
-    W4A16_PATH_TC = 2        /* tcgen05 tensor-core kernel (three tokens and more) */
+    W4A16_PATH_AUTO = 0,     /* choose by N (and by whether a workspace is given) */
+    W4A16_PATH_GEMV = 1,     /* CUDA-core decode kernel (any N, best at one or two tokens) */
+    W4A16_PATH_TC = 2,       /* tcgen05 tile kernel (any N, best from a few tokens on) */
+    W4A16_PATH_GEMV_TC = 3   /* tcgen05 decode kernel, weight stream split over every SM
+                                (N <= 16; needs a workspace) */
 } w4a16_path;
+
+/* Flags of the workspace entry points (w4a16_gemm_ws, w4a16_gemm_qkv_ws). */
+#define W4A16_FLAG_EARLY_WEIGHTS 1u
+/*   With W4A16_PATH_GEMV_TC, launch with programmatic dependent launch: the
+ *   call's CTAs may start, and read the packed weight, while the previous
+ *   kernel in the stream is still running; X, Y and the workspace are only
+ *   touched after that kernel has completed.  The caller guarantees that no
+ *   kernel still running writes the packed weight (true of weights loaded
+ *   once, before inference).  Ignored by the other paths. */
 
 /* Human-readable name of a status code.  Never returns NULL. */
 W4A16_API const char* w4a16_status_string(int status);
@@ -173,6 +184,51 @@ W4A16_API w4a16_status w4a16_gemm_qkv(const void* wq_packed, const void* scales_
                             int Mq, int Mk, int Mv, int K, int N, int group,
                             uint16_t* Yq, uint16_t* Yk, uint16_t* Yv, void* stream);
 
+/*
+ * Workspace of w4a16_gemm_ws / w4a16_gemm_qkv_ws for an M x K weight and N
+ * tokens on the current device (it depends on the device's SM count), in
+ * bytes; 0 when the automatic choice for these sizes needs none.  The size
+ * grows with N, so a workspace sized for the largest N serves every smaller
+ * one.  W4A16_ERR_INVALID_ARG / W4A16_ERR_UNSUPPORTED as w4a16_gemm.
+ */
+W4A16_API w4a16_status w4a16_gemm_workspace_size(int M, int K, int N, int group, size_t* bytes);
+
+/*
+ * w4a16_gemm with a caller-owned workspace, which lets the decode and
+ * few-token product run on every SM ("PerfXLLM on Snapdragon 8 Gen2",
+ * section 3.3 item 2: the GEMV is memory bound; the weight is tiled along
+ * both its rows and K so the whole device streams it).  With path AUTO and
+ * N <= 16 this is W4A16_PATH_GEMV_TC: CTA c of G streams units
+ * [c U / G, (c + 1) U / G) of the U = ceil(M/128) * K/128 (row block, group)
+ * units; a block split between CTAs is summed, in CTA order, from fp32
+ * partials in the workspace, so the result stays deterministic.
+ *   workspace  device, 16-byte aligned, at least w4a16_gemm_workspace_size
+ *              bytes; zero-filled before its first use.  A completed call
+ *              leaves its counters at zero again.  One workspace serves any
+ *              number of calls in one stream; calls that may run at the same
+ *              time (different streams) need different workspaces.  After a
+ *              W4A16_ERR_TIMEOUT the workspace must be zero-filled again.
+ *   workspace_bytes  its size.
+ *   flags      0 or W4A16_FLAG_EARLY_WEIGHTS.
+ * W4A16_ERR_INVALID_ARG when the forced path needs a workspace that is
+ * missing or too small, or when the workspace overlaps another buffer; other
+ * arguments as w4a16_gemm_ex.  workspace may be NULL (workspace_bytes 0):
+ * AUTO then chooses as w4a16_gemm.
+ */
+W4A16_API w4a16_status w4a16_gemm_ws(const void* wq_packed, const void* scales_packed,
+                           const void* zeros_packed, const uint16_t* X, uint16_t* Y,
+                           int M, int K, int N, int group, int path,
+                           void* workspace, size_t workspace_bytes, unsigned flags, void* stream);
+
+/* w4a16_gemm_qkv with a workspace: the fused QKV form on the kernel
+ * w4a16_gemm_ws would choose for M = Mq + Mk + Mv (automatic choice only);
+ * workspace and flags as there. */
+W4A16_API w4a16_status w4a16_gemm_qkv_ws(const void* wq_packed, const void* scales_packed,
+                               const void* zeros_packed, const uint16_t* X, const uint16_t* bias,
+                               int Mq, int Mk, int Mv, int K, int N, int group,
+                               uint16_t* Yq, uint16_t* Yk, uint16_t* Yv,
+                               void* workspace, size_t workspace_bytes, unsigned flags, void* stream);
+
 /* As w4a16_gemm, with the kernel forced (w4a16_path).  W4A16_PATH_AUTO is the
  * same as w4a16_gemm.  Used by tests and the benchmark to time both paths. */
 W4A16_API w4a16_status w4a16_gemm_ex(const void* wq_packed, const void* scales_packed,
@@ -182,6 +238,9 @@ W4A16_API w4a16_status w4a16_gemm_ex(const void* wq_packed, const void* scales_p
 /* The path w4a16_gemm would take for these sizes (a w4a16_path value other
  * than AUTO), or -1 if the sizes are invalid.  Host only; touches no GPU. */
 W4A16_API int w4a16_select_path(int M, int K, int N);
+
+/* The path w4a16_gemm_ws with a workspace would take. */
+W4A16_API int w4a16_select_path_ws(int M, int K, int N);
 
 /*
  * Writes the dequantised weight W[m][k] = fp16_RN((q - z) * s) as fp16,
@@ -194,8 +253,8 @@ W4A16_API w4a16_status w4a16_dequant_debug(const void* wq_packed, const void* sc
                                  int M, int K, int group, void* stream);
 
 /*
- * Synchronises `stream`, then reads and clears the device-side status word
- * that bounded waits inside the tensor-core kernel set when they give up.
+ * Synchronises `stream`, then reads and clears the device-side status words
+ * that bounded waits inside the kernels set when they give up.
  * Writes W4A16_OK or W4A16_ERR_TIMEOUT to *status.  Not for the hot path.
  */
 W4A16_API w4a16_status w4a16_device_status(void* stream, int* status);

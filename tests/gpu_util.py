@@ -51,9 +51,16 @@ def assert_close(y: np.ndarray, ref: np.ndarray, what: str = ""):
 
 
 def sample_rows(M: int, n: int = 96, seed: int = 0) -> np.ndarray:
-    """Sampled output rows: both ends, tile and block edges, and random rows."""
+    """Sampled output rows: both ends and lane-quarter edges, then from every
+    128-row tile (every row block of the packed weight, so every tile a
+    persistent CTA or a cluster takes) its first and last row and one random
+    row inside it, plus n random rows."""
     rng = np.random.default_rng(seed)
     fixed = [0, 1, 31, 32, 127, 128, M // 2, M - 129, M - 128, M - 2, M - 1]
     fixed = [r for r in fixed if 0 <= r < M]
+    tiles = []
+    for t0 in range(0, M, 128):
+        t1 = min(M, t0 + 128)
+        tiles += [t0, t1 - 1, int(rng.integers(t0, t1))]
     rnd = rng.choice(M, size=min(n, M), replace=False)
-    return np.unique(np.concatenate([np.asarray(fixed, dtype=np.int64), rnd.astype(np.int64)]))
+    return np.unique(np.concatenate([np.asarray(fixed + tiles, dtype=np.int64), rnd.astype(np.int64)]))

@@ -195,3 +195,69 @@ def test_select_path_is_monotone_in_n(L):
     first_tc = paths.index(w4a16.PATH_TC) if w4a16.PATH_TC in paths else len(paths)
     assert all(p == w4a16.PATH_GEMV for p in paths[:first_tc])
     assert all(p == w4a16.PATH_TC for p in paths[first_tc:])
+
+
+def test_workspace_size_closed_form(L):
+    """Workspace of the split decode path: one counter per (row block, lane
+    quarter), rounded up to 256 bytes, then per CTA two fp32 partials of
+    128 rows x N tokens; G = min(SMs, units) CTAs.  Zero where the automatic
+    choice needs no workspace (N > 16)."""
+    for M, K in [(12288, 4096), (4096, 11008), (200, 384), (128256, 4096)]:
+        nb, U = -(-M // 128), -(-M // 128) * (K // 128)
+        cnt = -(-nb * 16 // 256) * 256
+        one = w4a16.workspace_size(M, K, 1)
+        G = (one - cnt) // 1024
+        assert (one - cnt) % 1024 == 0 and 1 <= G <= U
+        for N in (2, 7, 16):
+            assert w4a16.workspace_size(M, K, N) == cnt + G * 2 * N * 128 * 4
+        assert w4a16.workspace_size(M, K, 17) == 0
+    n = ctypes.c_size_t()
+    assert L.w4a16_gemm_workspace_size(256, 256, 1, 128, None) == w4a16.ERR_INVALID_ARG
+    assert L.w4a16_gemm_workspace_size(256, 256, 0, 128, ctypes.byref(n)) == w4a16.ERR_INVALID_ARG
+    assert L.w4a16_gemm_workspace_size(256, 200, 1, 128, ctypes.byref(n)) == w4a16.ERR_UNSUPPORTED
+    assert L.w4a16_gemm_workspace_size(256, 256, 1, 64, ctypes.byref(n)) == w4a16.ERR_UNSUPPORTED
+
+
+def test_select_path_with_workspace(L):
+    for N in (1, 2, 5, 16):
+        assert w4a16.select_path_ws(12288, 4096, N) == w4a16.PATH_GEMV_TC
+    for N in (17, 64, 4096):
+        assert w4a16.select_path_ws(12288, 4096, N) == w4a16.PATH_TC
+    assert w4a16.select_path_ws(12288, 100, 1) == -1
+
+
+def test_workspace_entry_points_reject_bad_arguments_without_launching(L):
+    """Each call breaks one rule and fails on the host.  M = K = 256, N = 2;
+    fake buffers 1 MB apart; the workspace need is a few KB."""
+    p = lambda a: ctypes.c_void_p(a)
+    wq, sc, zp, x, y, ws, yq, yk, yv = (k << 20 for k in range(1, 10))
+    null = p(0)
+    need = w4a16.workspace_size(256, 256, 2)
+    GT = w4a16.PATH_GEMV_TC
+
+    def call(path=GT, W=ws, nbytes=need, flags=0, Y=y, N=2):
+        return L.w4a16_gemm_ws(p(wq), p(sc), p(zp), p(x), p(Y), 256, 256, N, 128, path, p(W), nbytes,
+                               flags, null)
+
+    assert call(W=0, nbytes=0) == w4a16.ERR_INVALID_ARG          # forced split path, no workspace
+    assert call(nbytes=need - 1) == w4a16.ERR_INVALID_ARG        # too small
+    assert call(W=0, nbytes=64) == w4a16.ERR_INVALID_ARG         # size without a buffer
+    assert call(flags=4) == w4a16.ERR_INVALID_ARG                # unknown flag
+    assert call(path=4) == w4a16.ERR_INVALID_ARG
+    assert call(W=ws + 8) == w4a16.ERR_MISALIGNED
+    assert call(W=y - 16) == w4a16.ERR_INVALID_ARG               # workspace runs into Y
+    assert call(W=x + 256) == w4a16.ERR_INVALID_ARG              # workspace on X
+    assert call(W=wq + 0x100) == w4a16.ERR_INVALID_ARG           # workspace inside the codes
+    assert call(N=17, nbytes=1 << 20) == w4a16.ERR_UNSUPPORTED   # more tokens than the kernel takes
+    assert L.w4a16_gemm_ex(p(wq), p(sc), p(zp), p(x), p(y), 256, 256, 2, 128, GT, null) == \
+        w4a16.ERR_INVALID_ARG                                    # no workspace on this entry point
+
+    def qkv(W=ws, nbytes=need, Yv=yv, flags=0):
+        return L.w4a16_gemm_qkv_ws(p(wq), p(sc), p(zp), p(x), null, 128, 64, 64, 256, 2, 128, p(yq), p(yk),
+                                   p(Yv), p(W), nbytes, flags, null)
+
+    assert qkv(nbytes=need - 1) == w4a16.ERR_INVALID_ARG
+    assert qkv(W=yk + 128) == w4a16.ERR_INVALID_ARG              # workspace over Yk
+    assert qkv(Yv=ws + 64) == w4a16.ERR_INVALID_ARG              # Yv inside the workspace
+    assert qkv(flags=2) == w4a16.ERR_INVALID_ARG
+    assert qkv(W=ws + 8) == w4a16.ERR_MISALIGNED

@@ -1,7 +1,9 @@
 """GPU parity: the CUDA library (through the C ABI) against the CPU oracle.
 
-Small cases compare every element; full-size workloads compare sampled output
-rows, which the oracle computes one by one.  Bars: bit-exact for the
+Small cases and every full-size workload with N <= 64 compare every element;
+the larger-N workloads (N >= 128, prefill) compare sampled output rows -- from
+every 128-row tile its first, last and one random row, plus random rows --
+which the oracle computes one by one.  Bars: bit-exact for the
 dequantised weights and for exactly representable special cases; otherwise
 max |Y - Y_ref| <= 2e-3 max |Y_ref| and relative L2 <= 5e-4 (tests/gpu_util.py).
 """
@@ -176,13 +178,16 @@ def test_output_guard_bands_untouched():
 
 @pytest.mark.parametrize("M,K", LLAMA7B)
 def test_llama7b_decode_n1(M, K):
-    sampled_case(M, K, 1, w4a16.PATH_AUTO)
+    full_case(M, K, 1, w4a16.PATH_AUTO, seed=M + K)
 
 
 @pytest.mark.parametrize("path", PATHS, ids=lambda p: PATH_NAMES[p])
 @pytest.mark.parametrize("N", SWEEP_N)
 def test_qkv_n_sweep(N, path):
-    sampled_case(12288, 4096, N, path, nrows=48 if N >= 1024 else 64)
+    if N <= 64:
+        full_case(12288, 4096, N, path)
+    else:
+        sampled_case(12288, 4096, N, path, nrows=48 if N >= 1024 else 64)
 
 
 @pytest.mark.parametrize("M,K,N", [(12288, 4096, 4096), (4096, 11008, 2048)])
@@ -193,7 +198,25 @@ def test_prefill_with_outlier_channels(M, K, N):
 @pytest.mark.parametrize("N", [1, 16, 64])
 @pytest.mark.parametrize("M,K", LLAMA3)
 def test_llama3_batched_decode(M, K, N):
-    sampled_case(M, K, N, w4a16.PATH_AUTO)
+    full_case(M, K, N, w4a16.PATH_AUTO, seed=M + N)
+
+
+@pytest.mark.parametrize("path,N", [(w4a16.PATH_GEMV, 1), (w4a16.PATH_TC, 16), (w4a16.PATH_TC, 4096)],
+                         ids=["gemv-n1", "tc-n16", "tc-n4096"])
+def test_output_guard_bands_full_size(path, N):
+    """The fused QKV shape written into the middle of a larger buffer: the
+    bytes around Y stay untouched (every row tile and token of the output)."""
+    M, K, pad = 12288, 4096, 4096
+    p = synth.make_problem(M, K, N, seed=77 + N)
+    w, x = pack_problem(p)
+    buf = torch.full((N * M + 2 * pad,), 12345, dtype=torch.int16, device="cuda")
+    y = buf[pad:pad + N * M].view(torch.float16).view(N, M)
+    w4a16.gemm_ex(w, x, Y=y, path=path)
+    torch.cuda.synchronize()
+    assert torch.all(buf[:pad] == 12345) and torch.all(buf[-pad:] == 12345)
+    assert torch.isfinite(y.float()).all()
+    if N <= 64:
+        assert_close(to_f64(y), oracle.gemm(p.q, p.zeros, p.scales, p.x), f"guarded full size N={N}")
 
 
 # --------------------------------------------------------- group quantiser ----
