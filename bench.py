@@ -20,7 +20,7 @@ every rank runs its own copy of the step (weak scaling), no collective on the
 data path; time is the max over ranks.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-    python bench.py --workload qkv_n1|prefill|sweep|quantize|qkv_fused|add_rmsnorm ...
+    python bench.py --workload qkv_n1|prefill|sweep|quantize|qkv_fused|gate_up_fused|add_rmsnorm ...
                                                           (secondary workloads)
 """
 from __future__ import annotations
@@ -429,6 +429,8 @@ def main_ours(args):
         return quantize_workload(args, device, peaks)
     if args.workload == "qkv_fused":
         return qkv_fused_workload(args, device, peaks)
+    if args.workload == "gate_up_fused":
+        return gate_up_fused_workload(args, device, peaks)
     if args.workload == "add_rmsnorm":
         return add_rmsnorm_workload(args, device, peaks)
 
@@ -762,6 +764,72 @@ def qkv_fused_workload(args, device, peaks):
     return 0
 
 
+def gate_up_fused_workload(args, device, peaks):
+    """Fused gate/up projection of LLaMA-7B (Mi = 11008, K = 4096) at N = 1
+    (8 rotated weight copies, 375 MB, beyond L2) and N = 4096 (2 copies),
+    three arms, each a CUDA graph through the workspace entry points:
+      fused     w4a16_gemm_gate_up_ws on the gate/up packing (H [N][Mi]);
+      plain     w4a16_gemm_ws on the same weight packed in row order (Y [N][2 Mi]);
+      unfused   the plain product, then torch silu(Y[:, :Mi]) * Y[:, Mi:]
+                (what a caller writes without the fused form; timing only).
+    Per-call microseconds, median / p10 / p90 over the replays, with the SM
+    clock of each window."""
+    import torch
+
+    from gemm_w4a16_b200 import synth, w4a16
+
+    Mi, K = 11008, 4096
+    M = 2 * Mi
+    sampler = ClockSampler(device.index or 0)
+    sampler.start()
+    try:
+        for N, copies_n in ((1, 8), (4096, 2)):
+            gen = torch.Generator(device=device)
+            gen.manual_seed(61)
+            sets = []
+            for _ in range(copies_n):
+                q, z, sc = synth.make_weights_torch(M, K, GROUP, gen, device)
+                sets.append((w4a16.pack_gate_up(q, sc, z), w4a16.pack(q, sc, z),
+                             synth.make_activations_torch(N, K, gen, device),
+                             torch.empty((N, Mi), dtype=torch.float16, device=device),
+                             torch.empty((N, M), dtype=torch.float16, device=device),
+                             torch.empty((N, Mi), dtype=torch.float16, device=device)))
+                del q, z, sc
+            ws = w4a16.Workspace(device, w4a16.workspace_size(M, K, N))
+            flags = w4a16.FLAG_EARLY_WEIGHTS
+
+            def fused():
+                for wg, _, x, h, _, _ in sets:
+                    w4a16.gemm_gate_up_ws(wg, x, H=h, workspace=ws, flags=flags)
+
+            def plain():
+                for _, wp, x, _, y, _ in sets:
+                    w4a16.gemm_ws(wp, x, Y=y, workspace=ws, flags=flags)
+
+            def unfused():
+                for _, wp, x, _, y, h2 in sets:
+                    w4a16.gemm_ws(wp, x, Y=y, workspace=ws, flags=flags)
+                    torch.mul(torch.nn.functional.silu(y[:, :Mi]), y[:, Mi:], out=h2)
+
+            for name, fn in (("fused", fused), ("plain", plain), ("unfused_plain_then_torch", unfused)):
+                g = capture(fn, device)
+                t0 = time.time()
+                _, per = time_steps(g, args.steps, args.warmup, device)
+                t1 = time.time()
+                us = pct(per, 1e3 / copies_n)
+                print(json.dumps({"workload": f"gate_up {name} Mi={Mi} K={K} N={N}", "us": us["median"],
+                                  "us_pct": us, "path": w4a16.select_path_ws(M, K, N),
+                                  "GBps": alg_bytes(M, K, N) / (us["median"] * 1e-6) / 1e9,
+                                  "TFLOPS": alg_flops(M, K, N) / (us["median"] * 1e-6) / 1e12,
+                                  "clocks": sampler.summary(t0, t1)}), flush=True)
+                del g
+            del sets
+            torch.cuda.empty_cache()
+    finally:
+        sampler.stop()
+    return 0
+
+
 def quantize_workload(args, device, peaks):
     """Group quantiser fp16 W -> (q, s, z) on the four LLaMA-7B projection
     shapes, 8 rotated weight copies per shape (beyond L2); HBM bytes per call:
@@ -910,7 +978,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["decode", "qkv_n1", "prefill", "sweep", "shape", "quantize",
-                                           "qkv_fused", "add_rmsnorm"],
+                                           "qkv_fused", "gate_up_fused", "add_rmsnorm"],
                     default="decode")
     ap.add_argument("--M", type=int, default=12288)
     ap.add_argument("--K", type=int, default=4096)

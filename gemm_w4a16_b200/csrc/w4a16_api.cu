@@ -147,7 +147,8 @@ w4a16_status gemm_qkv_impl(const void* wq_packed, const void* scales_packed, con
         if (overlap(outs[i], out_n[i], outs[j], out_n[j])) return W4A16_ERR_INVALID_ARG;
     }
   }
-  OutMap om;
+  OutMap om = {};
+  om.kind = kEpiQkv;
   om.y0 = Yq;
   om.y1 = Yk;
   om.y2 = Yv;
@@ -230,9 +231,12 @@ w4a16_status w4a16_add_rmsnorm(const uint16_t* h, const uint16_t* d, const uint1
   return map_cuda(launch_add_rmsnorm(h, d, gamma, eps, N, K, r_out, X, static_cast<cudaStream_t>(stream)));
 }
 
-w4a16_status w4a16_pack(const uint8_t* q, const uint16_t* scales, const uint8_t* zeros,
-                        int M, int K, int group, void* wq_packed, void* scales_packed,
-                        void* zeros_packed, void* stream) {
+}  // extern "C"
+
+namespace {
+
+w4a16_status pack_impl(const uint8_t* q, const uint16_t* scales, const uint8_t* zeros, int M, int K, int group,
+                       void* wq_packed, void* scales_packed, void* zeros_packed, void* stream, int mi) {
   if (!q || !scales || !zeros || !wq_packed || !scales_packed || !zeros_packed)
     return W4A16_ERR_INVALID_ARG;
   w4a16_status st = check_shape(M, K, group);
@@ -254,9 +258,85 @@ w4a16_status w4a16_pack(const uint8_t* q, const uint16_t* scales, const uint8_t*
     }
   }
   return map_cuda(launch_pack(q, scales, zeros, M, K, static_cast<uint8_t*>(wq_packed),
-                              static_cast<uint16_t*>(scales_packed),
-                              static_cast<uint8_t*>(zeros_packed),
-                              static_cast<cudaStream_t>(stream)));
+                              static_cast<uint16_t*>(scales_packed), static_cast<uint8_t*>(zeros_packed),
+                              static_cast<cudaStream_t>(stream), mi));
+}
+
+w4a16_status gemm_gate_up_impl(const void* wq_packed, const void* scales_packed, const void* zeros_packed,
+                               const uint16_t* X, uint16_t* H, int Mi, int K, int N, int group, int path,
+                               void* ws, size_t ws_bytes, unsigned flags, void* stream) {
+  if (!wq_packed || !scales_packed || !zeros_packed || !X || !H) return W4A16_ERR_INVALID_ARG;
+  if (Mi <= 0 || N <= 0 || path < W4A16_PATH_AUTO || path > W4A16_PATH_GEMV_TC) return W4A16_ERR_INVALID_ARG;
+  if (flags & ~W4A16_FLAG_EARLY_WEIGHTS) return W4A16_ERR_INVALID_ARG;
+  if (!ws && ws_bytes) return W4A16_ERR_INVALID_ARG;
+  if (Mi > kMaxM / 2) return W4A16_ERR_UNSUPPORTED;
+  const int M = 2 * Mi;
+  w4a16_status st = check_shape(M, K, group);
+  if (st != W4A16_OK) return st;
+  if (N > kMaxN) return W4A16_ERR_UNSUPPORTED;
+  if (!aligned16(wq_packed) || !aligned16(scales_packed) || !aligned16(zeros_packed) || !aligned16(X) ||
+      !aligned16(H) || (ws && !aligned16(ws)))
+    return W4A16_ERR_MISALIGNED;
+  if (path == W4A16_PATH_AUTO) path = select_path_impl(M, K, N, ws != nullptr);
+  if (path == W4A16_PATH_GEMV_TC && N > kGemvTcMaxTokens) return W4A16_ERR_UNSUPPORTED;
+  const size_t need = workspace_for(path, M, K, N);
+  if (need > ws_bytes) return W4A16_ERR_INVALID_ARG;
+  {
+    const PackedBytes pb = packed_bytes(M, K);
+    const size_t nh = (size_t)N * Mi * 2, nx = (size_t)N * K * 2;
+    if (overlap(H, nh, X, nx) || overlaps_weight(H, nh, wq_packed, scales_packed, zeros_packed, pb))
+      return W4A16_ERR_INVALID_ARG;
+    if (need && (overlap(ws, need, X, nx) || overlap(ws, need, H, nh) ||
+                 overlaps_weight(ws, need, wq_packed, scales_packed, zeros_packed, pb)))
+      return W4A16_ERR_INVALID_ARG;
+  }
+  OutMap om = {};
+  om.kind = kEpiGateUp;
+  om.h = H;
+  om.mi = Mi;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint8_t* wq = static_cast<const uint8_t*>(wq_packed);
+  const uint16_t* sp = static_cast<const uint16_t*>(scales_packed);
+  const uint8_t* zp = static_cast<const uint8_t*>(zeros_packed);
+  cudaError_t e;
+  if (path == W4A16_PATH_GEMV_TC)
+    e = launch_gemv_tc(wq, sp, zp, X, nullptr, M, K, N, ws, (flags & W4A16_FLAG_EARLY_WEIGHTS) != 0, s, &om);
+  else if (path == W4A16_PATH_TC)
+    e = launch_gemm_tc(wq, sp, zp, X, nullptr, M, K, N, s, &om);
+  else
+    e = launch_gemv(wq, sp, zp, X, nullptr, M, K, N, s, &om);
+  return map_cuda(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+w4a16_status w4a16_pack(const uint8_t* q, const uint16_t* scales, const uint8_t* zeros,
+                        int M, int K, int group, void* wq_packed, void* scales_packed,
+                        void* zeros_packed, void* stream) {
+  return pack_impl(q, scales, zeros, M, K, group, wq_packed, scales_packed, zeros_packed, stream, 0);
+}
+
+w4a16_status w4a16_pack_gate_up(const uint8_t* q, const uint16_t* scales, const uint8_t* zeros,
+                                int Mi, int K, int group, void* wq_packed, void* scales_packed,
+                                void* zeros_packed, void* stream) {
+  if (Mi <= 0) return W4A16_ERR_INVALID_ARG;
+  if (Mi > kMaxM / 2) return W4A16_ERR_UNSUPPORTED;
+  return pack_impl(q, scales, zeros, 2 * Mi, K, group, wq_packed, scales_packed, zeros_packed, stream, Mi);
+}
+
+w4a16_status w4a16_gemm_gate_up(const void* wq_packed, const void* scales_packed, const void* zeros_packed,
+                                const uint16_t* X, uint16_t* H, int Mi, int K, int N, int group, void* stream) {
+  return gemm_gate_up_impl(wq_packed, scales_packed, zeros_packed, X, H, Mi, K, N, group, W4A16_PATH_AUTO,
+                           nullptr, 0, 0u, stream);
+}
+
+w4a16_status w4a16_gemm_gate_up_ws(const void* wq_packed, const void* scales_packed, const void* zeros_packed,
+                                   const uint16_t* X, uint16_t* H, int Mi, int K, int N, int group, int path,
+                                   void* workspace, size_t workspace_bytes, unsigned flags, void* stream) {
+  return gemm_gate_up_impl(wq_packed, scales_packed, zeros_packed, X, H, Mi, K, N, group, path, workspace,
+                           workspace_bytes, flags, stream);
 }
 
 int w4a16_select_path(int M, int K, int N) { return select_path_impl(M, K, N, false); }

@@ -158,7 +158,7 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-template <int BN, bool kMap>
+template <int BN, int kEpi>
 __global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __restrict__ wq,
                const uint16_t* __restrict__ s_p, const uint8_t* __restrict__ z_p,
@@ -451,7 +451,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
       // The fused form's destination and bias of this row, loaded before the
       // wait so the load overlaps it.
       RowDst dst = {};
-      if constexpr (kMap) {
+      if constexpr (kEpi == kEpiQkv) {
         if (m < M) dst = row_dst(om, M, m);
       }
       if (!wait_bar_warp(&sh.acc_full[b], bph, sh.abort_flag, &g_tc_status)) break;
@@ -484,12 +484,19 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&sh.acc_empty[b]);
         }
-        if (m < M) {
+        if constexpr (kEpi == kEpiGateUp) {
+          // Whole warps: the gate/up pairing shuffles.
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int n = n0 + 16 * c + j;
+            store_gate_up(om, mt, row, n, sum[j], n < N);
+          }
+        } else if (m < M) {
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int n = n0 + 16 * c + j;
             if (n < N) {
-              if constexpr (kMap) store_row(dst, om.bias != nullptr, n, sum[j]);
+              if constexpr (kEpi == kEpiQkv) store_row(dst, om.bias != nullptr, n, sum[j]);
               else Y[(size_t)n * M + m] = __half_as_ushort(__float2half_rn(sum[j]));
             }
           }
@@ -509,12 +516,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
 
 // ------------------------------------------------------------------ host --
 
-template <int BN, bool kMap>
+template <int BN, int kEpi>
 cudaError_t launch_bn(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p, const uint16_t* X,
                       uint16_t* Y, int M, int K, int N, cudaStream_t stream, const OutMap& om) {
   using C = Cfg<BN>;
   static std::atomic<unsigned long long> smem_set{0};
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(gemm_tc_kernel<BN, kMap>), C::kSmemBytes,
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(gemm_tc_kernel<BN, kEpi>), C::kSmemBytes,
                                     smem_set);
   if (e != cudaSuccess) return e;
   CUtensorMap map;
@@ -522,7 +529,7 @@ cudaError_t launch_bn(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p
   if (e != cudaSuccess) return e;
   const int tiles = ceil_div(M, kBM) * ceil_div(N, BN);
   const int grid = tiles < num_sms() ? tiles : num_sms();
-  gemm_tc_kernel<BN, kMap><<<grid, C::kThreads, C::kSmemBytes, stream>>>(map, wq, s_p, z_p, Y, M, K, N, om);
+  gemm_tc_kernel<BN, kEpi><<<grid, C::kThreads, C::kSmemBytes, stream>>>(map, wq, s_p, z_p, Y, M, K, N, om);
   return cudaGetLastError();
 }
 
@@ -545,22 +552,24 @@ __global__ void wait_timeout_selftest_kernel(long long limit) {
 // shape); the tensor-core kernel from there on.
 int gemv_max_n() { return 2; }
 
-template <bool kMap>
+template <int kEpi>
 cudaError_t launch_tc_map(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros, const uint16_t* X,
                           uint16_t* Y, int M, int K, int N, cudaStream_t stream, const OutMap& om) {
-  if (N <= 16) return launch_bn<16, kMap>(wq, scales, zeros, X, Y, M, K, N, stream, om);
-  if (N <= 32) return launch_bn<32, kMap>(wq, scales, zeros, X, Y, M, K, N, stream, om);
-  if (N <= 64) return launch_bn<64, kMap>(wq, scales, zeros, X, Y, M, K, N, stream, om);
-  if (N <= 128) return launch_bn<128, kMap>(wq, scales, zeros, X, Y, M, K, N, stream, om);
-  return launch_bn<256, kMap>(wq, scales, zeros, X, Y, M, K, N, stream, om);
+  if (N <= 16) return launch_bn<16, kEpi>(wq, scales, zeros, X, Y, M, K, N, stream, om);
+  if (N <= 32) return launch_bn<32, kEpi>(wq, scales, zeros, X, Y, M, K, N, stream, om);
+  if (N <= 64) return launch_bn<64, kEpi>(wq, scales, zeros, X, Y, M, K, N, stream, om);
+  if (N <= 128) return launch_bn<128, kEpi>(wq, scales, zeros, X, Y, M, K, N, stream, om);
+  return launch_bn<256, kEpi>(wq, scales, zeros, X, Y, M, K, N, stream, om);
 }
 
 cudaError_t launch_gemm_tc(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros,
                            const uint16_t* X, uint16_t* Y, int M, int K, int N, cudaStream_t stream,
                            const OutMap* om) {
   if (K % kMaxSlotK) return cudaErrorNotSupported;
-  if (om) return launch_tc_map<true>(wq, scales, zeros, X, nullptr, M, K, N, stream, *om);
-  return launch_tc_map<false>(wq, scales, zeros, X, Y, M, K, N, stream, OutMap{});
+  if (om && om->kind == kEpiGateUp)
+    return launch_tc_map<kEpiGateUp>(wq, scales, zeros, X, nullptr, M, K, N, stream, *om);
+  if (om) return launch_tc_map<kEpiQkv>(wq, scales, zeros, X, nullptr, M, K, N, stream, *om);
+  return launch_tc_map<kEpiPlain>(wq, scales, zeros, X, Y, M, K, N, stream, OutMap{});
 }
 
 cudaError_t launch_wait_timeout_selftest(long long limit_cycles, cudaStream_t stream) {

@@ -66,7 +66,7 @@ __host__ __device__ inline GvLayout gv_layout(int nt, int gspan, int cl) {
   return L;
 }
 
-template <int NT, bool kMap>
+template <int NT, int kEpi>
 __global__ void __launch_bounds__(kGvThreads)
 gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
             const uint8_t* __restrict__ z_p, const uint16_t* __restrict__ X,
@@ -189,7 +189,7 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   // The fused form's destination and bias of row m, loaded before the
   // reductions so the load overlaps them.
   RowDst dst = {};
-  if constexpr (kMap) {
+  if constexpr (kEpi == kEpiQkv) {
     const int m = b * kRowBlock + r;
     if (r < kRowBlock && crank == 0 && m < M) dst = row_dst(om, M, m);
   }
@@ -230,8 +230,12 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   }
 
   const int m = b * kRowBlock + r;
-  if (m < M) {
-    if constexpr (kMap) {
+  if constexpr (kEpi == kEpiGateUp) {
+    // Threads 0..127 are whole warps here: the gate/up pairing shuffles.
+#pragma unroll
+    for (int n = 0; n < NT; ++n) store_gate_up(om, b, r, n, tot[n], true);
+  } else if (m < M) {
+    if constexpr (kEpi == kEpiQkv) {
 #pragma unroll
       for (int n = 0; n < NT; ++n) store_row(dst, om.bias != nullptr, n, tot[n]);
     } else {
@@ -241,11 +245,11 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   }
 }
 
-template <int NT, bool kMap>
+template <int NT, int kEpi>
 cudaError_t launch_nt(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p, const uint16_t* X,
                       uint16_t* Y, int M, int K, int cl, cudaStream_t stream, const OutMap& om) {
   static std::atomic<unsigned long long> smem_set{0};
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(gemv_kernel<NT, kMap>), 200 * 1024, smem_set);
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(gemv_kernel<NT, kEpi>), 200 * 1024, smem_set);
   if (e != cudaSuccess) return e;
   const int blocks = ceil_div(M, kRowBlock);
   const GvLayout L = gv_layout(NT, ceil_div(K / kGroup, cl), cl);
@@ -261,7 +265,7 @@ cudaError_t launch_nt(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_kernel<NT, kMap>, wq, s_p, z_p, X, Y, M, K, cl, om);
+  return cudaLaunchKernelEx(&cfg, gemv_kernel<NT, kEpi>, wq, s_p, z_p, X, Y, M, K, cl, om);
 }
 
 }  // namespace
@@ -310,26 +314,31 @@ cudaError_t launch_gemv(const uint8_t* wq, const uint16_t* scales, const uint8_t
     OutMap on = {};
     if (om) {
       on = *om;
-      on.y0 = om->y0 + (size_t)n0 * om->end0;
-      on.y1 = om->y1 + (size_t)n0 * (om->end1 - om->end0);
-      on.y2 = om->y2 + (size_t)n0 * (M - om->end1);
+      if (om->kind == kEpiGateUp) {
+        on.h = om->h + (size_t)n0 * om->mi;
+      } else {
+        on.y0 = om->y0 + (size_t)n0 * om->end0;
+        on.y1 = om->y1 + (size_t)n0 * (om->end1 - om->end0);
+        on.y2 = om->y2 + (size_t)n0 * (M - om->end1);
+      }
     }
+    const int kind = om ? om->kind : kEpiPlain;
     cudaError_t e;
-    if (om) {
-      switch (nt) {
-        case 1: e = launch_nt<1, true>(wq, scales, zeros, Xn, Yn, M, K, cl, stream, on); break;
-        case 2: e = launch_nt<2, true>(wq, scales, zeros, Xn, Yn, M, K, cl, stream, on); break;
-        case 3: e = launch_nt<3, true>(wq, scales, zeros, Xn, Yn, M, K, cl, stream, on); break;
-        default: e = launch_nt<4, true>(wq, scales, zeros, Xn, Yn, M, K, cl, stream, on); break;
-      }
-    } else {
-      switch (nt) {
-        case 1: e = launch_nt<1, false>(wq, scales, zeros, Xn, Yn, M, K, cl, stream, on); break;
-        case 2: e = launch_nt<2, false>(wq, scales, zeros, Xn, Yn, M, K, cl, stream, on); break;
-        case 3: e = launch_nt<3, false>(wq, scales, zeros, Xn, Yn, M, K, cl, stream, on); break;
-        default: e = launch_nt<4, false>(wq, scales, zeros, Xn, Yn, M, K, cl, stream, on); break;
-      }
+#define W4A16_GEMV_NT(EPI)                                                                          \
+    switch (nt) {                                                                                     \
+      case 1: e = launch_nt<1, EPI>(wq, scales, zeros, Xn, Yn, M, K, cl, stream, on); break;          \
+      case 2: e = launch_nt<2, EPI>(wq, scales, zeros, Xn, Yn, M, K, cl, stream, on); break;          \
+      case 3: e = launch_nt<3, EPI>(wq, scales, zeros, Xn, Yn, M, K, cl, stream, on); break;          \
+      default: e = launch_nt<4, EPI>(wq, scales, zeros, Xn, Yn, M, K, cl, stream, on); break;         \
     }
+    if (kind == kEpiGateUp) {
+      W4A16_GEMV_NT(kEpiGateUp)
+    } else if (kind == kEpiQkv) {
+      W4A16_GEMV_NT(kEpiQkv)
+    } else {
+      W4A16_GEMV_NT(kEpiPlain)
+    }
+#undef W4A16_GEMV_NT
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

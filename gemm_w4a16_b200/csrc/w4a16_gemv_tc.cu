@@ -115,7 +115,7 @@ __host__ __device__ __forceinline__ int cta_of(long long U, int G, long long u) 
   return (int)(((u + 1) * G - 1) / U);
 }
 
-template <class C, bool kMap>
+template <class C, int kEpi>
 __global__ void __launch_bounds__(C::kThreads, 2)
 gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __restrict__ wq,
                const uint16_t* __restrict__ s_p, const uint8_t* __restrict__ z_p, uint16_t* __restrict__ Y,
@@ -327,7 +327,7 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
       const int buf = bi % C::kAccBufs;
       const int m = b * kRowBlock + row;
       RowDst rd = {};
-      if constexpr (kMap) {
+      if constexpr (kEpi == kEpiQkv) {
         if (m < M) rd = row_dst(om, M, m);
       }
       if (!wait_bar_warp(&acc_full[buf], (uint32_t)((bi / C::kAccBufs) & 1), abort_flag, &g_gvtc_status)) break;
@@ -384,11 +384,17 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
           write = true;
         }
       }
-      if (write && m < M) {
+      if constexpr (kEpi == kEpiGateUp) {
+        // `write` is the same on every lane: the gate/up pairing shuffles.
+        if (write) {
+#pragma unroll
+          for (int n = 0; n < BN; ++n) store_gate_up(om, b, row, n, acc[n], n < N);
+        }
+      } else if (write && m < M) {
 #pragma unroll
         for (int n = 0; n < BN; ++n) {
           if (n < N) {
-            if constexpr (kMap) store_row(rd, om.bias != nullptr, n, acc[n]);
+            if constexpr (kEpi == kEpiQkv) store_row(rd, om.bias != nullptr, n, acc[n]);
             else Y[(size_t)n * M + m] = __half_as_ushort(__float2half_rn(acc[n]));
           }
         }
@@ -413,12 +419,12 @@ int grid_for(int M, int K) {
   return (int)(U < sms ? U : sms);
 }
 
-template <class C, bool kMap>
+template <class C, int kEpi>
 cudaError_t launch_cfg(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p, const uint16_t* X,
                        uint16_t* Y, int M, int K, int N, void* ws, bool pdl, cudaStream_t stream,
                        const OutMap& om) {
   static std::atomic<unsigned long long> smem_set{0};
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(gemv_tc_kernel<C, kMap>), C::kSmemBytes,
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(gemv_tc_kernel<C, kEpi>), C::kSmemBytes,
                                     smem_set);
   if (e != cudaSuccess) return e;
   CUtensorMap map;
@@ -436,7 +442,7 @@ cudaError_t launch_cfg(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, gemv_tc_kernel<C, kMap>, map, wq, s_p, z_p, Y, M, K, N, cnt, part, om);
+  return cudaLaunchKernelEx(&cfg, gemv_tc_kernel<C, kEpi>, map, wq, s_p, z_p, Y, M, K, N, cnt, part, om);
 }
 
 }  // namespace
@@ -453,8 +459,10 @@ cudaError_t launch_gemv_tc(const uint8_t* wq, const uint16_t* scales, const uint
                            uint16_t* Y, int M, int K, int N, void* workspace, bool pdl, cudaStream_t stream,
                            const OutMap* om) {
   if (N > kGemvTcMaxTokens) return cudaErrorNotSupported;
-  if (om) return launch_cfg<Cfg16, true>(wq, scales, zeros, X, nullptr, M, K, N, workspace, pdl, stream, *om);
-  return launch_cfg<Cfg16, false>(wq, scales, zeros, X, Y, M, K, N, workspace, pdl, stream, OutMap{});
+  if (om && om->kind == kEpiGateUp)
+    return launch_cfg<Cfg16, kEpiGateUp>(wq, scales, zeros, X, nullptr, M, K, N, workspace, pdl, stream, *om);
+  if (om) return launch_cfg<Cfg16, kEpiQkv>(wq, scales, zeros, X, nullptr, M, K, N, workspace, pdl, stream, *om);
+  return launch_cfg<Cfg16, kEpiPlain>(wq, scales, zeros, X, Y, M, K, N, workspace, pdl, stream, OutMap{});
 }
 
 cudaError_t read_and_clear_gvtc_status(int* v) {

@@ -102,18 +102,52 @@ __device__ __forceinline__ uint32_t zero_code(const uint8_t* zblock, int r) {
   return (zblock[r >> 1] >> ((r & 1) * 4)) & 0xFu;
 }
 
+// ------------------------------------------------------ gate/up rows ----
+
+// The gate/up row order of w4a16_pack_gate_up: packed block b holds the 64
+// intermediate channels i = 64 b + 16 q + j (q = 0..3 the 32-row lane quarter,
+// j = 0..15), the gate row of channel i at packed row 32 q + j and its up row
+// at 32 q + 16 + j, so one warp of an epilogue (thread = packed row) holds
+// both halves of 16 channels and pairs them with one shuffle.
+__host__ __device__ inline int gate_up_channel(int b, int r) { return b * 64 + (r >> 5) * 16 + (r & 15); }
+
+// Canonical row held by packed row r of block b (-1: a padding row).  mi == 0:
+// rows in order, M of them; mi > 0: the gate/up order over a canonical weight
+// whose rows are the gate projection's mi rows then the up projection's mi.
+__host__ __device__ inline int packed_source_row(int b, int r, int M, int mi) {
+  if (mi == 0) {
+    const int m = b * kRowBlock + r;
+    return m < M ? m : -1;
+  }
+  const int i = gate_up_channel(b, r);
+  if (i >= mi) return -1;
+  return (r & 16) ? mi + i : i;
+}
+
 // --------------------------------------------------------- output map ----
 
-// Where an epilogue puts row m of the result when the caller asked for the
-// fused form (w4a16_gemm_qkv): rows [0, end0), [end0, end1) and [end1, M) go
-// to three token-major outputs of their own widths, each value after adding
-// an optional fp16 bias of its row in fp32 and one RNE rounding to fp16.
+// Epilogue kinds of the GEMM kernels.
+enum Epi : int {
+  kEpiPlain = 0,    // Y[n][m], one RNE rounding of the fp32 accumulator
+  kEpiQkv = 1,      // three outputs plus an optional bias (w4a16_gemm_qkv)
+  kEpiGateUp = 2,   // H[n][i] = silu(gate) * up (w4a16_gemm_gate_up)
+};
+
+// Where an epilogue puts row m of the result when the caller asked for a
+// fused form.  QKV (w4a16_gemm_qkv): rows [0, end0), [end0, end1) and
+// [end1, M) go to three token-major outputs of their own widths, each value
+// after adding an optional fp16 bias of its row in fp32 and one RNE rounding
+// to fp16.  Gate/up (w4a16_gemm_gate_up): h [N][mi], from a weight packed in
+// the gate/up row order.
 struct OutMap {
+  int kind;               // Epi: kEpiQkv or kEpiGateUp
   uint16_t* y0;
   uint16_t* y1;
   uint16_t* y2;
   int end0, end1;
   const uint16_t* bias;   // [M] or null
+  uint16_t* h;
+  int mi;
 };
 
 // Row m's destination in the fused form, resolved once per row: its element
@@ -146,6 +180,20 @@ __device__ __forceinline__ RowDst row_dst(const OutMap& o, int M, int m) {
 __device__ __forceinline__ void store_row(const RowDst& d, bool has_bias, int n, float v) {
   if (has_bias) v = __fadd_rn(v, d.bias);
   d.y[(size_t)n * d.ld] = __half_as_ushort(__float2half_rn(v));
+}
+
+// Gate/up epilogue of one token: v is the fp32 accumulator of packed row r
+// (0..127, thread = row, all 32 lanes of the warp calling together) of block
+// b.  Lanes 0..15 hold gate rows and take their channel's up value from lane
+// + 16, then write H[n][i] = fp16_RN(silu(g) * u), silu(g) = g / (1 + e^-g),
+// in fp32 (e^-g overflowing to infinity gives silu = -0, not NaN).
+__device__ __forceinline__ void store_gate_up(const OutMap& o, int b, int r, int n, float v, bool valid) {
+  const float u = __shfl_down_sync(0xffffffffu, v, 16);
+  const int i = gate_up_channel(b, r);
+  if (valid && (r & 16) == 0 && i < o.mi) {
+    const float silu = v / (1.0f + expf(-v));
+    o.h[(size_t)n * o.mi + i] = __half_as_ushort(__float2half_rn(silu * u));
+  }
 }
 
 // ------------------------------------------------------- launch helpers ----
@@ -188,9 +236,10 @@ cudaError_t launch_add_rmsnorm(const uint16_t* h, const uint16_t* d, const uint1
 cudaError_t launch_quantize(const uint16_t* W, int M, int K, uint8_t* q, uint16_t* scales, uint8_t* zeros,
                             cudaStream_t stream);
 
+// mi > 0: the gate/up row order (packed_source_row), M = 2 mi.
 cudaError_t launch_pack(const uint8_t* q, const uint16_t* scales, const uint8_t* zeros,
                         int M, int K, uint8_t* wq_p, uint16_t* s_p, uint8_t* z_p,
-                        cudaStream_t stream);
+                        cudaStream_t stream, int mi = 0);
 
 cudaError_t launch_dequant(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros,
                            uint16_t* W, int M, int K, cudaStream_t stream);

@@ -15,7 +15,8 @@ namespace {
 __device__ __forceinline__ int nibble_of_offset(int o) { return (o & 1) ? 4 + (o >> 1) : (o >> 1); }
 
 // One thread per 16-byte output chunk (block b, chunk column c, row r).
-__global__ void pack_weights_kernel(const uint8_t* __restrict__ q, int M, int K,
+// mi > 0: the gate/up row order (packed_source_row).
+__global__ void pack_weights_kernel(const uint8_t* __restrict__ q, int M, int K, int mi,
                                     uint4* __restrict__ wq_p, long long n_chunks) {
   long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n_chunks) return;
@@ -24,9 +25,9 @@ __global__ void pack_weights_kernel(const uint8_t* __restrict__ q, int M, int K,
   long long t = i / kRowBlock;
   int c = (int)(t % kc_n);
   int b = (int)(t / kc_n);
-  int m = b * kRowBlock + r;
+  int m = packed_source_row(b, r, M, mi);
   uint32_t words[4] = {0u, 0u, 0u, 0u};
-  if (m < M) {
+  if (m >= 0) {
     const uint8_t* src = q + (size_t)m * K + (size_t)c * kChunkK;
 #pragma unroll
     for (int j = 0; j < kChunkK; ++j) {
@@ -39,7 +40,7 @@ __global__ void pack_weights_kernel(const uint8_t* __restrict__ q, int M, int K,
 
 // One thread per (block b, group g, row pair rp): two scales and one zero byte.
 __global__ void pack_meta_kernel(const uint16_t* __restrict__ scales,
-                                 const uint8_t* __restrict__ zeros, int M, int K,
+                                 const uint8_t* __restrict__ zeros, int M, int K, int mi,
                                  uint16_t* __restrict__ s_p, uint8_t* __restrict__ z_p,
                                  long long n_pairs) {
   long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -54,10 +55,10 @@ __global__ void pack_meta_kernel(const uint16_t* __restrict__ scales,
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     int r = 2 * rp + h;
-    int m = b * kRowBlock + r;
+    int m = packed_source_row(b, r, M, mi);
     uint16_t s = 0;
     uint32_t z = 0;
-    if (m < M) {
+    if (m >= 0) {
       s = scales[(size_t)m * kg + g];
       z = zeros[(size_t)m * kg + g] & 0xFu;
     }
@@ -100,17 +101,17 @@ __global__ void dequant_kernel(const uint4* __restrict__ wq_p, const uint16_t* _
 
 cudaError_t launch_pack(const uint8_t* q, const uint16_t* scales, const uint8_t* zeros,
                         int M, int K, uint8_t* wq_p, uint16_t* s_p, uint8_t* z_p,
-                        cudaStream_t stream) {
+                        cudaStream_t stream, int mi) {
   const int mb = ceil_div(M, kRowBlock);
   long long n_chunks = (long long)mb * (K / kChunkK) * kRowBlock;
   long long n_pairs = (long long)mb * (K / kGroup) * (kRowBlock / 2);
   const int threads = 256;
   pack_weights_kernel<<<(unsigned)((n_chunks + threads - 1) / threads), threads, 0, stream>>>(
-      q, M, K, reinterpret_cast<uint4*>(wq_p), n_chunks);
+      q, M, K, mi, reinterpret_cast<uint4*>(wq_p), n_chunks);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   pack_meta_kernel<<<(unsigned)((n_pairs + threads - 1) / threads), threads, 0, stream>>>(
-      scales, zeros, M, K, s_p, z_p, n_pairs);
+      scales, zeros, M, K, mi, s_p, z_p, n_pairs);
   return cudaGetLastError();
 }
 

@@ -25,7 +25,7 @@ EXPORTED = (
     "w4a16_gemm_ex", "w4a16_select_path", "w4a16_dequant_debug",
     "w4a16_device_status", "w4a16_selftest_wait_timeout", "w4a16_quantize", "w4a16_gemm_qkv",
     "w4a16_add_rmsnorm", "w4a16_gemm_workspace_size", "w4a16_gemm_ws", "w4a16_gemm_qkv_ws",
-    "w4a16_select_path_ws",
+    "w4a16_select_path_ws", "w4a16_pack_gate_up", "w4a16_gemm_gate_up", "w4a16_gemm_gate_up_ws",
 )
 
 _lib = None
@@ -80,6 +80,12 @@ def lib():
             L.w4a16_gemm_qkv_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp,
                                             _vp, _sz, _u, _vp]
             L.w4a16_gemm_qkv_ws.restype = _i
+            L.w4a16_pack_gate_up.argtypes = [_vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp]
+            L.w4a16_pack_gate_up.restype = _i
+            L.w4a16_gemm_gate_up.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]
+            L.w4a16_gemm_gate_up.restype = _i
+            L.w4a16_gemm_gate_up_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _sz, _u, _vp]
+            L.w4a16_gemm_gate_up_ws.restype = _i
             L.w4a16_dequant_debug.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _vp]
             L.w4a16_dequant_debug.restype = _i
             L.w4a16_device_status.argtypes = [_vp, ctypes.POINTER(_i)]
@@ -186,6 +192,7 @@ class PackedWeight:
     M: int
     K: int
     group: int = GROUP
+    mi: int = 0        # > 0: packed in the gate/up row order (w4a16_pack_gate_up), M = 2 mi
 
     @property
     def nbytes(self) -> int:
@@ -256,6 +263,65 @@ def pack(q, scales, zeros, group: int = GROUP, out: PackedWeight | None = None,
                             _ptr(out.wq), _ptr(out.scales), _ptr(out.zeros),
                             _stream_ptr(stream)), "w4a16_pack")
     return out
+
+
+def pack_gate_up(q, scales, zeros, group: int = GROUP, out: PackedWeight | None = None,
+                 stream=None) -> PackedWeight:
+    """Canonical device tensors of a [2 Mi, K] weight whose rows are the gate
+    projection then the up projection -> packed buffers in the gate/up row
+    order, via w4a16_pack_gate_up."""
+    M, K = q.shape
+    if M % 2:
+        raise ValueError("the gate/up weight has 2 Mi rows")
+    for t in (q, scales, zeros):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("pack_gate_up expects contiguous CUDA tensors")
+    if out is None:
+        out = empty_packed(M, K, q.device, group)
+    out.mi = M // 2
+    _check(lib().w4a16_pack_gate_up(_ptr(q), _ptr(scales), _ptr(zeros), M // 2, K, group,
+                                    _ptr(out.wq), _ptr(out.scales), _ptr(out.zeros),
+                                    _stream_ptr(stream)), "w4a16_pack_gate_up")
+    return out
+
+
+def _gate_up_args(w: PackedWeight, X, H):
+    import torch
+
+    if not w.mi:
+        raise ValueError("the weight must be packed with pack_gate_up")
+    N, K = X.shape
+    if K != w.K or X.dtype != torch.float16 or not X.is_cuda or not X.is_contiguous():
+        raise ValueError("X must be a contiguous CUDA fp16 [N, K] tensor")
+    if H is None:
+        H = torch.empty((N, w.mi), dtype=torch.float16, device=X.device)
+    elif H.dtype != torch.float16 or not H.is_cuda or not H.is_contiguous() or tuple(H.shape) != (N, w.mi):
+        raise ValueError("H must be a contiguous CUDA fp16 [N, Mi] tensor")
+    return N, K, H
+
+
+def gemm_gate_up(w: PackedWeight, X, H=None, stream=None):
+    """H [N, Mi] = silu(X . W_gate^T) * (X . W_up^T), fp16, via w4a16_gemm_gate_up."""
+    N, K, H = _gate_up_args(w, X, H)
+    _check(lib().w4a16_gemm_gate_up(_ptr(w.wq), _ptr(w.scales), _ptr(w.zeros), _ptr(X), _ptr(H), w.mi, K, N,
+                                    w.group, _stream_ptr(stream)), "w4a16_gemm_gate_up")
+    return H
+
+
+def gemm_gate_up_ws(w: PackedWeight, X, H=None, path: int = PATH_AUTO, workspace: Workspace | None = None,
+                    flags: int = 0, stream=None):
+    """gemm_gate_up through w4a16_gemm_gate_up_ws (forced path, workspace)."""
+    import torch
+
+    N, K, H = _gate_up_args(w, X, H)
+    st = torch.cuda.current_stream(X.device) if stream is None else stream
+    ws = workspace if workspace is not None else default_workspace(X.device, st)
+    need = workspace_size(w.M, K, N, w.group) if path in (PATH_AUTO, PATH_GEMV_TC) else 0
+    ws.ensure(need)
+    _check(lib().w4a16_gemm_gate_up_ws(_ptr(w.wq), _ptr(w.scales), _ptr(w.zeros), _ptr(X), _ptr(H), w.mi, K, N,
+                                       w.group, path, _ptr(ws.buf), ws.nbytes, int(flags),
+                                       _vp(st.cuda_stream)), "w4a16_gemm_gate_up_ws")
+    return H
 
 
 def gemm_ex(w: PackedWeight, X, Y=None, path: int = PATH_AUTO, stream=None):

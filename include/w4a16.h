@@ -154,6 +154,48 @@ W4A16_API w4a16_status w4a16_pack(const uint8_t* q, const uint16_t* scales, cons
                         void* stream);
 
 /*
+ * The gate/up row order, for w4a16_gemm_gate_up: canonical -> packed like
+ * w4a16_pack, for a weight of 2 * Mi rows whose rows [0, Mi) are the gate
+ * projection and rows [Mi, 2 Mi) the up projection (q [2 Mi][K], scales and
+ * zeros [2 Mi][K/128], as w4a16_pack).  Packed block b (128 rows) holds the
+ * intermediate channels i = 64 b + 16 q + j (q = 0..3, j = 0..15): the gate
+ * row of channel i as packed row 32 q + j, its up row as packed row
+ * 32 q + 16 + j; rows of channels i >= Mi are zero.  Output sizes are those
+ * of w4a16_packed_sizes(2 * Mi, K, group).  Errors as w4a16_pack, plus
+ * W4A16_ERR_INVALID_ARG for Mi <= 0.
+ */
+W4A16_API w4a16_status w4a16_pack_gate_up(const uint8_t* q, const uint16_t* scales, const uint8_t* zeros,
+                                int Mi, int K, int group,
+                                void* wq_packed, void* scales_packed, void* zeros_packed,
+                                void* stream);
+
+/*
+ * The gate/up projection with its activation fused into the epilogue
+ * ("PerfXLLM on Snapdragon 8 Gen2", section 3.2: operator fusion removes an
+ * intermediate's write to and read from global memory; the page lists the
+ * add + normalisation, merged-QKV and attention fusions, and this extends the
+ * principle to the feed-forward block).  With g and u the fp32 accumulators
+ * of channel i's gate and up rows (as w4a16_gemm computes them):
+ *     H[n][i] = fp16_RN(silu(g) * u),   silu(g) = g / (1 + e^(-g)),
+ * in fp32, one rounding to fp16; the [N][2 Mi] product is never written.
+ *   wq_packed, scales_packed, zeros_packed: packed by w4a16_pack_gate_up
+ *   X  device fp16 [N][K];  H  device fp16 [N][Mi] (token-major), written in full.
+ * Kernel choice as w4a16_gemm for M = 2 Mi; errors as w4a16_gemm, plus
+ * W4A16_ERR_INVALID_ARG for Mi <= 0.
+ */
+W4A16_API w4a16_status w4a16_gemm_gate_up(const void* wq_packed, const void* scales_packed,
+                                const void* zeros_packed, const uint16_t* X, uint16_t* H,
+                                int Mi, int K, int N, int group, void* stream);
+
+/* w4a16_gemm_gate_up with a forced path (w4a16_path) and the workspace and
+ * flags of w4a16_gemm_ws (workspace size: w4a16_gemm_workspace_size(2 Mi, K,
+ * N, group)). */
+W4A16_API w4a16_status w4a16_gemm_gate_up_ws(const void* wq_packed, const void* scales_packed,
+                                   const void* zeros_packed, const uint16_t* X, uint16_t* H,
+                                   int Mi, int K, int N, int group, int path,
+                                   void* workspace, size_t workspace_bytes, unsigned flags, void* stream);
+
+/*
  * Y[N][M] = X[N][K] . dequant(W)[M][K]^T   (fp16 in, fp32 accumulate, fp16 out)
  *   wq_packed, scales_packed, zeros_packed: device, packed as above.
  *   X  device fp16 [N][K] (token-major), 16-byte aligned.

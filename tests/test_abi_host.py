@@ -261,3 +261,32 @@ def test_workspace_entry_points_reject_bad_arguments_without_launching(L):
     assert qkv(Yv=ws + 64) == w4a16.ERR_INVALID_ARG              # Yv inside the workspace
     assert qkv(flags=2) == w4a16.ERR_INVALID_ARG
     assert qkv(W=ws + 8) == w4a16.ERR_MISALIGNED
+
+
+def test_gate_up_entry_points_reject_bad_arguments_without_launching(L):
+    """Mi = 128 (weight 256 x 256), N = 2; fake buffers 1 MB apart."""
+    p = lambda a: ctypes.c_void_p(a)
+    wq, sc, zp, x, h, ws, q = (k << 20 for k in range(1, 8))
+    null = p(0)
+    pk = L.w4a16_pack_gate_up
+    assert pk(p(q), p(sc), p(zp), 0, 256, 128, p(wq), p(ws), p(h), null) == w4a16.ERR_INVALID_ARG
+    assert pk(p(q), p(sc), p(zp), 128, 200, 128, p(wq), p(ws), p(h), null) == w4a16.ERR_UNSUPPORTED
+    assert pk(p(q), p(sc), p(zp), 128, 256, 128, p(wq + 8), p(ws), p(h), null) == w4a16.ERR_MISALIGNED
+    assert pk(p(q), p(sc), p(zp), 128, 256, 128, p(q + 0x100), p(ws), p(h), null) == w4a16.ERR_INVALID_ARG
+    g = L.w4a16_gemm_gate_up
+    assert g(p(wq), p(sc), p(zp), p(x), null, 128, 256, 2, 128, null) == w4a16.ERR_INVALID_ARG
+    assert g(p(wq), p(sc), p(zp), p(x), p(h), 0, 256, 2, 128, null) == w4a16.ERR_INVALID_ARG
+    assert g(p(wq), p(sc), p(zp), p(x), p(h), 128, 256, 2, 64, null) == w4a16.ERR_UNSUPPORTED
+    assert g(p(wq), p(sc), p(zp), p(x), p(h + 8), 128, 256, 2, 128, null) == w4a16.ERR_MISALIGNED
+    assert g(p(wq), p(sc), p(zp), p(x), p(x + 64), 128, 256, 2, 128, null) == w4a16.ERR_INVALID_ARG
+    assert g(p(wq), p(sc), p(zp), p(x), p(wq + 0x100), 128, 256, 2, 128, null) == w4a16.ERR_INVALID_ARG
+    gw = L.w4a16_gemm_gate_up_ws
+    need = w4a16.workspace_size(256, 256, 2)
+    GT = w4a16.PATH_GEMV_TC
+    assert gw(p(wq), p(sc), p(zp), p(x), p(h), 128, 256, 2, 128, GT, null, 0, 0, null) == w4a16.ERR_INVALID_ARG
+    assert gw(p(wq), p(sc), p(zp), p(x), p(h), 128, 256, 2, 128, GT, p(ws), need - 1, 0, null) == \
+        w4a16.ERR_INVALID_ARG
+    assert gw(p(wq), p(sc), p(zp), p(x), p(h), 128, 256, 2, 128, GT, p(h + 64), need, 0, null) == \
+        w4a16.ERR_INVALID_ARG                                    # workspace over H
+    assert gw(p(wq), p(sc), p(zp), p(x), p(h), 128, 256, 2, 128, 9, p(ws), need, 0, null) == \
+        w4a16.ERR_INVALID_ARG
