@@ -136,6 +136,21 @@ struct Cfg {
   static_assert((BN * 128) % 1024 == 0, "X slabs must stay 1024-byte aligned");
 };
 
+// Tile t -> (row tile mt, token tile nt).  Bands of kBand row tiles; inside
+// a band the token tiles run fastest, so the CTAs working at the same time
+// share a few weight blocks and every token tile of X in L2 instead of each
+// holding its own weight block (valid for t < mt_n * nt_n).
+constexpr int kBand = 8;
+
+__device__ __forceinline__ void tile_coords(int t, int mt_n, int nt_n, int& mt, int& nt) {
+  const int per_band = kBand * nt_n;
+  const int band = t / per_band;
+  const int rem = t - band * per_band;
+  const int bm = cmin(kBand, mt_n - band * kBand);
+  nt = rem / bm;
+  mt = band * kBand + (rem - nt * bm);
+}
+
 struct Shared {
   uint64_t* x_full;
   uint64_t* x_empty;
@@ -225,7 +240,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
       uint32_t issued_mask = 0, issued_par = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
-        const int nt = t / mt_n;
+        int mt, nt;
+        tile_coords(t, mt_n, nt_n, mt, nt);
         for (int xi = 0; xi < nx; ++xi) {
           if (!wait_bar(&sh.x_empty[xs], xph ^ 1, sh.abort_flag, &g_tc_status)) { ok = false; break; }
           ptx::mbar_arrive_expect_tx(&sh.x_full[xs], C::kXStageBytes);
@@ -308,12 +324,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
     // the tile, the tile's row block mt); advanced by kDqGroups slots at a
     // time without divisions.
     int f_i = gi, f_g = gi;
-    int f_mt = (int)blockIdx.x % mt_n;
-    while (f_g >= ks_n) { f_g -= ks_n; f_mt = (f_mt + (int)gridDim.x) % mt_n; }
+    int f_t = (int)blockIdx.x, f_mt = 0, f_nt = 0;
+    while (f_g >= ks_n) { f_g -= ks_n; f_t += (int)gridDim.x; }
+    if (f_t < tiles) tile_coords(f_t, mt_n, nt_n, f_mt, f_nt);
     auto advance = [&]() {
       f_i += kDqGroups;
       f_g += kDqGroups;
-      while (f_g >= ks_n) { f_g -= ks_n; f_mt += (int)gridDim.x; if (f_mt >= mt_n) f_mt %= mt_n; }
+      bool moved = false;
+      while (f_g >= ks_n) { f_g -= ks_n; f_t += (int)gridDim.x; moved = true; }
+      if (moved && f_t < tiles) tile_coords(f_t, mt_n, nt_n, f_mt, f_nt);
     };
     int a = gi % C::kASlots;
     uint32_t aph = (uint32_t)((gi / C::kASlots) & 1);
@@ -341,16 +360,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
         ptx::tc_fence_after();
 #pragma unroll
         for (int hlf = 0; hlf < C::kChunks / 2; ++hlf) {
-          uint32_t h[32];
+          // 16 columns at a time: with the next slot's codes held in
+          // registers, a 32-column buffer would not fit the thread's share.
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
+            uint32_t h[16];
             const uint4 w = cur[hlf * 2 + c];
-            dequant_word(w.x, gc, &h[c * 16 + 0]);
-            dequant_word(w.y, gc, &h[c * 16 + 4]);
-            dequant_word(w.z, gc, &h[c * 16 + 8]);
-            dequant_word(w.w, gc, &h[c * 16 + 12]);
+            dequant_word(w.x, gc, &h[0]);
+            dequant_word(w.y, gc, &h[4]);
+            dequant_word(w.z, gc, &h[8]);
+            dequant_word(w.w, gc, &h[12]);
+            ptx::tmem_st_x16(a_lane + a * C::kAColsPerSlot + hlf * 32 + c * 16, h);
           }
-          ptx::tmem_st_x32(a_lane + a * C::kAColsPerSlot + hlf * 32, h);
         }
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
@@ -445,7 +466,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
     int b = 0;
     uint32_t bph = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
-      const int mt = t % mt_n, nt = t / mt_n;
+      int mt, nt;
+      tile_coords(t, mt_n, nt_n, mt, nt);
       const int m = mt * kBM + row;
       const int n0 = nt * BN + col0;
       // The fused form's destination and bias of this row, loaded before the

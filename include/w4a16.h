@@ -73,6 +73,10 @@ W4A16_API const char* w4a16_status_string(int status);
 
 /*
  * Packed-weight sizes, in bytes, for an M x K weight with the given group.
+ * "PerfXLLM on Snapdragon 8 Gen2", section 3.1: int4 codes take a quarter of
+ * the fp16 weight and the scale and zero of each group of 128 about 1 % more;
+ * the layout below is this library's own (section 3.3 asks for vectorised
+ * weight loads, which the 16-byte row-interleaved chunks serve).
  *
  * Packed layout (all three buffers are padded to Mp = ceil(M / 128) * 128 rows;
  * padding rows hold q = 0, z = 0, s = 0, i.e. zero weights):
@@ -141,6 +145,10 @@ W4A16_API w4a16_status w4a16_add_rmsnorm(const uint16_t* h, const uint16_t* d, c
 
 /*
  * Canonical -> packed layout (offline; not on the per-token path).
+ * "PerfXLLM on Snapdragon 8 Gen2", section 3.1 (int4 codes, group 128, a
+ * scale and a zero per group) and section 3.3 (vectorised weight access).
+ * Argument order: codes, then the fp16 scales, then the zeros (the order of
+ * the packed buffers w4a16_packed_sizes reports).
  *   q       device uint8  [M][K], values 0..15 (higher bits are ignored)
  *   scales  device fp16   [M][K/128]
  *   zeros   device uint8  [M][K/128], values 0..15 (higher bits are ignored)
@@ -197,6 +205,9 @@ W4A16_API w4a16_status w4a16_gemm_gate_up_ws(const void* wq_packed, const void* 
 
 /*
  * Y[N][M] = X[N][K] . dequant(W)[M][K]^T   (fp16 in, fp32 accumulate, fp16 out)
+ * "PerfXLLM on Snapdragon 8 Gen2", section 3.3 item 1 (C[m, n] = A[m, k]
+ * B[k, n]) and item 2 (the GEMV is its n = 1 case); the weight is the
+ * section 3.1 int4 group-128 format.
  *   wq_packed, scales_packed, zeros_packed: device, packed as above.
  *   X  device fp16 [N][K] (token-major), 16-byte aligned.
  *   Y  device fp16 [N][M] (token-major), 16-byte aligned; fully overwritten.
@@ -272,13 +283,18 @@ W4A16_API w4a16_status w4a16_gemm_qkv_ws(const void* wq_packed, const void* scal
                                void* workspace, size_t workspace_bytes, unsigned flags, void* stream);
 
 /* As w4a16_gemm, with the kernel forced (w4a16_path).  W4A16_PATH_AUTO is the
- * same as w4a16_gemm.  Used by tests and the benchmark to time both paths. */
+ * same as w4a16_gemm.  Used by tests and the benchmark to time the kernels
+ * side by side ("PerfXLLM on Snapdragon 8 Gen2", section 3.3 item 1: each
+ * regime, few tokens or many, gets its own tiling).  W4A16_PATH_GEMV_TC needs
+ * a workspace, so it is W4A16_ERR_INVALID_ARG here (use w4a16_gemm_ws). */
 W4A16_API w4a16_status w4a16_gemm_ex(const void* wq_packed, const void* scales_packed,
                            const void* zeros_packed, const uint16_t* X, uint16_t* Y,
                            int M, int K, int N, int group, int path, void* stream);
 
 /* The path w4a16_gemm would take for these sizes (a w4a16_path value other
- * than AUTO), or -1 if the sizes are invalid.  Host only; touches no GPU. */
+ * than AUTO), or -1 if the sizes are invalid.  Host only; touches no GPU.
+ * "PerfXLLM on Snapdragon 8 Gen2", section 3.3 item 1: the operator switches
+ * tiling with the number of tokens; the crossovers here are measured. */
 W4A16_API int w4a16_select_path(int M, int K, int N);
 
 /* The path w4a16_gemm_ws with a workspace would take. */
@@ -286,7 +302,9 @@ W4A16_API int w4a16_select_path_ws(int M, int K, int N);
 
 /*
  * Writes the dequantised weight W[m][k] = fp16_RN((q - z) * s) as fp16,
- * row-major [M][K], from the packed buffers.  The values are bit-identical to
+ * row-major [M][K], from the packed buffers ("PerfXLLM on Snapdragon 8 Gen2",
+ * section 3.1: int4 with a scale and a zero per group of 128; the formula and
+ * its single rounding are this library's reading of that passage).  The values are bit-identical to
  * what the GEMM kernels multiply; parity checks compare them with an
  * independent CPU computation.
  */
