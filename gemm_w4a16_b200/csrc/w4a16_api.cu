@@ -65,7 +65,7 @@ w4a16_status map_cuda(cudaError_t e) {
 // with_ws: a workspace is available, which opens the split decode kernel.
 int select_path_impl(int M, int K, int N, bool with_ws) {
   if (M <= 0 || K <= 0 || N <= 0 || K % kGroup) return -1;
-  if (with_ws && N <= kGemvTcMaxTokens) return W4A16_PATH_GEMV_TC;
+  if (with_ws && N <= kGemvTcAutoTokens) return W4A16_PATH_GEMV_TC;
   return N <= gemv_max_n() ? W4A16_PATH_GEMV : W4A16_PATH_TC;
 }
 
@@ -361,7 +361,8 @@ w4a16_status w4a16_gemm_workspace_size(int M, int K, int N, int group, size_t* b
   w4a16_status st = check_shape(M, K, group);
   if (st != W4A16_OK) return st;
   if (N > kMaxN) return W4A16_ERR_UNSUPPORTED;
-  *bytes = workspace_for(select_path_impl(M, K, N, true), M, K, N);
+  // Enough for the automatic choice and for a forced W4A16_PATH_GEMV_TC.
+  *bytes = N <= kGemvTcMaxTokens ? workspace_for(W4A16_PATH_GEMV_TC, M, K, N) : 0;
   return W4A16_OK;
 }
 

@@ -330,38 +330,59 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
       if constexpr (kEpi == kEpiQkv) {
         if (m < M) rd = row_dst(om, M, m);
       }
+      // Tokens 8 h .. 8 h + 7 of row m: rounded once and written (whole
+      // warps call this: the gate/up pairing shuffles).
+      auto store8 = [&](int h, const float (&v)[8]) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int n = h * 8 + j;
+          if constexpr (kEpi == kEpiGateUp) {
+            store_gate_up(om, b, row, n, v[j], n < N);
+          } else if (n < N && m < M) {
+            if constexpr (kEpi == kEpiQkv) store_row(rd, om.bias != nullptr, n, v[j]);
+            else Y[(size_t)n * M + m] = __half_as_ushort(__float2half_rn(v[j]));
+          }
+        }
+      };
       if (!wait_bar_warp(&acc_full[buf], (uint32_t)((bi / C::kAccBufs) & 1), abort_flag, &g_gvtc_status)) break;
       ptx::tc_fence_after();
-      float acc[BN];
-      bool have = false;
+      const bool whole = span == kg;
+      // A split block's fp32 share goes to this CTA's workspace slot (0 for
+      // the CTA's first block, 1 for its last).
+      float* part = ws_part + (size_t)(c * 2 + (bi == 0 ? 0 : 1)) * N * kRowBlock + row;
+      // Eight tokens at a time, up to the last real one: the issuers'
+      // accumulators in issuer order.
+      const int chunks = ((N < BN ? N : BN) + 7) / 8;
+#pragma unroll 1
+      for (int h = 0; h < chunks; ++h) {
+        float v[8];
+        bool have = false;
 #pragma unroll
-      for (int p = 0; p < C::kIss; ++p) {
-        // Issuer p owns a unit of this block iff one of i0 .. i1 - 1 is p mod kIss.
-        if (span < C::kIss && ((p - i0 % C::kIss) + C::kIss) % C::kIss >= span) continue;
-#pragma unroll
-        for (int h = 0; h < BN / 16; ++h) {
-          uint32_t v[16];
-          ptx::tmem_ld_x16(lane_base + buf * C::kAccCols + p * BN + h * 16, v);
+        for (int p = 0; p < C::kIss; ++p) {
+          // Issuer p owns a unit of this block iff one of i0 .. i1 - 1 is p mod kIss.
+          if (span < C::kIss && ((p - i0 % C::kIss) + C::kIss) % C::kIss >= span) continue;
+          uint32_t t[8];
+          ptx::tmem_ld_x8(lane_base + buf * C::kAccCols + p * BN + h * 8, t);
           ptx::tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) acc[h * 16 + j] = have ? acc[h * 16 + j] + __uint_as_float(v[j])
-                                                              : __uint_as_float(v[j]);
+          for (int j = 0; j < 8; ++j) v[j] = have ? v[j] + __uint_as_float(t[j]) : __uint_as_float(t[j]);
+          have = true;
         }
-        have = true;
+        if (whole) {
+          store8(h, v);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (h * 8 + j < N) part[(size_t)(h * 8 + j) * kRowBlock] = v[j];
+        }
       }
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&acc_empty[buf]);
 
-      bool write = span == kg;
-      if (!write) {
-        // Partial of a split block: this CTA's fp32 share to the workspace;
-        // the last of the block's CTAs (per lane quarter) sums them all.
-        const int slot = bi == 0 ? 0 : 1;
-        float* part = ws_part + (size_t)(c * 2 + slot) * N * kRowBlock + row;
-#pragma unroll
-        for (int n = 0; n < BN; ++n)
-          if (n < N) part[(size_t)n * kRowBlock] = acc[n];
+      if (!whole) {
+        // The last of the block's CTAs (per lane quarter) adds every CTA's
+        // partial in CTA order and writes the row.
         __threadfence();
         __syncwarp();
         uint32_t old = 0;
@@ -371,32 +392,21 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
         const int cl = cta_of(U, G, (long long)(b + 1) * kg - 1);
         if (old == (uint32_t)(cl - cf)) {
           __threadfence();
+#pragma unroll 1
+          for (int h = 0; h < chunks; ++h) {
+            float v[8];
 #pragma unroll
-          for (int n = 0; n < BN; ++n) acc[n] = 0.f;
-          for (int cc = cf; cc <= cl; ++cc) {
-            const int sl = (long long)b == unit_start(U, G, cc) / kg ? 0 : 1;
-            const float* pp = ws_part + (size_t)(cc * 2 + sl) * N * kRowBlock + row;
+            for (int j = 0; j < 8; ++j) v[j] = 0.f;
+            for (int cc = cf; cc <= cl; ++cc) {
+              const int sl = (long long)b == unit_start(U, G, cc) / kg ? 0 : 1;
+              const float* pp = ws_part + (size_t)(cc * 2 + sl) * N * kRowBlock + row;
 #pragma unroll
-            for (int n = 0; n < BN; ++n)
-              if (n < N) acc[n] += __ldcg(pp + (size_t)n * kRowBlock);
+              for (int j = 0; j < 8; ++j)
+                if (h * 8 + j < N) v[j] += __ldcg(pp + (size_t)(h * 8 + j) * kRowBlock);
+            }
+            store8(h, v);
           }
           if (lane == 0) ws_cnt[b * 4 + quad] = 0u;
-          write = true;
-        }
-      }
-      if constexpr (kEpi == kEpiGateUp) {
-        // `write` is the same on every lane: the gate/up pairing shuffles.
-        if (write) {
-#pragma unroll
-          for (int n = 0; n < BN; ++n) store_gate_up(om, b, row, n, acc[n], n < N);
-        }
-      } else if (write && m < M) {
-#pragma unroll
-        for (int n = 0; n < BN; ++n) {
-          if (n < N) {
-            if constexpr (kEpi == kEpiQkv) store_row(rd, om.bias != nullptr, n, acc[n]);
-            else Y[(size_t)n * M + m] = __half_as_ushort(__float2half_rn(acc[n]));
-          }
         }
       }
     }
@@ -410,8 +420,15 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
   }
 }
 
-// Few tokens: three dequantiser groups, three issuers, one accumulator set.
+// Up to 16 tokens: three dequantiser groups, three issuers, one accumulator
+// set, six stages of 12.3 KB.
 using Cfg16 = GtCfg<16, 3, 3, 3, 1, 6>;
+// Up to 32 tokens: two groups, two issuers, two accumulator sets, six
+// stages of 16.3 KB.
+using Cfg32 = GtCfg<32, 2, 2, 2, 2, 6>;
+// Up to 64 tokens: two groups, two issuers, one accumulator set, four
+// stages of 24.3 KB.
+using Cfg64 = GtCfg<64, 2, 2, 2, 1, 4>;
 
 int grid_for(int M, int K) {
   const long long U = (long long)ceil_div(M, kRowBlock) * (K / kGroup);
@@ -459,10 +476,21 @@ cudaError_t launch_gemv_tc(const uint8_t* wq, const uint16_t* scales, const uint
                            uint16_t* Y, int M, int K, int N, void* workspace, bool pdl, cudaStream_t stream,
                            const OutMap* om) {
   if (N > kGemvTcMaxTokens) return cudaErrorNotSupported;
-  if (om && om->kind == kEpiGateUp)
-    return launch_cfg<Cfg16, kEpiGateUp>(wq, scales, zeros, X, nullptr, M, K, N, workspace, pdl, stream, *om);
-  if (om) return launch_cfg<Cfg16, kEpiQkv>(wq, scales, zeros, X, nullptr, M, K, N, workspace, pdl, stream, *om);
-  return launch_cfg<Cfg16, kEpiPlain>(wq, scales, zeros, X, Y, M, K, N, workspace, pdl, stream, OutMap{});
+  const int kind = om ? om->kind : kEpiPlain;
+  const OutMap o = om ? *om : OutMap{};
+  uint16_t* y = om ? nullptr : Y;
+#define W4A16_GVTC(CFG)                                                                               \
+  do {                                                                                                \
+    if (kind == kEpiGateUp) return launch_cfg<CFG, kEpiGateUp>(wq, scales, zeros, X, y, M, K, N,      \
+                                                                workspace, pdl, stream, o);           \
+    if (kind == kEpiQkv) return launch_cfg<CFG, kEpiQkv>(wq, scales, zeros, X, y, M, K, N, workspace, \
+                                                         pdl, stream, o);                             \
+    return launch_cfg<CFG, kEpiPlain>(wq, scales, zeros, X, y, M, K, N, workspace, pdl, stream, o);   \
+  } while (0)
+  if (N <= 16) W4A16_GVTC(Cfg16);
+  if (N <= 32) W4A16_GVTC(Cfg32);
+  W4A16_GVTC(Cfg64);
+#undef W4A16_GVTC
 }
 
 cudaError_t read_and_clear_gvtc_status(int* v) {

@@ -256,7 +256,9 @@ cudaError_t launch_gemm_tc(const uint8_t* wq, const uint16_t* scales, const uint
 // calls, then the fp32 partials of the blocks split between CTAs.  With pdl
 // the launch may overlap the previous kernel in the stream: the weights are
 // read before the grid dependency wait, X, Y and the workspace after it.
-constexpr int kGemvTcMaxTokens = 16;
+constexpr int kGemvTcMaxTokens = 64;
+// Tokens up to which the automatic choice (with a workspace) takes it.
+constexpr int kGemvTcAutoTokens = 16;
 size_t gemv_tc_counter_bytes(int M);
 size_t gemv_tc_workspace_bytes(int M, int K, int N);
 cudaError_t launch_gemv_tc(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros, const uint16_t* X,

@@ -17,7 +17,13 @@
 // reduction gives the mean; pass 2 scales r from shared memory.  h and d are
 // read once and r and X written once: 8 bytes of HBM traffic per channel plus
 // gamma, which stays in L2 across rows.  Bound by HBM.
+//
+// The kernel lets the next kernel in the stream be scheduled as soon as it
+// starts (programmatic dependent launch): a projection launched with early
+// weight streaming then reads its weights while this runs, and reads X only
+// after this kernel has completed.
 #include "w4a16_internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace w4a16 {
 
@@ -65,6 +71,7 @@ add_rmsnorm_kernel(const uint16_t* h, const uint16_t* d, const uint16_t* __restr
   const uint4* hv = reinterpret_cast<const uint4*>(h) + base;
   const uint4* dv = d ? reinterpret_cast<const uint4*>(d) + base : nullptr;
   uint4* rv = r_out ? reinterpret_cast<uint4*>(r_out) + base : nullptr;
+  ptx::griddep_launch_dependents();
 
   float ss = 0.0f;
   for (int c0 = threadIdx.x; c0 < chunks; c0 += kNormThreads * kNormBatch) {

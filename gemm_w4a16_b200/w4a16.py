@@ -17,7 +17,8 @@ LIB_PATH = os.path.join(HERE, "libw4a16.so")
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_CUDA, ERR_TIMEOUT = range(6)
 PATH_AUTO, PATH_GEMV, PATH_TC, PATH_GEMV_TC = 0, 1, 2, 3
 FLAG_EARLY_WEIGHTS = 1
-GEMV_TC_MAX_TOKENS = 16
+GEMV_TC_MAX_TOKENS = 64      # forced W4A16_PATH_GEMV_TC
+GEMV_TC_AUTO_TOKENS = 16     # AUTO with a workspace takes it up to here
 GROUP = 128
 
 EXPORTED = (
@@ -135,8 +136,9 @@ def select_path_ws(M: int, K: int, N: int) -> int:
 
 
 def workspace_size(M: int, K: int, N: int, group: int = GROUP) -> int:
-    """Bytes of workspace w4a16_gemm_ws needs for these sizes on the current
-    device (0 when its automatic choice needs none)."""
+    """Bytes of workspace the workspace entry points need for these sizes on
+    the current device (automatic choice or forced split decode path; 0 for
+    N > 64)."""
     n = ctypes.c_size_t()
     _check(lib().w4a16_gemm_workspace_size(M, K, N, group, ctypes.byref(n)), "w4a16_gemm_workspace_size")
     return n.value

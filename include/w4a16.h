@@ -56,7 +56,7 @@ typedef enum {
     W4A16_PATH_GEMV = 1,     /* CUDA-core decode kernel (any N, best at one or two tokens) */
     W4A16_PATH_TC = 2,       /* tcgen05 tile kernel (any N, best from a few tokens on) */
     W4A16_PATH_GEMV_TC = 3   /* tcgen05 decode kernel, weight stream split over every SM
-                                (N <= 16; needs a workspace) */
+                                (N <= 64; needs a workspace; AUTO takes it for N <= 16) */
 } w4a16_path;
 
 /* Flags of the workspace entry points (w4a16_gemm_ws, w4a16_gemm_qkv_ws). */
@@ -238,9 +238,10 @@ W4A16_API w4a16_status w4a16_gemm_qkv(const void* wq_packed, const void* scales_
                             uint16_t* Yq, uint16_t* Yk, uint16_t* Yv, void* stream);
 
 /*
- * Workspace of w4a16_gemm_ws / w4a16_gemm_qkv_ws for an M x K weight and N
- * tokens on the current device (it depends on the device's SM count), in
- * bytes; 0 when the automatic choice for these sizes needs none.  The size
+ * Workspace of w4a16_gemm_ws / w4a16_gemm_qkv_ws / w4a16_gemm_gate_up_ws
+ * for an M x K weight and N tokens on the current device (it depends on the
+ * device's SM count), in bytes: enough for the automatic choice and for a
+ * forced W4A16_PATH_GEMV_TC; 0 for N > 64, where no path needs one.  The size
  * grows with N, so a workspace sized for the largest N serves every smaller
  * one.  W4A16_ERR_INVALID_ARG / W4A16_ERR_UNSUPPORTED as w4a16_gemm.
  */
@@ -251,7 +252,7 @@ W4A16_API w4a16_status w4a16_gemm_workspace_size(int M, int K, int N, int group,
  * few-token product run on every SM ("PerfXLLM on Snapdragon 8 Gen2",
  * section 3.3 item 2: the GEMV is memory bound; the weight is tiled along
  * both its rows and K so the whole device streams it).  With path AUTO and
- * N <= 16 this is W4A16_PATH_GEMV_TC: CTA c of G streams units
+ * N <= 16 (or forced, N <= 64) this is W4A16_PATH_GEMV_TC: CTA c of G streams units
  * [c U / G, (c + 1) U / G) of the U = ceil(M/128) * K/128 (row block, group)
  * units; a block split between CTAs is summed, in CTA order, from fp32
  * partials in the workspace, so the result stays deterministic.

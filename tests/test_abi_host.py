@@ -201,16 +201,16 @@ def test_workspace_size_closed_form(L):
     """Workspace of the split decode path: one counter per (row block, lane
     quarter), rounded up to 256 bytes, then per CTA two fp32 partials of
     128 rows x N tokens; G = min(SMs, units) CTAs.  Zero where the automatic
-    choice needs no workspace (N > 16)."""
+    path needs a workspace (N > 64)."""
     for M, K in [(12288, 4096), (4096, 11008), (200, 384), (128256, 4096)]:
         nb, U = -(-M // 128), -(-M // 128) * (K // 128)
         cnt = -(-nb * 16 // 256) * 256
         one = w4a16.workspace_size(M, K, 1)
         G = (one - cnt) // 1024
         assert (one - cnt) % 1024 == 0 and 1 <= G <= U
-        for N in (2, 7, 16):
+        for N in (2, 7, 16, 17, 64):
             assert w4a16.workspace_size(M, K, N) == cnt + G * 2 * N * 128 * 4
-        assert w4a16.workspace_size(M, K, 17) == 0
+        assert w4a16.workspace_size(M, K, 65) == 0
     n = ctypes.c_size_t()
     assert L.w4a16_gemm_workspace_size(256, 256, 1, 128, None) == w4a16.ERR_INVALID_ARG
     assert L.w4a16_gemm_workspace_size(256, 256, 0, 128, ctypes.byref(n)) == w4a16.ERR_INVALID_ARG
@@ -248,7 +248,7 @@ def test_workspace_entry_points_reject_bad_arguments_without_launching(L):
     assert call(W=y - 16) == w4a16.ERR_INVALID_ARG               # workspace runs into Y
     assert call(W=x + 256) == w4a16.ERR_INVALID_ARG              # workspace on X
     assert call(W=wq + 0x100) == w4a16.ERR_INVALID_ARG           # workspace inside the codes
-    assert call(N=17, nbytes=1 << 20) == w4a16.ERR_UNSUPPORTED   # more tokens than the kernel takes
+    assert call(N=65, nbytes=1 << 24) == w4a16.ERR_UNSUPPORTED   # more tokens than the kernel takes
     assert L.w4a16_gemm_ex(p(wq), p(sc), p(zp), p(x), p(y), 256, 256, 2, 128, GT, null) == \
         w4a16.ERR_INVALID_ARG                                    # no workspace on this entry point
 

@@ -56,7 +56,8 @@ def test_auto_choice_with_workspace():
     assert w4a16.select_path_ws(12288, 4096, 1) == GT
     assert w4a16.select_path_ws(12288, 4096, 16) == GT
     assert w4a16.select_path_ws(12288, 4096, 17) == w4a16.PATH_TC
-    assert w4a16.workspace_size(12288, 4096, 17) == 0
+    assert w4a16.workspace_size(12288, 4096, 17) > 0      # a forced split path up to 64 tokens
+    assert w4a16.workspace_size(12288, 4096, 65) == 0
     assert w4a16.workspace_size(12288, 4096, 1) > 0
 
 
@@ -76,8 +77,10 @@ def test_ragged_and_few_unit_shapes(M, K, N):
     full_case(M, K, N, seed=M + K + N)
 
 
-@pytest.mark.parametrize("N", list(range(1, 17)))
+@pytest.mark.parametrize("N", list(range(1, 17)) + [17, 24, 31, 32, 33, 40, 48, 63, 64])
 def test_every_token_count(N):
+    """Every N of the 16-token configuration, then the 32- and 64-token ones
+    around their edges."""
     full_case(1536, 2048, N, seed=100 + N)
 
 
@@ -117,12 +120,12 @@ def test_llama7b_decode_n1_full(M, K):
     full_case(M, K, 1, seed=M + K)
 
 
-@pytest.mark.parametrize("N", [2, 4, 8, 16])
+@pytest.mark.parametrize("N", [2, 4, 8, 16, 32, 64])
 def test_qkv_few_tokens_full(N):
     full_case(12288, 4096, N, seed=N)
 
 
-@pytest.mark.parametrize("N", [1, 16])
+@pytest.mark.parametrize("N", [1, 16, 64])
 @pytest.mark.parametrize("M,K", LLAMA3)
 def test_llama3_batched_decode_full(M, K, N):
     full_case(M, K, N, seed=M + N)
@@ -192,10 +195,10 @@ def test_argument_checks():
     assert L.w4a16_gemm_ws(*args[:4], ws.data_ptr(), M, K, N, 128, GT, ws.data_ptr(), need, 0,
                            s) == w4a16.ERR_INVALID_ARG
     # More tokens than the split kernel takes.
-    x17 = torch.zeros((17, K), dtype=torch.float16, device="cuda")
-    y17 = torch.empty((17, M), dtype=torch.float16, device="cuda")
-    assert L.w4a16_gemm_ws(w.wq.data_ptr(), w.scales.data_ptr(), w.zeros.data_ptr(), x17.data_ptr(),
-                           y17.data_ptr(), M, K, 17, 128, GT, ws.data_ptr(), ws.numel(), 0,
+    x65 = torch.zeros((65, K), dtype=torch.float16, device="cuda")
+    y65 = torch.empty((65, M), dtype=torch.float16, device="cuda")
+    assert L.w4a16_gemm_ws(w.wq.data_ptr(), w.scales.data_ptr(), w.zeros.data_ptr(), x65.data_ptr(),
+                           y65.data_ptr(), M, K, 65, 128, GT, ws.data_ptr(), ws.numel(), 0,
                            s) == w4a16.ERR_UNSUPPORTED
     # Null workspace: AUTO falls back to the workspace-free choice.
     assert L.w4a16_gemm_ws(*args, w4a16.PATH_AUTO, None, 0, 0, s) == w4a16.OK
