@@ -909,28 +909,29 @@ def add_rmsnorm_workload(args, device, peaks):
 
 
 def single_shape(args, device, M, K, N, path=0):
-    """One shape, plain launches (used for ncu captures and quick timing)."""
+    """One shape, plain launches through w4a16_gemm_ws (any path, with a
+    workspace; used for ncu captures and quick timing)."""
     import torch
 
     from gemm_w4a16_b200 import w4a16
 
-    peaks, _ = load_peaks()
     w, x = make_device_problem(device, M, K, N, seed=3)
     y = torch.empty((N, M), dtype=torch.float16, device=device)
+    ws = w4a16.Workspace(device, w4a16.workspace_size(M, K, N))
     for _ in range(args.warmup):
-        w4a16.gemm_ex(w, x, Y=y, path=path)
+        w4a16.gemm_ws(w, x, Y=y, path=path, workspace=ws)
     torch.cuda.synchronize(device)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(args.steps):
-        w4a16.gemm_ex(w, x, Y=y, path=path)
+        w4a16.gemm_ws(w, x, Y=y, path=path, workspace=ws)
     e1.record()
     torch.cuda.synchronize(device)
     ms = e0.elapsed_time(e1) / args.steps
     b, f = alg_bytes(M, K, N), alg_flops(M, K, N)
     print(json.dumps({"workload": f"M={M} K={K} N={N}", "us": ms * 1e3,
                       "GBps": b / (ms * 1e-3) / 1e9, "TFLOPS": f / (ms * 1e-3) / 1e12,
-                      "path": path or w4a16.select_path(M, K, N),
+                      "path": path or w4a16.select_path_ws(M, K, N),
                       "note": "plain launches; weights may sit in L2 across iterations"}))
     return 0
 
@@ -983,7 +984,8 @@ def main(argv=None):
     ap.add_argument("--M", type=int, default=12288)
     ap.add_argument("--K", type=int, default=4096)
     ap.add_argument("--N", type=int, default=1)
-    ap.add_argument("--path", type=int, default=0, help="0 auto, 1 GEMV, 2 tensor cores")
+    ap.add_argument("--path", type=int, default=0,
+                    help="0 auto, 1 CUDA-core GEMV, 2 tensor-core tiles, 3 split tensor-core decode")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-extra", action="store_true",

@@ -99,6 +99,12 @@ __device__ __forceinline__ void griddep_wait() {
 
 // ------------------------------------------------------- global atomics
 
+// Acquire-release fence at GPU scope (lighter than the sequentially
+// consistent fence __threadfence() issues).
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
   uint32_t old;
   asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");

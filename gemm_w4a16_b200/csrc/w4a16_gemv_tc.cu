@@ -51,58 +51,65 @@ constexpr int kUnitCodes = kRowBlock * kGroup / 2;    // 8192 B of codes per uni
 constexpr int kUnitS = kRowBlock * 2;                 // 256 B of scales
 constexpr int kUnitZ = kRowBlock / 2;                 // 64 B of zeros
 constexpr int kUnitW = kUnitCodes + kUnitS + kUnitZ;  // one weight stage
-constexpr int kACols = kGroup / 2;                    // TMEM columns of one unit's A (fp16 pairs)
+constexpr int kHalfK = kGroup / 2;                    // k per A slot: half a unit
+constexpr int kACols = kHalfK / 2;                    // TMEM columns of one A slot (fp16 pairs)
 
-// True when n = t a + u b for some t >= 1, u >= 0.
-__host__ __device__ constexpr bool reachable(int n, int a, int b) {
-  for (int t = 1; t * a <= n; ++t)
-    if ((n - t * a) % b == 0) return true;
-  return false;
-}
-
-template <int BN_, int DQ, int ISS, int ASLOTS, int ACCB, int STAGES>
+template <int BN_, int XROWS, int DQ, int ACCB, int WSTAGES, int XSTAGES>
 struct GtCfg {
-  static constexpr int BN = BN_;
+  static constexpr int BN = BN_;            // MMA N
+  // Token rows an activation tile holds: BN, or 8 when at most 8 tokens are
+  // real (the MMA's rows 8..15 then read the next 1 KB of shared memory,
+  // which only reaches accumulator columns that are never read).
+  static constexpr int kXRows = XROWS;
   static constexpr int kDq = DQ;            // dequantiser groups of four warps
-  static constexpr int kIss = ISS;          // MMA issuer warps, one accumulator each
-  static constexpr int kASlots = ASLOTS;    // TMEM A slots, one unit each
+  static constexpr int kIss = DQ;           // MMA issuer warps, one accumulator each
+  // TMEM A slots of half a unit (64 k): two per group, so the MMAs of one
+  // half run while the group dequantises the other.
+  static constexpr int kASlots = 2 * DQ;
   static constexpr int kAccBufs = ACCB;     // accumulator sets
-  static constexpr int kStages = STAGES;    // shared-memory stages, one unit each
-  static constexpr int kXBytes = BN * kGroup * 2;
+  // Two rings: weight stages of kDq consecutive units (one per dequantiser
+  // group; freed once every group has read its codes into registers),
+  // filled by the producer warp with three copies per stage (codes, scales,
+  // zeros) issued from three lanes at once; and one-unit activation tiles
+  // (freed by the MMAs' commit), filled by each issuer for its own units a
+  // few units ahead.  The weight stream is never held back by MMA latency,
+  // and a copy of the codes moves kDq x 8 KB.
+  static constexpr int kWStages = WSTAGES;
+  static constexpr int kStageBytes = DQ * kUnitW;
+  static constexpr int kXStages = XSTAGES;
+  static constexpr int kXAhead = XSTAGES / DQ;     // activation tiles in flight per issuer
+  static constexpr int kSlab = kXRows * 128;       // one 64-k slab of a tile
+  static constexpr int kXBytes = 2 * kSlab;
   static constexpr int kAccCols = kIss * BN;
   static constexpr int kACol0 = kAccBufs * kAccCols;
   static constexpr int kTmemCols = 256;
   static constexpr uint32_t kIdesc = ptx::idesc_f16_f32(kRowBlock, BN);
-  // Warps: 0..3 epilogue, 4..4+kIss-1 issuers, then the producer, then the
-  // dequantiser groups.
+  // Warps: 0..3 epilogue, 4..4+kIss-1 issuers, then the weight producer,
+  // then the dequantiser groups.
   static constexpr int kFirstIss = 4;
-  static constexpr int kProducer = kFirstIss + kIss;
-  static constexpr int kFirstDq = kProducer + 1;
+  static constexpr int kWProducer = kFirstIss + kIss;
+  static constexpr int kFirstDq = kWProducer + 1;
   static constexpr int kThreads = (kFirstDq + 4 * kDq) * 32;
   // Shared memory: X ring (1024-byte aligned tiles), weight ring, barriers.
   static constexpr int kXOff = 0;
-  static constexpr int kWOff = kStages * kXBytes;
-  static constexpr int kBarOff = kWOff + kStages * kUnitW;
-  static constexpr int kNumBars = 3 * kStages + 2 * kASlots + 2 * kAccBufs + 1;
+  static constexpr int kWOff = kXStages * kXBytes;
+  static constexpr int kBarOff = kWOff + kWStages * kStageBytes;
+  static constexpr int kNumBars = 2 * kWStages + 2 * kXStages + 2 * kASlots + 2 * kAccBufs + 1;
   static constexpr int kSmemBytes = kBarOff + 8 * kNumBars + 16 + 1024;
 
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 64, "MMA N");
   static_assert(kACol0 + kASlots * kACols <= kTmemCols, "TMEM budget");
   static_assert(kSmemBytes <= 113 * 1024, "two CTAs per SM");
   static_assert(kXBytes % 1024 == 0, "swizzled X tiles stay 1024-byte aligned");
+  static_assert(kXRows == BN || (kXRows == 8 && BN == 16), "activation tile rows");
+  static_assert(kXAhead >= 1, "activation tiles in flight");
   // A parity wait cannot tell a phase from the one two steps later.  The
-  // waits below stay exact when each waiter already knows the phase before
-  // the one it waits for is complete:
-  //  - stage barriers: every dequantiser group and every issuer sees each
-  //    stage it uses, in order (kDq | kStages, kIss | kStages);
-  //  - an A slot's "empty" barrier: the fill before the previous one was
-  //    freed, which a group knows from its own earlier wait plus the in-order
-  //    commits of one issuer (kASlots = t kDq + u kIss, t >= 1);
-  //  - an A slot's "full" barrier: the fill before the one awaited is known
-  //    to be done from the issuer's own earlier waits and the in-order fills
-  //    of one group (kASlots = t kIss + u kDq, t >= 1).
-  static_assert(kStages % kDq == 0 && kStages % kIss == 0, "stage ring");
-  static_assert(reachable(kASlots, kDq, kIss) && reachable(kASlots, kIss, kDq), "A-slot phases");
+  // waits below stay exact because each waiter saw the barrier's previous
+  // phase: every group waits on every phase of every weight stage; unit i
+  // belongs to group and issuer i mod kDq, its halves to A slots
+  // 2 (i mod kDq) and 2 (i mod kDq) + 1, and its activation stage
+  // i mod kXStages is used by that issuer only (kDq divides kXStages).
+  static_assert(kXStages % kDq == 0, "activation ring");
 };
 
 // Units [start(c), start(c + 1)) belong to CTA c.
@@ -121,14 +128,16 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
                const uint16_t* __restrict__ s_p, const uint8_t* __restrict__ z_p, uint16_t* __restrict__ Y,
                int M, int K, int N, uint32_t* __restrict__ ws_cnt, float* __restrict__ ws_part, OutMap om) {
   constexpr int BN = C::BN;
-  constexpr int S = C::kStages;
+  constexpr int SW = C::kWStages;
+  constexpr int SX = C::kXStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint64_t* wfull = bars;
-  uint64_t* xfull = wfull + S;
-  uint64_t* empty = xfull + S;
-  uint64_t* a_full = empty + S;
+  uint64_t* wempty = wfull + SW;
+  uint64_t* xfull = wempty + SW;
+  uint64_t* xempty = xfull + SX;
+  uint64_t* a_full = xempty + SX;
   uint64_t* a_empty = a_full + C::kASlots;
   uint64_t* acc_full = a_empty + C::kASlots;
   uint64_t* acc_empty = acc_full + C::kAccBufs;
@@ -150,10 +159,13 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
   const int nblk = (u1 - 1) / kg - b_first + 1;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < S; ++i) {
+    for (int i = 0; i < SW; ++i) {
       ptx::mbar_init(&wfull[i], 1);
+      ptx::mbar_init(&wempty[i], 4 * C::kDq);  // the 4 warps of every group
+    }
+    for (int i = 0; i < SX; ++i) {
       ptx::mbar_init(&xfull[i], 1);
-      ptx::mbar_init(&empty[i], 5);           // the 4 warps of one group + one issuer's commit
+      ptx::mbar_init(&xempty[i], 1);          // the unit's issuer, by commit
     }
     for (int i = 0; i < C::kASlots; ++i) {
       ptx::mbar_init(&a_full[i], 4);
@@ -178,45 +190,37 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
   ptx::griddep_launch_dependents();
   const uint32_t tmem = *tmem_ptr;
 
-  if (warp == C::kProducer) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      const uint8_t* wsrc = wq + (size_t)u0 * kUnitCodes;
-      const uint8_t* ssrc = reinterpret_cast<const uint8_t*>(s_p) + (size_t)u0 * kUnitS;
-      const uint8_t* zsrc = z_p + (size_t)u0 * kUnitZ;
-      auto issue_w = [&](int i) {
-        uint8_t* dst = smem + C::kWOff + (i % S) * kUnitW;
-        uint64_t* bar = &wfull[i % S];
-        ptx::mbar_arrive_expect_tx(bar, kUnitW);
-        ptx::bulk_load(dst, wsrc + (size_t)i * kUnitCodes, kUnitCodes, bar);
-        ptx::bulk_load(dst + kUnitCodes, ssrc + (size_t)i * kUnitS, kUnitS, bar);
-        ptx::bulk_load(dst + kUnitCodes + kUnitS, zsrc + (size_t)i * kUnitZ, kUnitZ, bar);
-      };
-      auto issue_x = [&](int i) {
-        uint64_t* bar = &xfull[i % S];
-        ptx::mbar_arrive_expect_tx(bar, C::kXBytes);
-        ptx::tma_load_3d(smem + C::kXOff + (i % S) * C::kXBytes, &tmap_x, bar, 0, 0, 2 * ((u0 + i) % kg));
-      };
-      // The weights do not depend on the kernels before this one in the
-      // stream: the first stages' weights are requested before the grid
-      // dependency wait, the activations only after it.
-      const int pre = L < S ? L : S;
-      for (int i = 0; i < pre; ++i) issue_w(i);
-      ptx::griddep_wait();
-      for (int i = 0; i < pre; ++i) issue_x(i);
-      int issued = pre;
-      for (int i = pre; i < L; ++i) {
-        if (!wait_bar(&empty[i % S], (uint32_t)(((i / S) & 1) ^ 1), abort_flag, &g_gvtc_status)) break;
-        issue_w(i);
-        issue_x(i);
-        issued = i + 1;
-      }
-      // Drain: every copy issued into this CTA's shared memory has landed.
-      for (int i = issued - S > 0 ? issued - S : 0; i < issued; ++i) {
-        wait_bar(&wfull[i % S], (uint32_t)((i / S) & 1), abort_flag, &g_gvtc_status, false);
-        wait_bar(&xfull[i % S], (uint32_t)((i / S) & 1), abort_flag, &g_gvtc_status, false);
-      }
+  if (warp == C::kWProducer) {
+    // ----------------------------------------------------- weight producer
+    // The weights do not depend on the kernels before this one in the
+    // stream, so this warp never waits for them.  Stage t holds units
+    // t kDq .. t kDq + kDq - 1 (fewer at the CTA's end): their codes,
+    // scales and zeros are each one contiguous range, copied by lanes 0, 1
+    // and 2 in the same instruction.
+    const int n_st = (L + C::kDq - 1) / C::kDq;
+    int issued = 0;
+    for (int t = 0; t < n_st; ++t) {
+      if (t >= SW && !wait_bar_warp(&wempty[t % SW], (uint32_t)(((t / SW) & 1) ^ 1), abort_flag, &g_gvtc_status))
+        break;
+      const int i = t * C::kDq;
+      const int nu = L - i < C::kDq ? L - i : C::kDq;
+      uint8_t* dst = smem + C::kWOff + (t % SW) * C::kStageBytes;
+      uint64_t* bar = &wfull[t % SW];
+      if (lane == 0) ptx::mbar_arrive_expect_tx(bar, (uint32_t)(nu * kUnitW));
+      __syncwarp();
+      if (lane == 0)
+        ptx::bulk_load(dst, wq + (size_t)(u0 + i) * kUnitCodes, (uint32_t)(nu * kUnitCodes), bar);
+      else if (lane == 1)
+        ptx::bulk_load(dst + C::kDq * kUnitCodes, reinterpret_cast<const uint8_t*>(s_p) + (size_t)(u0 + i) * kUnitS,
+                       (uint32_t)(nu * kUnitS), bar);
+      else if (lane == 2)
+        ptx::bulk_load(dst + C::kDq * (kUnitCodes + kUnitS), z_p + (size_t)(u0 + i) * kUnitZ,
+                       (uint32_t)(nu * kUnitZ), bar);
+      issued = t + 1;
     }
+    // Drain: every copy issued into this CTA's shared memory has landed.
+    for (int t = issued - SW > 0 ? issued - SW : 0; t < issued; ++t)
+      wait_bar(&wfull[t % SW], (uint32_t)((t / SW) & 1), abort_flag, &g_gvtc_status, false);
   } else if (warp >= C::kFirstIss && warp < C::kFirstIss + C::kIss) {
     // --------------------------------------------------------- MMA issuers
     // Issuer ii takes the CTA's units i = ii, ii + kIss, ...; per block it
@@ -226,39 +230,89 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
     const int ii = warp - C::kFirstIss;
     if (lane == 0) {
       const uint64_t desc0 = ptx::smem_desc_sw128(ptx::smem_addr(smem + C::kXOff));
+      // This issuer's units i = ii + k kIss, k < n_my; unit i's activation
+      // tile lives in X stage i mod kXStages, a stage only this issuer uses.
+      const int n_my = ii < L ? (L - ii + C::kIss - 1) / C::kIss : 0;
+      auto issue_x = [&](int i) {
+        uint64_t* bar = &xfull[i % SX];
+        ptx::mbar_arrive_expect_tx(bar, C::kXBytes);
+        ptx::tma_load_3d(smem + C::kXOff + (i % SX) * C::kXBytes, &tmap_x, bar, 0, 0, 2 * ((u0 + i) % kg));
+      };
+      // X may be written by the kernel before this one: only after the grid
+      // dependency wait.
+      ptx::griddep_wait();
+      int x_issued = 0;
+      for (; x_issued < C::kXAhead && x_issued < n_my; ++x_issued) issue_x(ii + x_issued * C::kIss);
       bool ok = true;
-      for (int bi = 0; ok && bi < nblk; ++bi) {
-        const int b = b_first + bi;
-        const int i0 = (b * kg > u0 ? b * kg : u0) - u0;
-        const int i1 = ((b + 1) * kg < u1 ? (b + 1) * kg : u1) - u0;
-        const int buf = bi % C::kAccBufs;
-        if (!wait_bar(&acc_empty[buf], (uint32_t)(((bi / C::kAccBufs) & 1) ^ 1), abort_flag, &g_gvtc_status))
-          break;
+      int cur = -1;              // block being accumulated (CTA-local index)
+      bool first = true;         // no MMA of this issuer in block `cur` yet
+      // Close block `cur` (arrive on its "full" barrier: commit if this issuer
+      // issued MMAs there) and open the next one once the epilogue has freed
+      // its accumulator set.
+      auto next_block = [&]() -> bool {
+        if (cur >= 0) {
+          uint64_t* f = &acc_full[cur % C::kAccBufs];
+          if (first) ptx::mbar_arrive(f);
+          else ptx::mma_commit(f);
+        }
+        ++cur;
+        first = true;
+        if (!wait_bar(&acc_empty[cur % C::kAccBufs], (uint32_t)(((cur / C::kAccBufs) & 1) ^ 1), abort_flag,
+                      &g_gvtc_status))
+          return false;
         ptx::tc_fence_after();
-        const uint32_t d_tmem = tmem + buf * C::kAccCols + ii * BN;
-        bool first = true;
-        for (int i = i0 + ((ii - i0 % C::kIss) + C::kIss) % C::kIss; i < i1; i += C::kIss) {
-          const int st = i % S;
-          const int a = i % C::kASlots;
-          if (!wait_bar(&xfull[st], (uint32_t)((i / S) & 1), abort_flag, &g_gvtc_status) ||
-              !wait_bar(&a_full[a], (uint32_t)((i / C::kASlots) & 1), abort_flag, &g_gvtc_status)) {
+        return true;
+      };
+      for (int k = 0; ok && k < n_my; ++k) {
+        const int i = ii + k * C::kIss;
+        const int bl = (u0 + i) / kg - b_first;
+        while (ok && cur < bl) ok = next_block();
+        if (!ok) break;
+        // Refill the stage of this issuer's previous unit once its MMAs are done.
+        if (k >= 1 && x_issued < n_my) {
+          const int ip = i - C::kIss;
+          if (!wait_bar(&xempty[ip % SX], (uint32_t)((ip / SX) & 1), abort_flag, &g_gvtc_status)) break;
+          issue_x(ii + x_issued * C::kIss);
+          ++x_issued;
+        }
+        const int st = i % SX;
+        if (!wait_bar(&xfull[st], (uint32_t)((i / SX) & 1), abort_flag, &g_gvtc_status)) break;
+        const uint32_t d_tmem = tmem + (cur % C::kAccBufs) * C::kAccCols + ii * BN;
+        // The unit's two halves: four K = 16 MMAs each, over the matching
+        // 64-k slab of the activation tile.
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int j = 2 * i + hf;
+          const int a = j % C::kASlots;
+          if (!wait_bar(&a_full[a], (uint32_t)((j / C::kASlots) & 1), abort_flag, &g_gvtc_status)) {
             ok = false;
             break;
           }
           ptx::tc_fence_after();
-          const uint64_t desc = desc0 + (uint64_t)((st * C::kXBytes) >> 4);
-          ptx::mma_ts_f16_slot<8>(d_tmem, tmem + C::kACol0 + a * kACols, desc, C::kIdesc, first ? 0u : 1u,
-                                  &a_empty[a], (BN * 128) >> 4);
-          ptx::mma_commit(&empty[st]);
-          first = false;
+          const uint64_t desc = desc0 + (uint64_t)((st * C::kXBytes + hf * C::kSlab) >> 4);
+          ptx::mma_ts_f16_slot<4>(d_tmem, tmem + C::kACol0 + a * kACols, desc, C::kIdesc,
+                                  (first && hf == 0) ? 0u : 1u, &a_empty[a], 0u);
         }
         if (!ok) break;
-        if (first) ptx::mbar_arrive(&acc_full[buf]);
-        else ptx::mma_commit(&acc_full[buf]);
+        ptx::mma_commit(&xempty[st]);
+        first = false;
       }
-      // Drain: all MMAs issued by this thread have completed.
+      // Every block of the CTA gets this issuer's arrival, units or not.
+      while (ok && cur < nblk - 1) ok = next_block();
+      if (ok && cur >= 0) {
+        uint64_t* f = &acc_full[cur % C::kAccBufs];
+        if (first) ptx::mbar_arrive(f);
+        else ptx::mma_commit(f);
+      }
+      // Drain: all MMAs issued by this thread have completed, and every
+      // activation copy it issued has landed.
       ptx::mma_commit(drain);
       wait_bar(drain, 0, abort_flag, &g_gvtc_status, false);
+      for (int k = 0; k < x_issued; ++k) {
+        const int i = ii + k * C::kIss;
+        if (k + C::kXAhead >= x_issued)
+          wait_bar(&xfull[i % SX], (uint32_t)((i / SX) & 1), abort_flag, &g_gvtc_status, false);
+      }
     }
   } else if (warp >= C::kFirstDq) {
     // -------------------------------------------------------- dequantisers
@@ -269,47 +323,51 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
     const uint32_t a_lane = tmem + ((uint32_t)(quad * 32) << 16) + C::kACol0;
     const uint32_t wring = ptx::smem_addr(smem + C::kWOff);
     for (int i = gi; i < L; i += C::kDq) {
-      const int st = i % S;
-      if (!wait_bar_warp(&wfull[st], (uint32_t)((i / S) & 1), abort_flag, &g_gvtc_status)) break;
-      const uint32_t base = wring + st * kUnitW;
+      // Unit i is unit gi of weight stage t = i / kDq.
+      const int t = i / C::kDq;
+      const int st = t % SW;
+      if (!wait_bar_warp(&wfull[st], (uint32_t)((t / SW) & 1), abort_flag, &g_gvtc_status)) break;
+      const uint32_t sbase = wring + st * C::kStageBytes;
+      const uint32_t base = sbase + gi * kUnitCodes;
       const uint4 v0 = ptx::lds_v4(base + 0 * 2048 + row * 16);
       const uint4 v1 = ptx::lds_v4(base + 1 * 2048 + row * 16);
       const uint4 v2 = ptx::lds_v4(base + 2 * 2048 + row * 16);
       const uint4 v3 = ptx::lds_v4(base + 3 * 2048 + row * 16);
-      const uint32_t sv = ptx::lds_u16(base + kUnitCodes + row * 2);
-      const uint32_t zb = ptx::lds_u8(base + kUnitCodes + kUnitS + (row >> 1));
+      const uint32_t sv = ptx::lds_u16(sbase + C::kDq * kUnitCodes + gi * kUnitS + row * 2);
+      const uint32_t zb = ptx::lds_u8(sbase + C::kDq * (kUnitCodes + kUnitS) + gi * kUnitZ + (row >> 1));
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&empty[st]);
+      if (lane == 0) ptx::mbar_arrive(&wempty[st]);
       const GroupConsts gc = make_group_consts((zb >> ((row & 1) * 4)) & 0xFu, (uint16_t)sv);
-      const int a = i % C::kASlots;
-      const uint32_t dst = a_lane + a * kACols;
-      uint32_t h[16];
-      dequant_word(v0.x, gc, &h[0]);
-      dequant_word(v0.y, gc, &h[4]);
-      dequant_word(v0.z, gc, &h[8]);
-      dequant_word(v0.w, gc, &h[12]);
-      if (!wait_bar_warp(&a_empty[a], (uint32_t)(((i / C::kASlots) & 1) ^ 1), abort_flag, &g_gvtc_status)) break;
-      ptx::tc_fence_after();
-      ptx::tmem_st_x16(dst, h);
-      dequant_word(v1.x, gc, &h[0]);
-      dequant_word(v1.y, gc, &h[4]);
-      dequant_word(v1.z, gc, &h[8]);
-      dequant_word(v1.w, gc, &h[12]);
-      ptx::tmem_st_x16(dst + 16, h);
-      dequant_word(v2.x, gc, &h[0]);
-      dequant_word(v2.y, gc, &h[4]);
-      dequant_word(v2.z, gc, &h[8]);
-      dequant_word(v2.w, gc, &h[12]);
-      ptx::tmem_st_x16(dst + 32, h);
-      dequant_word(v3.x, gc, &h[0]);
-      dequant_word(v3.y, gc, &h[4]);
-      dequant_word(v3.z, gc, &h[8]);
-      dequant_word(v3.w, gc, &h[12]);
-      ptx::tmem_st_x16(dst + 48, h);
-      ptx::tmem_wait_st();
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&a_full[a]);
+      bool ok = true;
+      // Two halves of 64 k, each into its own A slot: chunks (v0, v1), then (v2, v3).
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const int j = 2 * i + hf;
+        const int a = j % C::kASlots;
+        const uint32_t dst = a_lane + a * kACols;
+        const uint4 c0 = hf ? v2 : v0, c1 = hf ? v3 : v1;
+        uint32_t h[16];
+        dequant_word(c0.x, gc, &h[0]);
+        dequant_word(c0.y, gc, &h[4]);
+        dequant_word(c0.z, gc, &h[8]);
+        dequant_word(c0.w, gc, &h[12]);
+        if (!wait_bar_warp(&a_empty[a], (uint32_t)(((j / C::kASlots) & 1) ^ 1), abort_flag, &g_gvtc_status)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        ptx::tmem_st_x16(dst, h);
+        dequant_word(c1.x, gc, &h[0]);
+        dequant_word(c1.y, gc, &h[4]);
+        dequant_word(c1.z, gc, &h[8]);
+        dequant_word(c1.w, gc, &h[12]);
+        ptx::tmem_st_x16(dst + 16, h);
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&a_full[a]);
+      }
+      if (!ok) break;
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------ epilogue
@@ -383,7 +441,7 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
       if (!whole) {
         // The last of the block's CTAs (per lane quarter) adds every CTA's
         // partial in CTA order and writes the row.
-        __threadfence();
+        ptx::fence_acq_rel_gpu();
         __syncwarp();
         uint32_t old = 0;
         if (lane == 0) old = ptx::atom_add_acq_rel_gpu(&ws_cnt[b * 4 + quad], 1u);
@@ -391,7 +449,7 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
         const int cf = cta_of(U, G, (long long)b * kg);
         const int cl = cta_of(U, G, (long long)(b + 1) * kg - 1);
         if (old == (uint32_t)(cl - cf)) {
-          __threadfence();
+          ptx::fence_acq_rel_gpu();
 #pragma unroll 1
           for (int h = 0; h < chunks; ++h) {
             float v[8];
@@ -420,15 +478,18 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
   }
 }
 
-// Up to 16 tokens: three dequantiser groups, three issuers, one accumulator
-// set, six stages of 12.3 KB.
-using Cfg16 = GtCfg<16, 3, 3, 3, 1, 6>;
-// Up to 32 tokens: two groups, two issuers, two accumulator sets, six
-// stages of 16.3 KB.
-using Cfg32 = GtCfg<32, 2, 2, 2, 2, 6>;
-// Up to 64 tokens: two groups, two issuers, one accumulator set, four
-// stages of 24.3 KB.
-using Cfg64 = GtCfg<64, 2, 2, 2, 1, 4>;
+// Up to 8 tokens: three dequantiser groups (and issuers), one accumulator
+// set, three weight stages of three units (24.9 KB) and nine activation
+// stages of 8 token rows (2 KB), three per issuer.
+using Cfg8 = GtCfg<16, 8, 3, 1, 3, 9>;
+// Up to 16 tokens: as above with 16-row activation tiles (4 KB), two per issuer.
+using Cfg16 = GtCfg<16, 16, 3, 1, 3, 6>;
+// Up to 32 tokens: two groups, two accumulator sets, four weight stages of
+// two units (16.6 KB) and four activation stages (8 KB).
+using Cfg32 = GtCfg<32, 32, 2, 2, 4, 4>;
+// Up to 64 tokens: two groups, one accumulator set, two weight stages of
+// two units and four activation stages (16 KB).
+using Cfg64 = GtCfg<64, 64, 2, 1, 2, 4>;
 
 int grid_for(int M, int K) {
   const long long U = (long long)ceil_div(M, kRowBlock) * (K / kGroup);
@@ -445,7 +506,7 @@ cudaError_t launch_cfg(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_
                                     smem_set);
   if (e != cudaSuccess) return e;
   CUtensorMap map;
-  e = make_x_map(&map, X, N, K, C::BN, 2);
+  e = make_x_map(&map, X, N, K, C::kXRows, 2);
   if (e != cudaSuccess) return e;
   uint32_t* cnt = static_cast<uint32_t*>(ws);
   float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + gemv_tc_counter_bytes(M));
@@ -487,6 +548,7 @@ cudaError_t launch_gemv_tc(const uint8_t* wq, const uint16_t* scales, const uint
                                                          pdl, stream, o);                             \
     return launch_cfg<CFG, kEpiPlain>(wq, scales, zeros, X, y, M, K, N, workspace, pdl, stream, o);   \
   } while (0)
+  if (N <= 8) W4A16_GVTC(Cfg8);
   if (N <= 16) W4A16_GVTC(Cfg16);
   if (N <= 32) W4A16_GVTC(Cfg32);
   W4A16_GVTC(Cfg64);
