@@ -65,7 +65,7 @@ w4a16_status map_cuda(cudaError_t e) {
 // with_ws: a workspace is available, which opens the split decode kernel.
 int select_path_impl(int M, int K, int N, bool with_ws) {
   if (M <= 0 || K <= 0 || N <= 0 || K % kGroup) return -1;
-  if (with_ws && N <= kGemvTcAutoTokens) return W4A16_PATH_GEMV_TC;
+  (void)with_ws;   // the split decode path is never the faster one (forced only)
   return N <= gemv_max_n() ? W4A16_PATH_GEMV : W4A16_PATH_TC;
 }
 
@@ -97,8 +97,8 @@ w4a16_status gemm_impl(const void* wq_packed, const void* scales_packed, const v
     const size_t ny = (size_t)N * M * 2, nx = (size_t)N * K * 2;
     if (overlap(Y, ny, X, nx) || overlaps_weight(Y, ny, wq_packed, scales_packed, zeros_packed, pb))
       return W4A16_ERR_INVALID_ARG;
-    if (need && (overlap(ws, need, X, nx) || overlap(ws, need, Y, ny) ||
-                 overlaps_weight(ws, need, wq_packed, scales_packed, zeros_packed, pb)))
+    if (ws && (overlap(ws, ws_bytes, X, nx) || overlap(ws, ws_bytes, Y, ny) ||
+               overlaps_weight(ws, ws_bytes, wq_packed, scales_packed, zeros_packed, pb)))
       return W4A16_ERR_INVALID_ARG;
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -111,7 +111,7 @@ w4a16_status gemm_impl(const void* wq_packed, const void* scales_packed, const v
   else if (path == W4A16_PATH_TC)
     e = launch_gemm_tc(wq, sp, zp, X, Y, M, K, N, s);
   else
-    e = launch_gemv(wq, sp, zp, X, Y, M, K, N, s);
+    e = launch_gemv(wq, sp, zp, X, Y, M, K, N, s, nullptr, (flags & W4A16_FLAG_EARLY_WEIGHTS) != 0);
   return map_cuda(e);
 }
 
@@ -137,8 +137,8 @@ w4a16_status gemm_qkv_impl(const void* wq_packed, const void* scales_packed, con
   if (need > ws_bytes) return W4A16_ERR_INVALID_ARG;
   {
     const PackedBytes pb = packed_bytes(M, K);
-    const void* outs[4] = {Yq, Yk, Yv, need ? ws : nullptr};
-    const size_t out_n[4] = {(size_t)N * Mq * 2, (size_t)N * Mk * 2, (size_t)N * Mv * 2, need};
+    const void* outs[4] = {Yq, Yk, Yv, ws};
+    const size_t out_n[4] = {(size_t)N * Mq * 2, (size_t)N * Mk * 2, (size_t)N * Mv * 2, ws ? ws_bytes : 0};
     for (int i = 0; i < 4; ++i) {
       if (overlap(outs[i], out_n[i], X, (size_t)N * K * 2) || overlap(outs[i], out_n[i], bias, (size_t)M * 2) ||
           overlaps_weight(outs[i], out_n[i], wq_packed, scales_packed, zeros_packed, pb))
@@ -165,7 +165,7 @@ w4a16_status gemm_qkv_impl(const void* wq_packed, const void* scales_packed, con
   else if (path == W4A16_PATH_TC)
     e = launch_gemm_tc(wq, sp, zp, X, nullptr, M, K, N, s, &om);
   else
-    e = launch_gemv(wq, sp, zp, X, nullptr, M, K, N, s, &om);
+    e = launch_gemv(wq, sp, zp, X, nullptr, M, K, N, s, &om, (flags & W4A16_FLAG_EARLY_WEIGHTS) != 0);
   return map_cuda(e);
 }
 
@@ -286,8 +286,8 @@ w4a16_status gemm_gate_up_impl(const void* wq_packed, const void* scales_packed,
     const size_t nh = (size_t)N * Mi * 2, nx = (size_t)N * K * 2;
     if (overlap(H, nh, X, nx) || overlaps_weight(H, nh, wq_packed, scales_packed, zeros_packed, pb))
       return W4A16_ERR_INVALID_ARG;
-    if (need && (overlap(ws, need, X, nx) || overlap(ws, need, H, nh) ||
-                 overlaps_weight(ws, need, wq_packed, scales_packed, zeros_packed, pb)))
+    if (ws && (overlap(ws, ws_bytes, X, nx) || overlap(ws, ws_bytes, H, nh) ||
+               overlaps_weight(ws, ws_bytes, wq_packed, scales_packed, zeros_packed, pb)))
       return W4A16_ERR_INVALID_ARG;
   }
   OutMap om = {};
@@ -304,7 +304,7 @@ w4a16_status gemm_gate_up_impl(const void* wq_packed, const void* scales_packed,
   else if (path == W4A16_PATH_TC)
     e = launch_gemm_tc(wq, sp, zp, X, nullptr, M, K, N, s, &om);
   else
-    e = launch_gemv(wq, sp, zp, X, nullptr, M, K, N, s, &om);
+    e = launch_gemv(wq, sp, zp, X, nullptr, M, K, N, s, &om, (flags & W4A16_FLAG_EARLY_WEIGHTS) != 0);
   return map_cuda(e);
 }
 

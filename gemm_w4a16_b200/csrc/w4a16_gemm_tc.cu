@@ -570,9 +570,9 @@ __global__ void wait_timeout_selftest_kernel(long long limit) {
 
 }  // namespace
 
-// The CUDA-core GEMV runs up to this many tokens (measured N sweep, fused QKV
-// shape); the tensor-core kernel from there on.
-int gemv_max_n() { return 2; }
+// The decode kernel runs up to this many tokens (one launch; measured N sweep,
+// fused QKV shape); the tensor-core tile kernel from there on.
+int gemv_max_n() { return kGemvMaxTokens; }
 
 template <int kEpi>
 cudaError_t launch_tc_map(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros, const uint16_t* X,

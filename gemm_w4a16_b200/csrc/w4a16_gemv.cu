@@ -1,26 +1,32 @@
-// Decode GEMV / tiny-N kernel on CUDA cores (memory-bound regime).
+// Decode GEMV / few-token kernel (memory-bound regime).
 //
 // "PerfXLLM on Snapdragon 8 Gen2", section 3.3 item 2: the GEMV is memory
 // bound; its design goals there are vectorised loads, unrolling to keep many
-// loads in flight, the zero and scale of each int4 group kept in shared
-// memory, the vector read through a texture-like path, and tiling both
-// dimensions of the weight (rows and K) for parallelism.  On sm_100a:
+// loads in flight, the zero and scale of each int4 group at hand, the vector
+// read through a fast on-chip path, and tiling both dimensions of the weight
+// (rows and K) for parallelism.  On sm_100a:
 //
 //  * a CTA owns one 128-row block of the packed weight and a range of whole
-//    groups along K; a producer warp streams each group (8 KB of codes, 256 B
-//    of scales, 64 B of zeros, contiguous in the packed layout) into a
-//    6-stage shared-memory ring with bulk asynchronous copies, so tens of KB
-//    per CTA are in flight without holding registers;
-//  * the CTA's slice of the activations is staged once in shared memory and
-//    read back as broadcast 16-byte loads;
-//  * two consumer warpgroups take alternate groups; thread = one weight row;
-//    the exact in-register dequant (dequant_word) feeds fma.rn.f32.f16 into
-//    four independent fp32 chains per token;
-//  * split-K: the two warpgroups reduce through shared memory, and CTAs of a
-//    thread-block cluster (up to 8 along K) through distributed shared memory
-//    into the cluster's rank-0 CTA, in a fixed order (deterministic, no
-//    atomics);
-//  * every mbarrier wait is bounded (device status word on expiry).
+//    groups along K; each of its 8 warps owns one 16-row tile of that block
+//    and streams the tile's codes, scales and zeros straight from HBM into
+//    registers with 16-byte non-allocating loads, kGvDepth groups ahead of
+//    the one it computes (no shared-memory staging, no barriers);
+//  * the first groups are requested before the grid dependency wait, so with
+//    programmatic dependent launch the weight stream starts while the
+//    previous kernel finishes; the activations (written by that kernel) are
+//    staged in shared memory after the wait;
+//  * the products run on the tensor cores as warp-level mma.sync m16n8k16
+//    (f16 inputs, fp32 accumulation): lane l = 4 g + c holds rows g and g + 8
+//    of the tile and chunk c (32 codes) of each; the exact dequant of one
+//    32-bit word (8 codes) of each row gives the lane's A fragments of two
+//    MMAs, whose B fragments are token g's activations at the same eight k
+//    (one 16-byte shared load).  The MMA's k order is thus a permutation of
+//    the group that A and B share; tokens g >= NT are zero columns.  One MMA
+//    instruction replaces 256 fp32 FMAs, so the kernel issues about 2.3
+//    instructions per weight (1.6 of them the exact dequant);
+//  * split-K: CTAs of a thread-block cluster (up to 8 along K) reduce through
+//    distributed shared memory into the cluster's rank-0 CTA in a fixed order
+//    (deterministic, no atomics).
 #include "w4a16_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -28,46 +34,158 @@
 
 namespace w4a16 {
 
+// Status word of the decode kernel's family.  The kernel has no waits, so it
+// stays 0; it is kept so every kernel family reports through the same call.
 __device__ int g_gemv_status = 0;
 
 namespace {
 
-constexpr int kGvHalves = 2;                          // consumer warpgroups (alternate groups)
-constexpr int kGvConsumerWarps = 4 * kGvHalves;
-constexpr int kGvProducerWarp = kGvConsumerWarps;
-constexpr int kGvThreads = (kGvConsumerWarps + 1) * 32;
+constexpr int kGvWarps = 8;                           // one 16-row MMA tile each
+constexpr int kGvThreads = kGvWarps * 32;
+constexpr int kGvDepth = 3;                           // groups of codes in flight per warp
+constexpr int kGvCtasPerSm = 3;                       // resident CTAs per SM (register budget)
 constexpr int kGvWBytes = 4 * kRowBlock * 16;         // one group of 128 rows: 8 KB
-constexpr int kGvStageBytes = kGvWBytes + kRowBlock * 2 + kRowBlock / 2;   // + scales + zeros
-constexpr int kGvStages = 6;                          // multiple of kGvHalves
 constexpr int kMaxCluster = 8;
 constexpr int kMaxXSmem = 64 * 1024;                  // largest staged activation slice
-static_assert(kGvStages % kGvHalves == 0, "stage ring");
 
-__device__ __forceinline__ void fma_h2(float& acc, uint32_t w, uint32_t x) {
-  asm("{\n\t.reg .f16 wl, wh, xl, xh;\n\t"
-      "mov.b32 {wl, wh}, %1;\n\t"
-      "mov.b32 {xl, xh}, %2;\n\t"
-      "fma.rn.f32.f16 %0, wl, xl, %0;\n\t"
-      "fma.rn.f32.f16 %0, wh, xh, %0;\n\t}"
-      : "+f"(acc) : "r"(w), "r"(x));
+// D += A B for one m16n8k16 tile: A 16 x 16 f16 (row), B 16 x 8 f16 (col),
+// fp32 accumulators, in the warp-level fragment layout of mma.sync.
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+               "{%0,%1,%2,%3};"
+               : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+               : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Non-allocating loads at p + OFF bytes (OFF folded into the instruction).
+template <int OFF>
+__device__ __forceinline__ uint4 ldg_v4_at(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4+%5];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p), "n"(OFF));
+  return r;
+}
+
+template <int OFF>
+__device__ __forceinline__ uint32_t ldg_u16_at(const void* p) {
+  unsigned short v;
+  asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1+%2];" : "=h"(v) : "l"(p), "n"(OFF));
+  return v;
+}
+
+template <int OFF>
+__device__ __forceinline__ uint32_t ldg_u8_at(const void* p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.u8 %0, [%1+%2];" : "=r"(v) : "l"(p), "n"(OFF));
+  return v;
+}
+
+// Halves between consecutive tokens of the staged activation slice: the
+// slice of one token plus 16 halves, so the 16-byte loads of the two tokens
+// in one quarter-warp fall on different banks.
+__host__ __device__ inline int gv_xstride(int ng) { return ng * kGroup + 16; }
+
 struct GvLayout {
-  int x_off, red_off, cred_off, bar_off, total;
+  int x_off, red_off, cred_off, total;
 };
 
 __host__ __device__ inline GvLayout gv_layout(int nt, int gspan, int cl) {
   GvLayout L;
-  L.x_off = kGvStages * kGvStageBytes;
-  L.red_off = L.x_off + nt * gspan * kGroup * 2;
-  L.cred_off = L.red_off + kGvHalves * nt * kRowBlock * 4;
-  L.bar_off = L.cred_off + (cl > 1 ? cl * nt * kRowBlock * 4 : 0);
-  L.total = L.bar_off + 8 * (2 * kGvStages + 1) + 16;
+  L.x_off = 0;
+  L.red_off = L.x_off + nt * gv_xstride(gspan) * 2;
+  L.cred_off = L.red_off + nt * kRowBlock * 4;
+  L.total = L.cred_off + (cl > 1 ? cl * nt * kRowBlock * 4 : 0);
   return L;
 }
 
+// One group's operands of one lane: chunk c of rows r (lo) and r + 8 (hi),
+// their scales and the bytes holding their zero codes.
+struct GvFrag {
+  uint4 lo, hi;
+  uint32_t s_lo, s_hi, z_lo, z_hi;
+};
+
+// Group J of the lane's streams: pw points at chunk c of row r of group 0,
+// ps at the scale of row r, pz at the zero byte of row r (row r + 8: 128,
+// 8 and 4 bytes further).
+template <int J>
+__device__ __forceinline__ void gv_load(GvFrag& f, const uint8_t* pw, const uint16_t* ps, const uint8_t* pz) {
+  f.lo = ldg_v4_at<J * kGvWBytes>(pw);
+  f.hi = ldg_v4_at<J * kGvWBytes + 8 * 16>(pw);
+  f.s_lo = ldg_u16_at<J * kRowBlock * 2>(ps);
+  f.s_hi = ldg_u16_at<J * kRowBlock * 2 + 16>(ps);
+  f.z_lo = ldg_u8_at<J * (kRowBlock / 2)>(pz);
+  f.z_hi = ldg_u8_at<J * (kRowBlock / 2) + 4>(pz);
+}
+
+template <uint32_t SEL>
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "n"(SEL));
+  return d;
+}
+
+// The dequant constants (as make_group_consts) of the lane's two rows at
+// once: the two zero codes side by side in one register (row lo in the low
+// half), both fp16 forms built there, then each half copied to both halves.
+// zsh = 4 for odd rows (their code sits in bits 4..7 of the zero byte).
+__device__ __forceinline__ void gv_consts(const GvFrag& f, int zsh, GroupConsts& lo, GroupConsts& hi) {
+  const uint32_t zz = prmt<0x5410>(f.z_lo, f.z_hi);                       // bytes: z_lo, 0, z_hi, 0
+  const uint32_t a = lop3_and_or(zz >> zsh, 0x000F000Fu, 0x64006400u);     // 1024 + z per half
+  const uint32_t b = lop3_and_or(zz << (4 - zsh), 0x00F000F0u, 0xD400D400u);  // -(64 + z) per half
+  lo.z1024 = prmt<0x1010>(a, a);
+  hi.z1024 = prmt<0x3232>(a, a);
+  lo.zneg64 = prmt<0x1010>(b, b);
+  hi.zneg64 = prmt<0x3232>(b, b);
+  lo.s2 = prmt<0x1010>(f.s_lo, f.s_lo);
+  hi.s2 = prmt<0x1010>(f.s_hi, f.s_hi);
+}
+
+// Dequantise one group of the lane's two rows and accumulate its eight MMAs;
+// xg points at token g's activations at k = 32 c of the group.
+__device__ __forceinline__ void gv_consume(const GvFrag& f, int zsh, const uint16_t* xg, float (&acc)[4]) {
+  GroupConsts clo, chi;
+  gv_consts(f, zsh, clo, chi);
+  const uint32_t wl[4] = {f.lo.x, f.lo.y, f.lo.z, f.lo.w};
+  const uint32_t wh[4] = {f.hi.x, f.hi.y, f.hi.z, f.hi.w};
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const uint4 xb = *reinterpret_cast<const uint4*>(xg + 8 * t);
+    uint32_t al[4], ah[4];
+    dequant_word(wl[t], clo, al);
+    dequant_word(wh[t], chi, ah);
+    mma_16816(acc, al[0], ah[0], al[1], ah[1], xb.x, xb.y);
+    mma_16816(acc, al[2], ah[2], al[3], ah[3], xb.z, xb.w);
+  }
+}
+
+template <int U>
+__device__ __forceinline__ void gv_load_first(GvFrag (&f)[kGvDepth], int ng, const uint8_t* pw, const uint16_t* ps,
+                                              const uint8_t* pz) {
+  if constexpr (U < kGvDepth) {
+    if (U < ng) gv_load<U>(f[U], pw, ps, pz);
+    gv_load_first<U + 1>(f, ng, pw, ps, pz);
+  }
+}
+
+// Slots U.. of one step of kGvDepth groups starting at group i0: consume
+// group i0 + U from slot U, refill the slot with group i0 + U + kGvDepth.
+template <int U>
+__device__ __forceinline__ void gv_step(GvFrag (&f)[kGvDepth], int i0, int ng, const uint8_t* pw,
+                                        const uint16_t* ps, const uint8_t* pz, int zsh, const uint16_t* xg,
+                                        float (&acc)[4]) {
+  if constexpr (U < kGvDepth) {
+    if (i0 + U < ng) {
+      gv_consume(f[U], zsh, xg + U * kGroup, acc);
+      if (i0 + U + kGvDepth < ng) gv_load<U + kGvDepth>(f[U], pw, ps, pz);
+      gv_step<U + 1>(f, i0, ng, pw, ps, pz, zsh, xg, acc);
+    }
+  }
+}
+
 template <int NT, int kEpi>
-__global__ void __launch_bounds__(kGvThreads)
+__global__ void __launch_bounds__(kGvThreads, kGvCtasPerSm)
 gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
             const uint8_t* __restrict__ z_p, const uint16_t* __restrict__ X,
             uint16_t* __restrict__ Y, int M, int K, int cl, OutMap om) {
@@ -76,115 +194,72 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   const int kc_n = K / kChunkK;
   const int gspan = ceil_div(kg, cl);
   const GvLayout L = gv_layout(NT, gspan, cl);
-  uint4* xs = reinterpret_cast<uint4*>(smem + L.x_off);
-  float* red = reinterpret_cast<float*>(smem + L.red_off);     // [halves][NT][128]
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem + L.x_off);  // [NT][xstride]
+  float* red = reinterpret_cast<float*>(smem + L.red_off);     // [NT][128]
   float* cred = reinterpret_cast<float*>(smem + L.cred_off);   // [cl][NT][128], rank 0 only
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off);
-  uint64_t* empty = full + kGvStages;
-  uint64_t* xbar = empty + kGvStages;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(xbar + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
   const int b = blockIdx.x / cl;
   const int crank = blockIdx.x % cl;
   const int ga = (kg * crank) / cl, gb = (kg * (crank + 1)) / cl;
   const int ng = gb - ga;
+  const int xstride = gv_xstride(ng);
 
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kGvStages; ++i) {
-      ptx::mbar_init(&full[i], 1);
-      ptx::mbar_init(&empty[i], 4);              // the 4 warps of one consumer half
-    }
-    ptx::mbar_init(xbar, 1);
-    *abort_flag = 0;
-    ptx::fence_mbar_init();
-  }
-  __syncthreads();
+  ptx::griddep_launch_dependents();
   if (cl > 1) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 
-  float tot[NT];
-  if (warp == kGvProducerWarp) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0 && ng > 0) {
-      ptx::mbar_arrive_expect_tx(xbar, (uint32_t)(NT * ng * kGroup * 2));
-      for (int n = 0; n < NT; ++n)
-        ptx::bulk_load(reinterpret_cast<uint8_t*>(xs) + n * ng * kGroup * 2,
-                       X + (size_t)n * K + (size_t)ga * kGroup, (uint32_t)(ng * kGroup * 2), xbar);
-      const uint8_t* wblk = wq + (size_t)b * kc_n * kRowBlock * 16;
-      const uint16_t* sblk = s_p + (size_t)b * kg * kRowBlock;
-      const uint8_t* zblk = z_p + (size_t)b * kg * (kRowBlock / 2);
-      int last = -1;
-      for (int i = 0; i < ng; ++i) {
-        const int st = i % kGvStages;
-        const uint32_t ph = (uint32_t)((i / kGvStages) & 1);
-        if (!wait_bar(&empty[st], ph ^ 1, abort_flag, &g_gemv_status)) break;
-        uint8_t* dst = smem + st * kGvStageBytes;
-        const int g = ga + i;
-        ptx::mbar_arrive_expect_tx(&full[st], kGvStageBytes);
-        ptx::bulk_load(dst, wblk + (size_t)g * kGvWBytes, kGvWBytes, &full[st]);
-        ptx::bulk_load(dst + kGvWBytes, sblk + (size_t)g * kRowBlock, kRowBlock * 2, &full[st]);
-        ptx::bulk_load(dst + kGvWBytes + kRowBlock * 2, zblk + (size_t)g * (kRowBlock / 2), kRowBlock / 2,
-                       &full[st]);
-        last = i;
-      }
-      // Drain: every copy issued into this CTA's shared memory has landed.
-      for (int i = (last - kGvStages + 1 > 0 ? last - kGvStages + 1 : 0); i <= last; ++i)
-        wait_bar(&full[i % kGvStages], (uint32_t)((i / kGvStages) & 1), abort_flag, &g_gemv_status, false);
-      wait_bar(xbar, 0, abort_flag, &g_gemv_status, false);
+  // This lane's rows within the block, and its group streams (pointers at
+  // group ga; slot offsets are folded into the loads).
+  const int rl = 16 * warp + g;
+  const int zsh = (g & 1) * 4;          // rows rl and rl + 8 have the same parity
+  const uint8_t* pw = wq + (size_t)b * kc_n * kRowBlock * 16 + (size_t)ga * kGvWBytes + c * (kRowBlock * 16) + rl * 16;
+  const uint16_t* ps = s_p + ((size_t)b * kg + ga) * kRowBlock + rl;
+  const uint8_t* pz = z_p + ((size_t)b * kg + ga) * (kRowBlock / 2) + (rl >> 1);
+
+  // The first groups depend on no earlier kernel: request them before the
+  // grid dependency wait (which returns at once unless the launch is
+  // programmatic).
+  GvFrag f[kGvDepth];
+  gv_load_first<0>(f, ng, pw, ps, pz);
+  ptx::griddep_wait();
+
+  // Stage the activations of this CTA's K range, 16 bytes per thread-step.
+  {
+    const int pieces = ng * (kGroup / 8);
+    for (int idx = threadIdx.x; idx < NT * pieces; idx += kGvThreads) {
+      const int n = idx / pieces, p = idx - n * pieces;
+      const uint4 v = *reinterpret_cast<const uint4*>(X + (size_t)n * K + (size_t)ga * kGroup + p * 8);
+      *reinterpret_cast<uint4*>(xs + n * xstride + p * 8) = v;
     }
-    __syncwarp();
-  } else {
-    // ----------------------------------------------------------- consumers
-    // Thread = weight row r of block b; consumer half h takes groups
-    // i = h, h + 2, ...; four independent fp32 chains per token.
-    const int h = warp >> 2;
-    const int r = (warp & 3) * 32 + lane;
-    float acc[NT][4];
-#pragma unroll
-    for (int n = 0; n < NT; ++n)
-#pragma unroll
-      for (int t = 0; t < 4; ++t) acc[n][t] = 0.f;
-    bool ok = ng == 0 || wait_bar_warp(xbar, 0, abort_flag, &g_gemv_status);
-    for (int i = h; ok && i < ng; i += kGvHalves) {
-      const int st = i % kGvStages;
-      const uint32_t ph = (uint32_t)((i / kGvStages) & 1);
-      if (!wait_bar_warp(&full[st], ph, abort_flag, &g_gemv_status)) break;
-      const uint8_t* src = smem + st * kGvStageBytes;
-      uint4 v[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const uint4*>(src + j * kRowBlock * 16 + r * 16);
-      const uint16_t sv = reinterpret_cast<const uint16_t*>(src + kGvWBytes)[r];
-      const uint32_t zb = src[kGvWBytes + kRowBlock * 2 + (r >> 1)];
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&empty[st]);
-      const GroupConsts gc = make_group_consts((zb >> ((r & 1) * 4)) & 0xFu, sv);
-      // The group's activations: token n at xg + n * ng * 16, then fixed offsets.
-      const uint4* xg = xs + i * (kGroup / 8);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint32_t words[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          uint32_t hw[4];
-          dequant_word(words[t], gc, hw);
-#pragma unroll
-          for (int n = 0; n < NT; ++n) {
-            const uint4 xv = xg[n * ng * (kGroup / 8) + j * 4 + t];
-            fma_h2(acc[n][t], hw[0], xv.x);
-            fma_h2(acc[n][t], hw[1], xv.y);
-            fma_h2(acc[n][t], hw[2], xv.z);
-            fma_h2(acc[n][t], hw[3], xv.w);
-          }
-        }
-      }
-    }
-#pragma unroll
-    for (int n = 0; n < NT; ++n)
-      red[(h * NT + n) * kRowBlock + r] = (acc[n][0] + acc[n][1]) + (acc[n][2] + acc[n][3]);
   }
   __syncthreads();
 
+  // Lanes of tokens g >= NT read token NT - 1: MMA columns are independent,
+  // and those columns are never stored.
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  const uint16_t* xg = xs + (g < NT ? g : NT - 1) * xstride + 32 * c;
+  for (int i0 = 0; i0 < ng; i0 += kGvDepth) {
+    gv_step<0>(f, i0, ng, pw, ps, pz, zsh, xg, acc);
+    pw += kGvDepth * kGvWBytes;
+    ps += kGvDepth * kRowBlock;
+    pz += kGvDepth * (kRowBlock / 2);
+    xg += kGvDepth * kGroup;
+  }
+  // Accumulator fragment: rows g (entries 0, 1) and g + 8 (entries 2, 3) of
+  // the tile, tokens 2 c and 2 c + 1.
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int n = 2 * c + e;
+    if (n < NT) {
+      red[n * kRowBlock + rl] = acc[e];
+      red[n * kRowBlock + rl + 8] = acc[2 + e];
+    }
+  }
+  __syncthreads();
+
+  float tot[NT];
   const int r = threadIdx.x;   // rows for the reduction: threads 0..127
   // The fused form's destination and bias of row m, loaded before the
   // reductions so the load overlaps them.
@@ -195,12 +270,7 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   }
   if (r < kRowBlock) {
 #pragma unroll
-    for (int n = 0; n < NT; ++n) {
-      float sum = 0.f;
-#pragma unroll
-      for (int h = 0; h < kGvHalves; ++h) sum += red[(h * NT + n) * kRowBlock + r];
-      tot[n] = sum;
-    }
+    for (int n = 0; n < NT; ++n) tot[n] = red[n * kRowBlock + r];
   }
 
   if (cl > 1) {
@@ -247,9 +317,9 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
 
 template <int NT, int kEpi>
 cudaError_t launch_nt(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p, const uint16_t* X,
-                      uint16_t* Y, int M, int K, int cl, cudaStream_t stream, const OutMap& om) {
+                      uint16_t* Y, int M, int K, int cl, bool pdl, cudaStream_t stream, const OutMap& om) {
   static std::atomic<unsigned long long> smem_set{0};
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(gemv_kernel<NT, kEpi>), 200 * 1024, smem_set);
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(gemv_kernel<NT, kEpi>), 128 * 1024, smem_set);
   if (e != cudaSuccess) return e;
   const int blocks = ceil_div(M, kRowBlock);
   const GvLayout L = gv_layout(NT, ceil_div(K / kGroup, cl), cl);
@@ -258,34 +328,35 @@ cudaError_t launch_nt(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p
   cfg.blockDim = dim3(kGvThreads, 1, 1);
   cfg.dynamicSmemBytes = (size_t)L.total;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)cl;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, gemv_kernel<NT, kEpi>, wq, s_p, z_p, X, Y, M, K, cl, om);
 }
 
 }  // namespace
 
 // Cluster size along K (1..8), from the measured LLaMA-7B N = 1 shapes:
-// all CTAs resident in one wave (kGvCtasPerSm per SM, set by the shared
-// memory of one CTA), and at least 2.5 CTAs per SM on average when the shape
+// all CTAs resident in one wave (kGvCtasPerSm per SM, set by the registers
+// of one CTA), and at least 2.5 CTAs per SM on average when the shape
 // allows it (fewer warps per SM hide the shared-memory and FMA latencies
 // badly); among those the smallest busiest-SM share of groups,
 // ceil(CTAs / SMs) x ceil(groups / cluster), then the smaller cluster.  When
 // no cluster reaches 2.5 CTAs per SM, the most CTAs.  The staged activation
 // slice must fit.
 int gemv_cluster_size(int M, int K, int sms, int nt) {
-  constexpr int kGvCtasPerSm = 4;
   const int blocks = ceil_div(M, kRowBlock);
   const int kg = K / kGroup;
   int best = 0;
   long long best_key[3] = {0, 0, 0};
   for (int cl = 1; cl <= kMaxCluster && cl <= kg; ++cl) {
-    if (nt * ceil_div(kg, cl) * kGroup * 2 > kMaxXSmem) continue;
+    if (nt * gv_xstride(ceil_div(kg, cl)) * 2 > kMaxXSmem) continue;
     const long long ctas = (long long)blocks * cl;
     if (cl > 1 && ctas > (long long)kGvCtasPerSm * sms) continue;
     const bool dense = 2 * ctas >= 5LL * sms;
@@ -302,11 +373,11 @@ int gemv_cluster_size(int M, int K, int sms, int nt) {
 
 cudaError_t launch_gemv(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros,
                         const uint16_t* X, uint16_t* Y, int M, int K, int N,
-                        cudaStream_t stream, const OutMap* om) {
+                        cudaStream_t stream, const OutMap* om, bool pdl) {
   for (int n0 = 0; n0 < N; n0 += kGemvMaxTokens) {
     const int nt = std::min(kGemvMaxTokens, N - n0);
     const int cl = gemv_cluster_size(M, K, num_sms(), nt);
-    if (nt * ceil_div(K / kGroup, cl) * kGroup * 2 > kMaxXSmem) return cudaErrorNotSupported;
+    if (nt * gv_xstride(ceil_div(K / kGroup, cl)) * 2 > kMaxXSmem) return cudaErrorNotSupported;
     const uint16_t* Xn = X + (size_t)n0 * K;
     uint16_t* Yn = om ? nullptr : Y + (size_t)n0 * M;
     // The fused outputs of tokens n0 .. n0 + nt - 1: each segment moves by
@@ -326,10 +397,14 @@ cudaError_t launch_gemv(const uint8_t* wq, const uint16_t* scales, const uint8_t
     cudaError_t e;
 #define W4A16_GEMV_NT(EPI)                                                                          \
     switch (nt) {                                                                                     \
-      case 1: e = launch_nt<1, EPI>(wq, scales, zeros, Xn, Yn, M, K, cl, stream, on); break;          \
-      case 2: e = launch_nt<2, EPI>(wq, scales, zeros, Xn, Yn, M, K, cl, stream, on); break;          \
-      case 3: e = launch_nt<3, EPI>(wq, scales, zeros, Xn, Yn, M, K, cl, stream, on); break;          \
-      default: e = launch_nt<4, EPI>(wq, scales, zeros, Xn, Yn, M, K, cl, stream, on); break;         \
+      case 1: e = launch_nt<1, EPI>(wq, scales, zeros, Xn, Yn, M, K, cl, pdl, stream, on); break;          \
+      case 2: e = launch_nt<2, EPI>(wq, scales, zeros, Xn, Yn, M, K, cl, pdl, stream, on); break;          \
+      case 3: e = launch_nt<3, EPI>(wq, scales, zeros, Xn, Yn, M, K, cl, pdl, stream, on); break;          \
+      case 4: e = launch_nt<4, EPI>(wq, scales, zeros, Xn, Yn, M, K, cl, pdl, stream, on); break;          \
+      case 5: e = launch_nt<5, EPI>(wq, scales, zeros, Xn, Yn, M, K, cl, pdl, stream, on); break;          \
+      case 6: e = launch_nt<6, EPI>(wq, scales, zeros, Xn, Yn, M, K, cl, pdl, stream, on); break;          \
+      case 7: e = launch_nt<7, EPI>(wq, scales, zeros, Xn, Yn, M, K, cl, pdl, stream, on); break;          \
+      default: e = launch_nt<8, EPI>(wq, scales, zeros, Xn, Yn, M, K, cl, pdl, stream, on); break;         \
     }
     if (kind == kEpiGateUp) {
       W4A16_GEMV_NT(kEpiGateUp)

@@ -537,6 +537,11 @@ cudaError_t launch_gemv_tc(const uint8_t* wq, const uint16_t* scales, const uint
                            uint16_t* Y, int M, int K, int N, void* workspace, bool pdl, cudaStream_t stream,
                            const OutMap* om) {
   if (N > kGemvTcMaxTokens) return cudaErrorNotSupported;
+  // The split-block counters must start at zero.  A completed call leaves
+  // its own counters at zero, but a call with more row blocks reaches bytes
+  // that an earlier, smaller call used for its fp32 partials: clear them.
+  cudaError_t e = cudaMemsetAsync(workspace, 0, gemv_tc_counter_bytes(M), stream);
+  if (e != cudaSuccess) return e;
   const int kind = om ? om->kind : kEpiPlain;
   const OutMap o = om ? *om : OutMap{};
   uint16_t* y = om ? nullptr : Y;

@@ -220,12 +220,15 @@ inline cudaError_t ensure_smem_limit(const void* fn, int bytes, std::atomic<unsi
 }
 
 // GEMV (CUDA cores): N in 1..kGemvMaxTokens per launch.
-constexpr int kGemvMaxTokens = 4;
+constexpr int kGemvMaxTokens = 8;
 
 // om: null for the plain [N][M] output Y, else the fused output map (Y unused).
+// With pdl the launch may overlap the previous kernel in the stream: the
+// first weight stages are read before the grid dependency wait, X and Y
+// after it.
 cudaError_t launch_gemv(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros,
                         const uint16_t* X, uint16_t* Y, int M, int K, int N,
-                        cudaStream_t stream, const OutMap* om = nullptr);
+                        cudaStream_t stream, const OutMap* om = nullptr, bool pdl = false);
 
 // Residual add + RMS normalisation: one CTA per token row, K a multiple of 8
 // and at most kMaxNormK (the row's residual is held in shared memory).
@@ -257,8 +260,6 @@ cudaError_t launch_gemm_tc(const uint8_t* wq, const uint16_t* scales, const uint
 // the launch may overlap the previous kernel in the stream: the weights are
 // read before the grid dependency wait, X, Y and the workspace after it.
 constexpr int kGemvTcMaxTokens = 64;
-// Tokens up to which the automatic choice (with a workspace) takes it.
-constexpr int kGemvTcAutoTokens = 16;
 size_t gemv_tc_counter_bytes(int M);
 size_t gemv_tc_workspace_bytes(int M, int K, int N);
 cudaError_t launch_gemv_tc(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros, const uint16_t* X,

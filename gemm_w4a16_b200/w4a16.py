@@ -18,7 +18,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_CUDA, ERR_TIMEOUT = ra
 PATH_AUTO, PATH_GEMV, PATH_TC, PATH_GEMV_TC = 0, 1, 2, 3
 FLAG_EARLY_WEIGHTS = 1
 GEMV_TC_MAX_TOKENS = 64      # forced W4A16_PATH_GEMV_TC
-GEMV_TC_AUTO_TOKENS = 16     # AUTO with a workspace takes it up to here
+GEMV_MAX_TOKENS = 8          # tokens of one decode-kernel launch; AUTO takes it up to here
 GROUP = 128
 
 EXPORTED = (
@@ -145,8 +145,8 @@ def workspace_size(M: int, K: int, N: int, group: int = GROUP) -> int:
 
 
 class Workspace:
-    """A zero-filled device buffer for the workspace entry points.  The
-    kernels leave it zero-filled after every completed call, so one buffer
+    """A device buffer for the workspace entry points (zero-filled when made;
+    each split-path call clears the counters it uses), so one buffer
     serves any number of calls in one stream; `ensure` grows it (outside
     CUDA-graph capture) to the size a call needs."""
 

@@ -52,21 +52,25 @@ typedef enum {
 
 /* Kernel selection for w4a16_gemm_ex and w4a16_gemm_ws. */
 typedef enum {
-    W4A16_PATH_AUTO = 0,     /* choose by N (and by whether a workspace is given) */
-    W4A16_PATH_GEMV = 1,     /* CUDA-core decode kernel (any N, best at one or two tokens) */
-    W4A16_PATH_TC = 2,       /* tcgen05 tile kernel (any N, best from a few tokens on) */
+    W4A16_PATH_AUTO = 0,     /* choose by N: GEMV for N <= 8, TC above */
+    W4A16_PATH_GEMV = 1,     /* decode kernel: weights streamed to registers, warp-level
+                                MMAs (any N, 8 tokens per launch; best up to 8) */
+    W4A16_PATH_TC = 2,       /* tcgen05 tile kernel (any N, best from 9 tokens on) */
     W4A16_PATH_GEMV_TC = 3   /* tcgen05 decode kernel, weight stream split over every SM
-                                (N <= 64; needs a workspace; AUTO takes it for N <= 16) */
+                                (N <= 64; needs a workspace; never chosen by AUTO: slower
+                                than GEMV and TC at every N measured) */
 } w4a16_path;
 
-/* Flags of the workspace entry points (w4a16_gemm_ws, w4a16_gemm_qkv_ws). */
+/* Flags of the workspace entry points (w4a16_gemm_ws, w4a16_gemm_qkv_ws,
+ * w4a16_gemm_gate_up_ws). */
 #define W4A16_FLAG_EARLY_WEIGHTS 1u
-/*   With W4A16_PATH_GEMV_TC, launch with programmatic dependent launch: the
- *   call's CTAs may start, and read the packed weight, while the previous
- *   kernel in the stream is still running; X, Y and the workspace are only
- *   touched after that kernel has completed.  The caller guarantees that no
- *   kernel still running writes the packed weight (true of weights loaded
- *   once, before inference).  Ignored by the other paths. */
+/*   On the decode paths (W4A16_PATH_GEMV, W4A16_PATH_GEMV_TC), launch with
+ *   programmatic dependent launch: the call's CTAs may start, and read the
+ *   packed weight, while the previous kernel in the stream is still running;
+ *   X, the bias, Y and the workspace are only touched after that kernel has
+ *   completed.  The caller guarantees that no kernel still running writes the
+ *   packed weight (true of weights loaded once, before inference).  Ignored
+ *   by the tensor-core tile path. */
 
 /* Human-readable name of a status code.  Never returns NULL. */
 W4A16_API const char* w4a16_status_string(int status);
@@ -251,17 +255,18 @@ W4A16_API w4a16_status w4a16_gemm_workspace_size(int M, int K, int N, int group,
  * w4a16_gemm with a caller-owned workspace, which lets the decode and
  * few-token product run on every SM ("PerfXLLM on Snapdragon 8 Gen2",
  * section 3.3 item 2: the GEMV is memory bound; the weight is tiled along
- * both its rows and K so the whole device streams it).  With path AUTO and
- * N <= 16 (or forced, N <= 64) this is W4A16_PATH_GEMV_TC: CTA c of G streams units
+ * both its rows and K so the whole device streams it).  With path AUTO it
+ * chooses as w4a16_gemm; forced W4A16_PATH_GEMV_TC (N <= 64): CTA c of G streams units
  * [c U / G, (c + 1) U / G) of the U = ceil(M/128) * K/128 (row block, group)
  * units; a block split between CTAs is summed, in CTA order, from fp32
  * partials in the workspace, so the result stays deterministic.
  *   workspace  device, 16-byte aligned, at least w4a16_gemm_workspace_size
- *              bytes; zero-filled before its first use.  A completed call
- *              leaves its counters at zero again.  One workspace serves any
- *              number of calls in one stream; calls that may run at the same
- *              time (different streams) need different workspaces.  After a
- *              W4A16_ERR_TIMEOUT the workspace must be zero-filled again.
+ *              bytes; its contents on entry do not matter: each call on the
+ *              split path first clears the counters it uses (an asynchronous
+ *              memset on `stream`), and a completed call leaves them at zero.
+ *              One workspace serves any number of calls in one stream; calls
+ *              that may run at the same time (different streams) need
+ *              different workspaces.
  *   workspace_bytes  its size.
  *   flags      0 or W4A16_FLAG_EARLY_WEIGHTS.
  * W4A16_ERR_INVALID_ARG when the forced path needs a workspace that is

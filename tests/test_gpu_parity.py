@@ -104,6 +104,14 @@ def test_ragged_shapes(M, K, N, path):
     full_case(M, K, N, path, seed=M + K + N)
 
 
+@pytest.mark.parametrize("N", list(range(1, 18)))
+def test_gemv_every_token_count(N):
+    """Every token count of one CUDA-core decode launch (1..8, the eight
+    columns of its MMA tile), then two launches (9..16) and a third (17), on
+    a shape with a ragged row block and a K split across a cluster."""
+    full_case(1500, 2048, N, w4a16.PATH_GEMV, seed=300 + N)
+
+
 @pytest.mark.parametrize("path", PATHS, ids=lambda p: PATH_NAMES[p])
 def test_outlier_channels_small(path):
     full_case(384, 1024, 33, path, seed=5, outlier_frac=0.01)
