@@ -5,9 +5,10 @@ Default workload (one "step"): a LLaMA-7B-shaped decode step at N = 1 token --
 32 layers x {fused QKV 12288x4096, O 4096x4096, fused gate/up 22016x4096,
 down 4096x11008}, 128 distinct packed weight sets resident in HBM (3.37 GB, far
 beyond the 126 MB L2, so no flush is needed), each projection one
-w4a16_gemm_ws call (the split tensor-core decode kernel, weights streamed
-early under programmatic dependent launch), the step captured once in a CUDA
-graph.  The metric is algorithmic HBM bytes per second (packed int4 weights +
+w4a16_gemm_ws call on the automatic path (the decode kernel: weights streamed
+from HBM into registers, warp-level MMAs on the exact dequant, the first
+weight groups requested before the grid dependency wait under programmatic
+dependent launch), the step captured once in a CUDA graph.  The metric is algorithmic HBM bytes per second (packed int4 weights +
 2.5 B per group of metadata + fp16 X and Y), reported against the measured HBM
 copy bandwidth.  The same JSON line carries, each with its own clock summary
 and median / p10 / p90 over its repeats: every projection alone, the two
@@ -46,10 +47,10 @@ N_LAYERS = 32
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one decode
-# launch of the split tensor-core kernel on the fused QKV shape at N = 1, from
-# an ncu capture of this repository's kernel; it holds only while the kernel
-# source is the one captured (sha256 prefix of csrc/w4a16_gemv_tc.cu), and
-# the bench reports null otherwise.
+# launch of the decode kernel on the fused QKV shape at N = 1, from an ncu
+# capture of this repository's kernel; it holds only while the kernel source
+# is the one captured (sha256 prefix of csrc/w4a16_gemv.cu), and the bench
+# reports null otherwise.
 DECODE_TRAFFIC = {"src_sha256_prefix": "", "qkv_dram_bytes": 0, "qkv_alg_bytes": 26181632}
 NOMINAL_DENSE_FP16_TFLOPS = 2250.0   # B200 dense fp16/bf16 tensor rate, NVIDIA's figure
 
@@ -69,7 +70,7 @@ def decode_traffic_per_launch(alg_bytes_per_launch):
     the kernel source changed since the capture."""
     import hashlib
 
-    src = os.path.join(ROOT, "gemm_w4a16_b200", "csrc", "w4a16_gemv_tc.cu")
+    src = os.path.join(ROOT, "gemm_w4a16_b200", "csrc", "w4a16_gemv.cu")
     try:
         h = hashlib.sha256(open(src, "rb").read()).hexdigest()
     except OSError:
@@ -505,9 +506,9 @@ def main_ours(args):
                    "bytes_per_step": step_bytes, "global_batch": 1, "seq_len": 1,
                    "l2": "inputs 3.37 GB per step > 126 MB L2 (no flush needed)",
                    "launch": "cuda_graph, programmatic dependent launch (early weights)",
-                   "api": "w4a16_gemm_ws (auto path: split tensor-core decode kernel)",
+                   "api": "w4a16_gemm_ws (auto path: decode kernel gemv_kernel, early weights)",
                    "parallelism": f"replicas{world}"},
-        "roofline": {"bound": "hbm", "kernel": "gemv_tc_kernel", "achieved": achieved,
+        "roofline": {"bound": "hbm", "kernel": "gemv_kernel", "achieved": achieved,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks_src,
                      "traffic": decode_traffic_per_launch(step_bytes / launches_per_step),
@@ -606,8 +607,8 @@ SWEEP_N = (1, 2, 4, 8, 16, 32, 64, 128, 256, 512, 1024, 2048, 4096)
 
 def n_sweep_measure(device, peaks, sampler, copies=16, reps=20):
     """N sweep on the fused QKV shape (M = 12288, K = 4096), every kernel that
-    takes the N (CUDA-core GEMV up to 64 tokens, split tensor-core decode up
-    to 16, tensor-core tiles always), 16 rotated weight copies (420 MB,
+    takes the N (decode kernel up to 64 tokens, 8 per launch; split
+    tensor-core decode up to 64; tensor-core tiles always), 16 rotated weight copies (420 MB,
     beyond L2).  Rows: [N, path, median us, roofline fraction, chosen]."""
     import torch
 
@@ -630,7 +631,7 @@ def n_sweep_measure(device, peaks, sampler, copies=16, reps=20):
         if N <= w4a16.GEMV_TC_MAX_TOKENS:
             paths.append(w4a16.PATH_GEMV_TC)
         for path in paths:
-            flags = w4a16.FLAG_EARLY_WEIGHTS if path == w4a16.PATH_GEMV_TC else 0
+            flags = w4a16.FLAG_EARLY_WEIGHTS if path != w4a16.PATH_TC else 0
             g = capture(lambda path=path, flags=flags: [w4a16.gemm_ws(w, x, Y=y, path=path, workspace=wsp,
                                                                      flags=flags) for w in ws_copies], device)
             _, per = time_steps(g, reps, 3, device)
@@ -985,7 +986,7 @@ def main(argv=None):
     ap.add_argument("--K", type=int, default=4096)
     ap.add_argument("--N", type=int, default=1)
     ap.add_argument("--path", type=int, default=0,
-                    help="0 auto, 1 CUDA-core GEMV, 2 tensor-core tiles, 3 split tensor-core decode")
+                    help="0 auto, 1 decode kernel, 2 tensor-core tiles, 3 split tensor-core decode")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-extra", action="store_true",

@@ -16,14 +16,16 @@
 //    previous kernel finishes; the activations (written by that kernel) are
 //    staged in shared memory after the wait;
 //  * the products run on the tensor cores as warp-level mma.sync m16n8k16
-//    (f16 inputs, fp32 accumulation): lane l = 4 g + c holds rows g and g + 8
-//    of the tile and chunk c (32 codes) of each; the exact dequant of one
-//    32-bit word (8 codes) of each row gives the lane's A fragments of two
-//    MMAs, whose B fragments are token g's activations at the same eight k
-//    (one 16-byte shared load).  The MMA's k order is thus a permutation of
-//    the group that A and B share; tokens g >= NT are zero columns.  One MMA
-//    instruction replaces 256 fp32 FMAs, so the kernel issues about 2.3
-//    instructions per weight (1.6 of them the exact dequant);
+//    (f16 inputs, fp32 accumulation): lane l = 4 g + c holds MMA rows g and
+//    g + 8, which are the adjacent block rows 2 g and 2 g + 1 of the tile (so
+//    one 32-bit load brings both scales and one byte both zero codes), and
+//    chunk c (32 codes) of each; the exact dequant of one 32-bit word (8
+//    codes) of each row gives the lane's A fragments of two MMAs, whose B
+//    fragments are token g's activations at the same eight k (one 16-byte
+//    shared load).  The MMA's k order is thus a permutation of the group that
+//    A and B share; lanes of tokens g >= NT feed columns that are never
+//    stored.  One MMA instruction replaces 256 fp32 FMAs, so the kernel issues
+//    about 2.5 instructions per weight, 1.6 of them the exact dequant;
 //  * split-K: CTAs of a thread-block cluster (up to 8 along K) reduce through
 //    distributed shared memory into the cluster's rank-0 CTA in a fixed order
 //    (deterministic, no atomics).
@@ -68,9 +70,9 @@ __device__ __forceinline__ uint4 ldg_v4_at(const void* p) {
 }
 
 template <int OFF>
-__device__ __forceinline__ uint32_t ldg_u16_at(const void* p) {
-  unsigned short v;
-  asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1+%2];" : "=h"(v) : "l"(p), "n"(OFF));
+__device__ __forceinline__ uint32_t ldg_u32_at(const void* p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1+%2];" : "=r"(v) : "l"(p), "n"(OFF));
   return v;
 }
 
@@ -99,24 +101,22 @@ __host__ __device__ inline GvLayout gv_layout(int nt, int gspan, int cl) {
   return L;
 }
 
-// One group's operands of one lane: chunk c of rows r (lo) and r + 8 (hi),
-// their scales and the bytes holding their zero codes.
+// One group's operands of one lane: chunk c of the adjacent rows r (even)
+// and r + 1 (two 16-byte halves of 32 contiguous bytes), their two scales
+// (one 32-bit word) and the zero byte that holds both codes.
 struct GvFrag {
   uint4 lo, hi;
-  uint32_t s_lo, s_hi, z_lo, z_hi;
+  uint32_t s, z;
 };
 
 // Group J of the lane's streams: pw points at chunk c of row r of group 0,
-// ps at the scale of row r, pz at the zero byte of row r (row r + 8: 128,
-// 8 and 4 bytes further).
+// ps at the scale of row r, pz at the zero byte of rows r and r + 1.
 template <int J>
 __device__ __forceinline__ void gv_load(GvFrag& f, const uint8_t* pw, const uint16_t* ps, const uint8_t* pz) {
   f.lo = ldg_v4_at<J * kGvWBytes>(pw);
-  f.hi = ldg_v4_at<J * kGvWBytes + 8 * 16>(pw);
-  f.s_lo = ldg_u16_at<J * kRowBlock * 2>(ps);
-  f.s_hi = ldg_u16_at<J * kRowBlock * 2 + 16>(ps);
-  f.z_lo = ldg_u8_at<J * (kRowBlock / 2)>(pz);
-  f.z_hi = ldg_u8_at<J * (kRowBlock / 2) + 4>(pz);
+  f.hi = ldg_v4_at<J * kGvWBytes + 16>(pw);
+  f.s = ldg_u32_at<J * kRowBlock * 2>(ps);
+  f.z = ldg_u8_at<J * (kRowBlock / 2)>(pz);
 }
 
 template <uint32_t SEL>
@@ -127,26 +127,25 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b) {
 }
 
 // The dequant constants (as make_group_consts) of the lane's two rows at
-// once: the two zero codes side by side in one register (row lo in the low
+// once: the two zero codes side by side in one register (row r in the low
 // half), both fp16 forms built there, then each half copied to both halves.
-// zsh = 4 for odd rows (their code sits in bits 4..7 of the zero byte).
-__device__ __forceinline__ void gv_consts(const GvFrag& f, int zsh, GroupConsts& lo, GroupConsts& hi) {
-  const uint32_t zz = prmt<0x5410>(f.z_lo, f.z_hi);                       // bytes: z_lo, 0, z_hi, 0
-  const uint32_t a = lop3_and_or(zz >> zsh, 0x000F000Fu, 0x64006400u);     // 1024 + z per half
-  const uint32_t b = lop3_and_or(zz << (4 - zsh), 0x00F000F0u, 0xD400D400u);  // -(64 + z) per half
+__device__ __forceinline__ void gv_consts(const GvFrag& f, GroupConsts& lo, GroupConsts& hi) {
+  const uint32_t t = f.z | (f.z << 12);                                   // code of row r + 1 at bits 16..19
+  const uint32_t a = lop3_and_or(t, 0x000F000Fu, 0x64006400u);             // 1024 + z per half
+  const uint32_t b = lop3_and_or(t << 4, 0x00F000F0u, 0xD400D400u);        // -(64 + z) per half
   lo.z1024 = prmt<0x1010>(a, a);
   hi.z1024 = prmt<0x3232>(a, a);
   lo.zneg64 = prmt<0x1010>(b, b);
   hi.zneg64 = prmt<0x3232>(b, b);
-  lo.s2 = prmt<0x1010>(f.s_lo, f.s_lo);
-  hi.s2 = prmt<0x1010>(f.s_hi, f.s_hi);
+  lo.s2 = prmt<0x1010>(f.s, f.s);
+  hi.s2 = prmt<0x3232>(f.s, f.s);
 }
 
 // Dequantise one group of the lane's two rows and accumulate its eight MMAs;
 // xg points at token g's activations at k = 32 c of the group.
-__device__ __forceinline__ void gv_consume(const GvFrag& f, int zsh, const uint16_t* xg, float (&acc)[4]) {
+__device__ __forceinline__ void gv_consume(const GvFrag& f, const uint16_t* xg, float (&acc)[4]) {
   GroupConsts clo, chi;
-  gv_consts(f, zsh, clo, chi);
+  gv_consts(f, clo, chi);
   const uint32_t wl[4] = {f.lo.x, f.lo.y, f.lo.z, f.lo.w};
   const uint32_t wh[4] = {f.hi.x, f.hi.y, f.hi.z, f.hi.w};
 #pragma unroll
@@ -173,13 +172,13 @@ __device__ __forceinline__ void gv_load_first(GvFrag (&f)[kGvDepth], int ng, con
 // group i0 + U from slot U, refill the slot with group i0 + U + kGvDepth.
 template <int U>
 __device__ __forceinline__ void gv_step(GvFrag (&f)[kGvDepth], int i0, int ng, const uint8_t* pw,
-                                        const uint16_t* ps, const uint8_t* pz, int zsh, const uint16_t* xg,
+                                        const uint16_t* ps, const uint8_t* pz, const uint16_t* xg,
                                         float (&acc)[4]) {
   if constexpr (U < kGvDepth) {
     if (i0 + U < ng) {
-      gv_consume(f[U], zsh, xg + U * kGroup, acc);
+      gv_consume(f[U], xg + U * kGroup, acc);
       if (i0 + U + kGvDepth < ng) gv_load<U + kGvDepth>(f[U], pw, ps, pz);
-      gv_step<U + 1>(f, i0, ng, pw, ps, pz, zsh, xg, acc);
+      gv_step<U + 1>(f, i0, ng, pw, ps, pz, xg, acc);
     }
   }
 }
@@ -210,10 +209,10 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   ptx::griddep_launch_dependents();
   if (cl > 1) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 
-  // This lane's rows within the block, and its group streams (pointers at
-  // group ga; slot offsets are folded into the loads).
-  const int rl = 16 * warp + g;
-  const int zsh = (g & 1) * 4;          // rows rl and rl + 8 have the same parity
+  // This lane's rows within the block: MMA rows g and g + 8 of the warp's
+  // tile are the adjacent block rows rl and rl + 1.  Its group streams
+  // (pointers at group ga; slot offsets are folded into the loads).
+  const int rl = 16 * warp + 2 * g;
   const uint8_t* pw = wq + (size_t)b * kc_n * kRowBlock * 16 + (size_t)ga * kGvWBytes + c * (kRowBlock * 16) + rl * 16;
   const uint16_t* ps = s_p + ((size_t)b * kg + ga) * kRowBlock + rl;
   const uint8_t* pz = z_p + ((size_t)b * kg + ga) * (kRowBlock / 2) + (rl >> 1);
@@ -241,20 +240,20 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   const uint16_t* xg = xs + (g < NT ? g : NT - 1) * xstride + 32 * c;
   for (int i0 = 0; i0 < ng; i0 += kGvDepth) {
-    gv_step<0>(f, i0, ng, pw, ps, pz, zsh, xg, acc);
+    gv_step<0>(f, i0, ng, pw, ps, pz, xg, acc);
     pw += kGvDepth * kGvWBytes;
     ps += kGvDepth * kRowBlock;
     pz += kGvDepth * (kRowBlock / 2);
     xg += kGvDepth * kGroup;
   }
-  // Accumulator fragment: rows g (entries 0, 1) and g + 8 (entries 2, 3) of
-  // the tile, tokens 2 c and 2 c + 1.
+  // Accumulator fragment: MMA rows g (entries 0, 1: block row rl) and g + 8
+  // (entries 2, 3: block row rl + 1), tokens 2 c and 2 c + 1.
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
     const int n = 2 * c + e;
     if (n < NT) {
       red[n * kRowBlock + rl] = acc[e];
-      red[n * kRowBlock + rl + 8] = acc[2 + e];
+      red[n * kRowBlock + rl + 1] = acc[2 + e];
     }
   }
   __syncthreads();
