@@ -339,6 +339,31 @@ w4a16_status w4a16_gemm_gate_up_ws(const void* wq_packed, const void* scales_pac
                            workspace_bytes, flags, stream);
 }
 
+w4a16_status w4a16_gemm_noalloc(const void* wq_packed, const void* scales_packed, const void* zeros_packed,
+                                const uint16_t* X, uint16_t* Y, int M, int K, int N, int group, unsigned flags,
+                                void* stream) {
+  if (!wq_packed || !scales_packed || !zeros_packed || !X || !Y || N <= 0) return W4A16_ERR_INVALID_ARG;
+  if (flags & ~W4A16_FLAG_EARLY_WEIGHTS) return W4A16_ERR_INVALID_ARG;
+  w4a16_status st = check_shape(M, K, group);
+  if (st != W4A16_OK) return st;
+  if (N > kGemvTcMaxTokens || gemv_tc_workspace_bytes(M, K, N) > kNoallocScratchBytes)
+    return W4A16_ERR_UNSUPPORTED;
+  if (!aligned16(wq_packed) || !aligned16(scales_packed) || !aligned16(zeros_packed) || !aligned16(X) ||
+      !aligned16(Y))
+    return W4A16_ERR_MISALIGNED;
+  {
+    const PackedBytes pb = packed_bytes(M, K);
+    const size_t ny = (size_t)N * M * 2, nx = (size_t)N * K * 2;
+    if (overlap(Y, ny, X, nx) || overlaps_weight(Y, ny, wq_packed, scales_packed, zeros_packed, pb))
+      return W4A16_ERR_INVALID_ARG;
+  }
+  return map_cuda(launch_gemv_tc_noalloc(static_cast<const uint8_t*>(wq_packed),
+                                         static_cast<const uint16_t*>(scales_packed),
+                                         static_cast<const uint8_t*>(zeros_packed), X, Y, M, K, N,
+                                         (flags & W4A16_FLAG_EARLY_WEIGHTS) != 0,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
 int w4a16_select_path(int M, int K, int N) { return select_path_impl(M, K, N, false); }
 
 int w4a16_select_path_ws(int M, int K, int N) { return select_path_impl(M, K, N, true); }

@@ -560,6 +560,51 @@ cudaError_t launch_gemv_tc(const uint8_t* wq, const uint16_t* scales, const uint
 #undef W4A16_GVTC
 }
 
+// ------------------------------------------------ allocation-free variant
+//
+// Scratch of w4a16_gemm_noalloc: the split-block counters and fp32 partials
+// of the split decode kernel live in this fixed device array instead of a
+// caller workspace, so that call allocates nothing.  Every GPU that loads the
+// library holds the array until the process exits.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoallocScratchBytes];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::atomic<void*> g_noalloc_ptr[kMaxDevices];
+
+// Device address of the array on the current device, looked up once per
+// device (the first call on a device does it, with that device current).
+cudaError_t noalloc_scratch(void** ptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorNotSupported;
+  void* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (!p) {
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[dev].store(p, std::memory_order_release);
+  }
+  *ptr = p;
+  return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_gemv_tc_noalloc(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros,
+                                   const uint16_t* X, uint16_t* Y, int M, int K, int N, bool pdl,
+                                   cudaStream_t stream) {
+  if (N > kGemvTcMaxTokens || gemv_tc_workspace_bytes(M, K, N) > kNoallocScratchBytes)
+    return cudaErrorNotSupported;
+  void* ws = nullptr;
+  const cudaError_t e = noalloc_scratch(&ws);
+  if (e != cudaSuccess) return e;
+  // launch_gemv_tc clears the counters first; the partials are written
+  // before they are read.
+  return launch_gemv_tc(wq, scales, zeros, X, Y, M, K, N, ws, pdl, stream, nullptr);
+}
+
 cudaError_t read_and_clear_gvtc_status(int* v) {
   cudaError_t e = cudaMemcpyFromSymbol(v, g_gvtc_status, sizeof(int));
   if (e != cudaSuccess) return e;

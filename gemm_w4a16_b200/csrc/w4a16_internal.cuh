@@ -261,6 +261,13 @@ cudaError_t launch_gemm_tc(const uint8_t* wq, const uint16_t* scales, const uint
 // read before the grid dependency wait, X, Y and the workspace after it.
 constexpr int kGemvTcMaxTokens = 64;
 size_t gemv_tc_counter_bytes(int M);
+// w4a16_gemm_noalloc: the same kernel on a fixed device array of this many
+// bytes instead of a caller workspace (cudaErrorNotSupported when the sizes
+// need more).
+constexpr size_t kNoallocScratchBytes = (size_t)4 << 20;
+cudaError_t launch_gemv_tc_noalloc(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros,
+                                   const uint16_t* X, uint16_t* Y, int M, int K, int N, bool pdl,
+                                   cudaStream_t stream);
 size_t gemv_tc_workspace_bytes(int M, int K, int N);
 cudaError_t launch_gemv_tc(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros, const uint16_t* X,
                            uint16_t* Y, int M, int K, int N, void* workspace, bool pdl, cudaStream_t stream,

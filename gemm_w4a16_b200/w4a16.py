@@ -27,6 +27,7 @@ EXPORTED = (
     "w4a16_device_status", "w4a16_selftest_wait_timeout", "w4a16_quantize", "w4a16_gemm_qkv",
     "w4a16_add_rmsnorm", "w4a16_gemm_workspace_size", "w4a16_gemm_ws", "w4a16_gemm_qkv_ws",
     "w4a16_select_path_ws", "w4a16_pack_gate_up", "w4a16_gemm_gate_up", "w4a16_gemm_gate_up_ws",
+    "w4a16_gemm_noalloc",
 )
 
 _lib = None
@@ -76,6 +77,8 @@ def lib():
             L.w4a16_select_path_ws.restype = _i
             L.w4a16_gemm_workspace_size.argtypes = [_i, _i, _i, _i, _szp]
             L.w4a16_gemm_workspace_size.restype = _i
+            L.w4a16_gemm_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _u, _vp]
+            L.w4a16_gemm_noalloc.restype = _i
             L.w4a16_gemm_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _sz, _u, _vp]
             L.w4a16_gemm_ws.restype = _i
             L.w4a16_gemm_qkv_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp,

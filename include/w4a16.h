@@ -303,6 +303,35 @@ W4A16_API w4a16_status w4a16_gemm_ex(const void* wq_packed, const void* scales_p
  * tiling with the number of tokens; the crossovers here are measured. */
 W4A16_API int w4a16_select_path(int M, int K, int N);
 
+/*
+ * w4a16_gemm on the split decode kernel (W4A16_PATH_GEMV_TC) without any
+ * allocation, for callers that cannot call cudaMalloc: plug-ins inside a
+ * framework whose caching allocator or fixed arena owns all device memory
+ * (a cudaMalloc behind its back fragments or overcommits it), and servers
+ * that reserve their whole memory budget at start-up and may not allocate
+ * afterwards.  Such callers also have no workspace to hand to
+ * w4a16_gemm_ws.  The papers have no counterpart to this entry point: it is
+ * an interface choice of this library.
+ *   The kernel's scratch (split-block counters and fp32 partials) is a
+ *   file-scope device array of 4 MiB, held by every GPU that loads the
+ *   library until the process exits.  Sizes whose scratch
+ *   (w4a16_gemm_workspace_size) exceeds 4 MiB, or N > 64, return
+ *   W4A16_ERR_UNSUPPORTED; on a 148-SM device that allows N <= 16 for every
+ *   LLaMA shape.
+ *   The first call on a device looks up the array's address with that device
+ *   current (cudaGetSymbolAddress); make that first call before any stream
+ *   capture.  Each call clears the counters (an asynchronous memset on
+ *   `stream`) and then launches the kernel.
+ *   Every call on a device shares the one array, which keeps the last call's
+ *   contents: calls that overlap on the GPU (different streams, or
+ *   programmatic overlap with another such call) race on it and must be
+ *   ordered by the caller.
+ *   flags as w4a16_gemm_ws; other arguments as w4a16_gemm_ex.
+ */
+W4A16_API w4a16_status w4a16_gemm_noalloc(const void* wq_packed, const void* scales_packed,
+                           const void* zeros_packed, const uint16_t* X, uint16_t* Y,
+                           int M, int K, int N, int group, unsigned flags, void* stream);
+
 /* The path w4a16_gemm_ws with a workspace would take. */
 W4A16_API int w4a16_select_path_ws(int M, int K, int N);
 
