@@ -69,6 +69,11 @@ __device__ __forceinline__ uint4 ldg_v4_at(const void* p) {
   return r;
 }
 
+// 16-byte asynchronous global -> shared copy (no register staging).
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ptx::smem_addr(smem_dst)), "l"(src) : "memory");
+}
+
 template <int OFF>
 __device__ __forceinline__ uint32_t ldg_u32_at(const void* p) {
   uint32_t v;
@@ -168,6 +173,17 @@ __device__ __forceinline__ void gv_load_first(GvFrag (&f)[kGvDepth], int ng, con
   }
 }
 
+// Slots U.. of a step whose groups and refills all exist (no checks).
+template <int U>
+__device__ __forceinline__ void gv_step_full(GvFrag (&f)[kGvDepth], const uint8_t* pw, const uint16_t* ps,
+                                             const uint8_t* pz, const uint16_t* xg, float (&acc)[4]) {
+  if constexpr (U < kGvDepth) {
+    gv_consume(f[U], xg + U * kGroup, acc);
+    gv_load<U + kGvDepth>(f[U], pw, ps, pz);
+    gv_step_full<U + 1>(f, pw, ps, pz, xg, acc);
+  }
+}
+
 // Slots U.. of one step of kGvDepth groups starting at group i0: consume
 // group i0 + U from slot U, refill the slot with group i0 + U + kGvDepth.
 template <int U>
@@ -187,7 +203,7 @@ template <int NT, int kEpi>
 __global__ void __launch_bounds__(kGvThreads, kGvCtasPerSm)
 gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
             const uint8_t* __restrict__ z_p, const uint16_t* __restrict__ X,
-            uint16_t* __restrict__ Y, int M, int K, int cl, OutMap om) {
+            uint16_t* __restrict__ Y, int M, int K, int cl, int early, OutMap om) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int kg = K / kGroup;
   const int kc_n = K / kChunkK;
@@ -217,29 +233,41 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   const uint16_t* ps = s_p + ((size_t)b * kg + ga) * kRowBlock + rl;
   const uint8_t* pz = z_p + ((size_t)b * kg + ga) * (kRowBlock / 2) + (rl >> 1);
 
-  // The first groups depend on no earlier kernel: request them before the
-  // grid dependency wait (which returns at once unless the launch is
-  // programmatic).
-  GvFrag f[kGvDepth];
-  gv_load_first<0>(f, ng, pw, ps, pz);
-  ptx::griddep_wait();
-
-  // Stage the activations of this CTA's K range, 16 bytes per thread-step.
-  {
+  // The activations of this CTA's K range go to shared memory with
+  // asynchronous 16-byte copies.  Without programmatic launch they are
+  // requested first, so they do not queue behind the weight stream.
+  auto stage_x = [&]() {
     const int pieces = ng * (kGroup / 8);
     for (int idx = threadIdx.x; idx < NT * pieces; idx += kGvThreads) {
       const int n = idx / pieces, p = idx - n * pieces;
-      const uint4 v = *reinterpret_cast<const uint4*>(X + (size_t)n * K + (size_t)ga * kGroup + p * 8);
-      *reinterpret_cast<uint4*>(xs + n * xstride + p * 8) = v;
+      cp_async16(xs + n * xstride + p * 8, X + (size_t)n * K + (size_t)ga * kGroup + p * 8);
     }
-  }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  if (!early) stage_x();
+  // The first groups depend on no earlier kernel: request them before the
+  // grid dependency wait (which returns at once unless the launch is
+  // programmatic); X, written by that kernel, only after it.
+  GvFrag f[kGvDepth];
+  gv_load_first<0>(f, ng, pw, ps, pz);
+  ptx::griddep_wait();
+  if (early) stage_x();
+  asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
 
   // Lanes of tokens g >= NT read token NT - 1: MMA columns are independent,
   // and those columns are never stored.
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   const uint16_t* xg = xs + (g < NT ? g : NT - 1) * xstride + 32 * c;
-  for (int i0 = 0; i0 < ng; i0 += kGvDepth) {
+  int i0 = 0;
+  for (; i0 + 2 * kGvDepth <= ng; i0 += kGvDepth) {   // every refill exists
+    gv_step_full<0>(f, pw, ps, pz, xg, acc);
+    pw += kGvDepth * kGvWBytes;
+    ps += kGvDepth * kRowBlock;
+    pz += kGvDepth * (kRowBlock / 2);
+    xg += kGvDepth * kGroup;
+  }
+  for (; i0 < ng; i0 += kGvDepth) {
     gv_step<0>(f, i0, ng, pw, ps, pz, xg, acc);
     pw += kGvDepth * kGvWBytes;
     ps += kGvDepth * kRowBlock;
@@ -336,7 +364,7 @@ cudaError_t launch_nt(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, gemv_kernel<NT, kEpi>, wq, s_p, z_p, X, Y, M, K, cl, om);
+  return cudaLaunchKernelEx(&cfg, gemv_kernel<NT, kEpi>, wq, s_p, z_p, X, Y, M, K, cl, pdl ? 1 : 0, om);
 }
 
 }  // namespace
