@@ -62,11 +62,23 @@ w4a16_status map_cuda(cudaError_t e) {
   return W4A16_ERR_CUDA;
 }
 
-// with_ws: a workspace is available, which opens the split decode kernel.
+// Largest M at which two decode launches beat the tile kernel: up to 64 row
+// blocks the tile kernel has too few tiles to fill the SMs (32 at M = 4096).
+// Measured at N = 16: the 4096 x 4096 projection takes 12 us as two decode
+// launches against 24 us on the tile kernel; the 12288 x 4096 one 22 us
+// against 17 us.
+constexpr int kTwoLaunchMaxM = 8192;
+
+// The decode kernel up to one launch of tokens, or two launches on weights of
+// at most kTwoLaunchMaxM rows; the tile kernel above.  with_ws: a workspace is
+// available (it would open the split decode kernel, which is never the faster
+// one: forced only).
 int select_path_impl(int M, int K, int N, bool with_ws) {
   if (M <= 0 || K <= 0 || N <= 0 || K % kGroup) return -1;
-  (void)with_ws;   // the split decode path is never the faster one (forced only)
-  return N <= gemv_max_n() ? W4A16_PATH_GEMV : W4A16_PATH_TC;
+  (void)with_ws;
+  if (N <= gemv_max_n()) return W4A16_PATH_GEMV;
+  if (N <= 2 * gemv_max_n() && M <= kTwoLaunchMaxM) return W4A16_PATH_GEMV;
+  return W4A16_PATH_TC;
 }
 
 size_t workspace_for(int path, int M, int K, int N) {

@@ -52,10 +52,11 @@ typedef enum {
 
 /* Kernel selection for w4a16_gemm_ex and w4a16_gemm_ws. */
 typedef enum {
-    W4A16_PATH_AUTO = 0,     /* choose by N: GEMV for N <= 8, TC above */
+    W4A16_PATH_AUTO = 0,     /* choose by N and M: GEMV for N <= 8, and for N <= 16
+                                when M <= 8192; TC above */
     W4A16_PATH_GEMV = 1,     /* decode kernel: weights streamed to registers, warp-level
-                                MMAs (any N, 8 tokens per launch; best up to 8) */
-    W4A16_PATH_TC = 2,       /* tcgen05 tile kernel (any N, best from 9 tokens on) */
+                                MMAs (any N, 8 tokens per launch) */
+    W4A16_PATH_TC = 2,       /* tcgen05 tile kernel (any N) */
     W4A16_PATH_GEMV_TC = 3   /* tcgen05 decode kernel, weight stream split over every SM
                                 (N <= 64; needs a workspace; never chosen by AUTO: slower
                                 than GEMV and TC at every N measured) */
@@ -351,6 +352,10 @@ W4A16_API w4a16_status w4a16_dequant_debug(const void* wq_packed, const void* sc
  * Synchronises `stream`, then reads and clears the device-side status words
  * that bounded waits inside the kernels set when they give up.
  * Writes W4A16_OK or W4A16_ERR_TIMEOUT to *status.  Not for the hot path.
+ * The words are per device, shared by every stream, and read and cleared by
+ * two separate copies: the answer is exact only while no other stream runs
+ * this library's kernels on the device (a timeout recorded between the two
+ * copies would be cleared unseen).
  */
 W4A16_API w4a16_status w4a16_device_status(void* stream, int* status);
 

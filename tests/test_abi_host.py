@@ -226,6 +226,11 @@ def test_select_path_with_workspace(L):
         assert w4a16.select_path(12288, 4096, N) == w4a16.PATH_GEMV
     for N in (w4a16.GEMV_MAX_TOKENS + 1, 64, 4096):
         assert w4a16.select_path_ws(12288, 4096, N) == w4a16.PATH_TC
+    # Up to 8192 rows (64 row blocks) two decode launches beat the tile kernel.
+    for M in (4096, 6144, 8192):
+        assert w4a16.select_path(M, 4096, 2 * w4a16.GEMV_MAX_TOKENS) == w4a16.PATH_GEMV
+        assert w4a16.select_path(M, 4096, 2 * w4a16.GEMV_MAX_TOKENS + 1) == w4a16.PATH_TC
+    assert w4a16.select_path(8320, 4096, 2 * w4a16.GEMV_MAX_TOKENS) == w4a16.PATH_TC
     assert w4a16.select_path_ws(12288, 100, 1) == -1
 
 
