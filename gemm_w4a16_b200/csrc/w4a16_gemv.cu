@@ -97,11 +97,11 @@ struct GvLayout {
   int x_off, red_off, cred_off, total;
 };
 
-__host__ __device__ inline GvLayout gv_layout(int nt, int gspan, int cl) {
+__host__ __device__ inline GvLayout gv_layout(int nt, int gspan, int cl, int kw) {
   GvLayout L;
   L.x_off = 0;
   L.red_off = L.x_off + nt * gv_xstride(gspan) * 2;
-  L.cred_off = L.red_off + nt * kRowBlock * 4;
+  L.cred_off = L.red_off + kw * nt * kRowBlock * 4;
   L.total = L.cred_off + (cl > 1 ? cl * nt * kRowBlock * 4 : 0);
   return L;
 }
@@ -199,7 +199,11 @@ __device__ __forceinline__ void gv_step(GvFrag (&f)[kGvDepth], int i0, int ng, c
   }
 }
 
-template <int NT, int kEpi>
+// KW = 1: the CTA's 8 warps are the 8 row tiles of a 128-row block; KW = 2:
+// 4 row tiles (half a block) with two warps each, which take the two halves
+// of the CTA's K range and meet in shared memory (more warps per row for
+// shapes with few row blocks).
+template <int NT, int kEpi, int KW>
 __global__ void __launch_bounds__(kGvThreads, kGvCtasPerSm)
 gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
             const uint8_t* __restrict__ z_p, const uint16_t* __restrict__ X,
@@ -208,19 +212,27 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   const int kg = K / kGroup;
   const int kc_n = K / kChunkK;
   const int gspan = ceil_div(kg, cl);
-  const GvLayout L = gv_layout(NT, gspan, cl);
+  const GvLayout L = gv_layout(NT, gspan, cl, KW);
+  constexpr int kRows = kRowBlock / KW;    // rows of the CTA
+  constexpr int kTiles = kGvWarps / KW;    // 16-row tiles of the CTA
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem + L.x_off);  // [NT][xstride]
-  float* red = reinterpret_cast<float*>(smem + L.red_off);     // [NT][128]
+  float* red = reinterpret_cast<float*>(smem + L.red_off);     // [KW][NT][128]
   float* cred = reinterpret_cast<float*>(smem + L.cred_off);   // [cl][NT][128], rank 0 only
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
-  const int b = blockIdx.x / cl;
+  const int chunk = blockIdx.x / cl;       // (row block, part of it)
+  const int b = chunk / KW;
+  const int ro = (chunk % KW) * kRows;     // the CTA's first row in the block
   const int crank = blockIdx.x % cl;
   const int ga = (kg * crank) / cl, gb = (kg * (crank + 1)) / cl;
   const int ng = gb - ga;
   const int xstride = gv_xstride(ng);
+  // This warp's tile and its share [gw0, gw0 + ngw) of the CTA's groups.
+  const int tile = warp % kTiles, ks = warp / kTiles;
+  const int gw0 = (ks * ng) / KW;
+  const int ngw = ((ks + 1) * ng) / KW - gw0;
 
   ptx::griddep_launch_dependents();
   if (cl > 1) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
@@ -228,10 +240,11 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   // This lane's rows within the block: MMA rows g and g + 8 of the warp's
   // tile are the adjacent block rows rl and rl + 1.  Its group streams
   // (pointers at group ga; slot offsets are folded into the loads).
-  const int rl = 16 * warp + 2 * g;
-  const uint8_t* pw = wq + (size_t)b * kc_n * kRowBlock * 16 + (size_t)ga * kGvWBytes + c * (kRowBlock * 16) + rl * 16;
-  const uint16_t* ps = s_p + ((size_t)b * kg + ga) * kRowBlock + rl;
-  const uint8_t* pz = z_p + ((size_t)b * kg + ga) * (kRowBlock / 2) + (rl >> 1);
+  const int rl = ro + 16 * tile + 2 * g;
+  const int g0 = ga + gw0;
+  const uint8_t* pw = wq + (size_t)b * kc_n * kRowBlock * 16 + (size_t)g0 * kGvWBytes + c * (kRowBlock * 16) + rl * 16;
+  const uint16_t* ps = s_p + ((size_t)b * kg + g0) * kRowBlock + rl;
+  const uint8_t* pz = z_p + ((size_t)b * kg + g0) * (kRowBlock / 2) + (rl >> 1);
 
   // The activations of this CTA's K range go to shared memory with
   // asynchronous 16-byte copies.  Without programmatic launch they are
@@ -249,7 +262,7 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   // grid dependency wait (which returns at once unless the launch is
   // programmatic); X, written by that kernel, only after it.
   GvFrag f[kGvDepth];
-  gv_load_first<0>(f, ng, pw, ps, pz);
+  gv_load_first<0>(f, ngw, pw, ps, pz);
   ptx::griddep_wait();
   if (early) stage_x();
   asm volatile("cp.async.wait_all;" ::: "memory");
@@ -258,17 +271,17 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   // Lanes of tokens g >= NT read token NT - 1: MMA columns are independent,
   // and those columns are never stored.
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  const uint16_t* xg = xs + (g < NT ? g : NT - 1) * xstride + 32 * c;
+  const uint16_t* xg = xs + (g < NT ? g : NT - 1) * xstride + 32 * c + gw0 * kGroup;
   int i0 = 0;
-  for (; i0 + 2 * kGvDepth <= ng; i0 += kGvDepth) {   // every refill exists
+  for (; i0 + 2 * kGvDepth <= ngw; i0 += kGvDepth) {   // every refill exists
     gv_step_full<0>(f, pw, ps, pz, xg, acc);
     pw += kGvDepth * kGvWBytes;
     ps += kGvDepth * kRowBlock;
     pz += kGvDepth * (kRowBlock / 2);
     xg += kGvDepth * kGroup;
   }
-  for (; i0 < ng; i0 += kGvDepth) {
-    gv_step<0>(f, i0, ng, pw, ps, pz, xg, acc);
+  for (; i0 < ngw; i0 += kGvDepth) {
+    gv_step<0>(f, i0, ngw, pw, ps, pz, xg, acc);
     pw += kGvDepth * kGvWBytes;
     ps += kGvDepth * kRowBlock;
     pz += kGvDepth * (kRowBlock / 2);
@@ -280,31 +293,37 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   for (int e = 0; e < 2; ++e) {
     const int n = 2 * c + e;
     if (n < NT) {
-      red[n * kRowBlock + rl] = acc[e];
-      red[n * kRowBlock + rl + 1] = acc[2 + e];
+      red[(ks * NT + n) * kRowBlock + rl] = acc[e];
+      red[(ks * NT + n) * kRowBlock + rl + 1] = acc[2 + e];
     }
   }
   __syncthreads();
 
   float tot[NT];
-  const int r = threadIdx.x;   // rows for the reduction: threads 0..127
+  const int rr = threadIdx.x;        // the CTA's rows: threads 0 .. kRows - 1
+  const int r = ro + rr;             // row within the block
   // The fused form's destination and bias of row m, loaded before the
   // reductions so the load overlaps them.
   RowDst dst = {};
   if constexpr (kEpi == kEpiQkv) {
     const int m = b * kRowBlock + r;
-    if (r < kRowBlock && crank == 0 && m < M) dst = row_dst(om, M, m);
+    if (rr < kRows && crank == 0 && m < M) dst = row_dst(om, M, m);
   }
-  if (r < kRowBlock) {
+  if (rr < kRows) {
 #pragma unroll
-    for (int n = 0; n < NT; ++n) tot[n] = red[n * kRowBlock + r];
+    for (int n = 0; n < NT; ++n) {
+      float sum = red[n * kRowBlock + r];
+#pragma unroll
+      for (int k = 1; k < KW; ++k) sum += red[(k * NT + n) * kRowBlock + r];   // K halves in order
+      tot[n] = sum;
+    }
   }
 
   if (cl > 1) {
     // Every CTA of the cluster has started once this wait returns, so its
     // shared memory may be written remotely.
     asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-    if (r < kRowBlock) {
+    if (rr < kRows) {
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
         const uint32_t local = ptx::smem_addr(&cred[(crank * NT + n) * kRowBlock + r]);
@@ -315,20 +334,21 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
     }
     asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-    if (crank != 0 || r >= kRowBlock) return;
+    if (crank != 0 || rr >= kRows) return;
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
       float sum = 0.f;
       for (int c = 0; c < cl; ++c) sum += cred[(c * NT + n) * kRowBlock + r];
       tot[n] = sum;
     }
-  } else if (r >= kRowBlock) {
+  } else if (rr >= kRows) {
     return;
   }
 
   const int m = b * kRowBlock + r;
   if constexpr (kEpi == kEpiGateUp) {
-    // Threads 0..127 are whole warps here: the gate/up pairing shuffles.
+    // Threads 0 .. kRows - 1 are whole warps here: the gate/up pairing
+    // shuffles within 32-row groups, which a CTA's rows never split.
 #pragma unroll
     for (int n = 0; n < NT; ++n) store_gate_up(om, b, r, n, tot[n], true);
   } else if (m < M) {
@@ -342,16 +362,17 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   }
 }
 
-template <int NT, int kEpi>
+template <int NT, int kEpi, int KW>
 cudaError_t launch_nt(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p, const uint16_t* X,
                       uint16_t* Y, int M, int K, int cl, bool pdl, cudaStream_t stream, const OutMap& om) {
   static std::atomic<unsigned long long> smem_set{0};
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(gemv_kernel<NT, kEpi>), 128 * 1024, smem_set);
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(gemv_kernel<NT, kEpi, KW>), 128 * 1024,
+                                    smem_set);
   if (e != cudaSuccess) return e;
   const int blocks = ceil_div(M, kRowBlock);
-  const GvLayout L = gv_layout(NT, ceil_div(K / kGroup, cl), cl);
+  const GvLayout L = gv_layout(NT, ceil_div(K / kGroup, cl), cl, KW);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(blocks * cl), 1, 1);
+  cfg.gridDim = dim3((unsigned)(blocks * KW * cl), 1, 1);
   cfg.blockDim = dim3(kGvThreads, 1, 1);
   cfg.dynamicSmemBytes = (size_t)L.total;
   cfg.stream = stream;
@@ -364,38 +385,50 @@ cudaError_t launch_nt(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, gemv_kernel<NT, kEpi>, wq, s_p, z_p, X, Y, M, K, cl, pdl ? 1 : 0, om);
+  return cudaLaunchKernelEx(&cfg, gemv_kernel<NT, kEpi, KW>, wq, s_p, z_p, X, Y, M, K, cl, pdl ? 1 : 0, om);
 }
+
+struct GvShape {
+  int kw, cl;
+};
 
 }  // namespace
 
-// Cluster size along K (1..8), from the measured LLaMA-7B N = 1 shapes:
-// all CTAs resident in one wave (kGvCtasPerSm per SM, set by the registers
-// of one CTA), and at least 2.5 CTAs per SM on average when the shape
-// allows it (fewer warps per SM hide the shared-memory and FMA latencies
-// badly); among those the smallest busiest-SM share of groups,
-// ceil(CTAs / SMs) x ceil(groups / cluster), then the smaller cluster.  When
-// no cluster reaches 2.5 CTAs per SM, the most CTAs.  The staged activation
-// slice must fit.
-int gemv_cluster_size(int M, int K, int sms, int nt) {
+// Row split KW (1 or 2 CTAs per 128-row block, see gemv_kernel) and cluster
+// size along K (1..8), from the measured LLaMA N = 1 shapes: all CTAs
+// resident in one wave (kGvCtasPerSm per SM, set by the registers of one
+// CTA), and at least 2.5 CTAs per SM on average when the shape allows it
+// (fewer warps per SM hide the load and MMA latencies badly); among those
+// the smallest busiest-SM work, ceil(CTAs / SMs) x the groups of one warp,
+// then the smaller KW, then the smaller cluster.  When no choice reaches 2.5
+// CTAs per SM, the most CTAs.  The staged activation slice must fit.
+GvShape gemv_shape(int M, int K, int sms, int nt) {
   const int blocks = ceil_div(M, kRowBlock);
   const int kg = K / kGroup;
-  int best = 0;
-  long long best_key[3] = {0, 0, 0};
-  for (int cl = 1; cl <= kMaxCluster && cl <= kg; ++cl) {
-    if (nt * gv_xstride(ceil_div(kg, cl)) * 2 > kMaxXSmem) continue;
-    const long long ctas = (long long)blocks * cl;
-    if (cl > 1 && ctas > (long long)kGvCtasPerSm * sms) continue;
-    const bool dense = 2 * ctas >= 5LL * sms;
-    const long long load = (long long)ceil_div((int)ctas, sms) * ceil_div(kg, cl);
-    const long long key[3] = {dense ? 0 : 1, dense ? load : -ctas, cl};
-    if (best == 0 || key[0] < best_key[0] || (key[0] == best_key[0] && (key[1] < best_key[1] ||
-        (key[1] == best_key[1] && key[2] < best_key[2])))) {
-      best = cl;
-      for (int i = 0; i < 3; ++i) best_key[i] = key[i];
+  GvShape best = {0, 0};
+  long long best_key[4] = {0, 0, 0, 0};
+  for (int kw = 1; kw <= 2; ++kw) {
+    for (int cl = 1; cl <= kMaxCluster && cl <= kg; ++cl) {
+      if (nt * gv_xstride(ceil_div(kg, cl)) * 2 > kMaxXSmem) continue;
+      const long long ctas = (long long)blocks * kw * cl;
+      if ((kw > 1 || cl > 1) && ctas > (long long)kGvCtasPerSm * sms) continue;
+      const bool dense = 2 * ctas >= 5LL * sms;
+      const long long load = (long long)ceil_div((int)ctas, sms) * ceil_div(ceil_div(kg, cl), kw);
+      const long long key[4] = {dense ? 0 : 1, dense ? load : -ctas, kw, cl};
+      bool better = best.cl == 0;
+      for (int i = 0; i < 4 && !better; ++i) {
+        if (key[i] != best_key[i]) {
+          better = key[i] < best_key[i];
+          break;
+        }
+      }
+      if (better) {
+        best = {kw, cl};
+        for (int i = 0; i < 4; ++i) best_key[i] = key[i];
+      }
     }
   }
-  return best > 0 ? best : kMaxCluster;
+  return best.cl > 0 ? best : GvShape{1, kMaxCluster};
 }
 
 cudaError_t launch_gemv(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros,
@@ -403,7 +436,8 @@ cudaError_t launch_gemv(const uint8_t* wq, const uint16_t* scales, const uint8_t
                         cudaStream_t stream, const OutMap* om, bool pdl) {
   for (int n0 = 0; n0 < N; n0 += kGemvMaxTokens) {
     const int nt = std::min(kGemvMaxTokens, N - n0);
-    const int cl = gemv_cluster_size(M, K, num_sms(), nt);
+    const GvShape sh = gemv_shape(M, K, num_sms(), nt);
+    const int cl = sh.cl;
     if (nt * gv_xstride(ceil_div(K / kGroup, cl)) * 2 > kMaxXSmem) return cudaErrorNotSupported;
     const uint16_t* Xn = X + (size_t)n0 * K;
     uint16_t* Yn = om ? nullptr : Y + (size_t)n0 * M;
@@ -422,17 +456,8 @@ cudaError_t launch_gemv(const uint8_t* wq, const uint16_t* scales, const uint8_t
     }
     const int kind = om ? om->kind : kEpiPlain;
     cudaError_t e;
-#define W4A16_GEMV_NT(EPI)                                                                          \
-    switch (nt) {                                                                                     \
-      case 1: e = launch_nt<1, EPI>(wq, scales, zeros, Xn, Yn, M, K, cl, pdl, stream, on); break;          \
-      case 2: e = launch_nt<2, EPI>(wq, scales, zeros, Xn, Yn, M, K, cl, pdl, stream, on); break;          \
-      case 3: e = launch_nt<3, EPI>(wq, scales, zeros, Xn, Yn, M, K, cl, pdl, stream, on); break;          \
-      case 4: e = launch_nt<4, EPI>(wq, scales, zeros, Xn, Yn, M, K, cl, pdl, stream, on); break;          \
-      case 5: e = launch_nt<5, EPI>(wq, scales, zeros, Xn, Yn, M, K, cl, pdl, stream, on); break;          \
-      case 6: e = launch_nt<6, EPI>(wq, scales, zeros, Xn, Yn, M, K, cl, pdl, stream, on); break;          \
-      case 7: e = launch_nt<7, EPI>(wq, scales, zeros, Xn, Yn, M, K, cl, pdl, stream, on); break;          \
-      default: e = launch_nt<8, EPI>(wq, scales, zeros, Xn, Yn, M, K, cl, pdl, stream, on); break;         \
-    }
+#define W4A16_GEMV_KW(NT, EPI)                                                                           e = sh.kw == 2 ? launch_nt<NT, EPI, 2>(wq, scales, zeros, Xn, Yn, M, K, cl, pdl, stream, on)                        : launch_nt<NT, EPI, 1>(wq, scales, zeros, Xn, Yn, M, K, cl, pdl, stream, on)
+#define W4A16_GEMV_NT(EPI)                                                                              switch (nt) {                                                                                           case 1: W4A16_GEMV_KW(1, EPI); break;                                                                 case 2: W4A16_GEMV_KW(2, EPI); break;                                                                 case 3: W4A16_GEMV_KW(3, EPI); break;                                                                 case 4: W4A16_GEMV_KW(4, EPI); break;                                                                 case 5: W4A16_GEMV_KW(5, EPI); break;                                                                 case 6: W4A16_GEMV_KW(6, EPI); break;                                                                 case 7: W4A16_GEMV_KW(7, EPI); break;                                                                 default: W4A16_GEMV_KW(8, EPI); break;                                                              }
     if (kind == kEpiGateUp) {
       W4A16_GEMV_NT(kEpiGateUp)
     } else if (kind == kEpiQkv) {
@@ -441,6 +466,7 @@ cudaError_t launch_gemv(const uint8_t* wq, const uint16_t* scales, const uint8_t
       W4A16_GEMV_NT(kEpiPlain)
     }
 #undef W4A16_GEMV_NT
+#undef W4A16_GEMV_KW
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
