@@ -400,7 +400,8 @@ struct GvShape {
 // CTA), and at least 2.5 CTAs per SM on average when the shape allows it
 // (fewer warps per SM hide the load and MMA latencies badly); among those
 // the smallest busiest-SM work, ceil(CTAs / SMs) x the groups of one warp,
-// then the smaller KW, then the smaller cluster.  When no choice reaches 2.5
+// then the larger KW (measured: gate/up 15.7 against 16.3 us at equal CTA
+// counts), then the smaller cluster.  When no choice reaches 2.5
 // CTAs per SM, the most CTAs.  The staged activation slice must fit.
 GvShape gemv_shape(int M, int K, int sms, int nt) {
   const int blocks = ceil_div(M, kRowBlock);
@@ -414,7 +415,7 @@ GvShape gemv_shape(int M, int K, int sms, int nt) {
       if ((kw > 1 || cl > 1) && ctas > (long long)kGvCtasPerSm * sms) continue;
       const bool dense = 2 * ctas >= 5LL * sms;
       const long long load = (long long)ceil_div((int)ctas, sms) * ceil_div(ceil_div(kg, cl), kw);
-      const long long key[4] = {dense ? 0 : 1, dense ? load : -ctas, kw, cl};
+      const long long key[4] = {dense ? 0 : 1, dense ? load : -ctas, -kw, cl};
       bool better = best.cl == 0;
       for (int i = 0; i < 4 && !better; ++i) {
         if (key[i] != best_key[i]) {
