@@ -428,6 +428,8 @@ def main_ours(args):
         return single_shape(args, device, args.M, args.K, args.N, args.path)
     if args.workload == "quantize":
         return quantize_workload(args, device, peaks)
+    if args.workload == "qkv_norm":
+        return qkv_norm_workload(args, device, peaks)
     if args.workload == "qkv_fused":
         return qkv_fused_workload(args, device, peaks)
     if args.workload == "gate_up_fused":
@@ -688,6 +690,63 @@ def llama3_measure(device, peaks, sampler, reps=20):
     t1 = time.time()
     return {"columns": ["shape", "N", "path", "us", "GBps", "roof_frac"], "rows": rows,
             "clocks": sampler.summary(t0, t1)}
+
+
+def qkv_norm_workload(args, device, peaks):
+    """Residual add + RMS norm + fused QKV projection of LLaMA-7B at N = 1
+    (h, d [1, 4096]; weight 12288 x 4096 as (4096, 4096, 4096); 8 rotated
+    weight copies, beyond L2), two arms, each a CUDA graph:
+      chain  w4a16_add_rmsnorm (X and r to memory), then w4a16_gemm_qkv_ws
+             with early weights (its weight stream overlaps the norm kernel);
+      fused  w4a16_add_rmsnorm_gemm_qkv with early weights (X never stored).
+    Microseconds per (norm + projection) pair, three passes of alternating
+    order, median clock per pass."""
+    import torch
+
+    from gemm_w4a16_b200 import w4a16
+
+    M, K, N, splits = 12288, 4096, 1, (4096, 4096, 4096)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(31)
+    gamma = (1.0 + 0.1 * torch.randn(K, device=device, generator=gen)).half()
+    sets = []
+    for c in range(8):
+        w, _ = make_device_problem(device, M, K, N, seed=60 + c)
+        h = torch.randn((N, K), device=device, generator=gen).half()
+        d = torch.randn((N, K), device=device, generator=gen).half()
+        outs = tuple(torch.empty((N, m), dtype=torch.float16, device=device) for m in splits)
+        sets.append((w, h, d, torch.empty_like(h), torch.empty_like(h), outs))
+    ws = w4a16.Workspace(device, w4a16.workspace_size(M, K, N))
+    fl = w4a16.FLAG_EARLY_WEIGHTS
+
+    def chain():
+        for w, h, d, r, X, outs in sets:
+            w4a16.add_rmsnorm(h, gamma, eps=1e-6, d=d, r_out=r, X=X)
+            w4a16.gemm_qkv_ws(w, X, splits, out=outs, workspace=ws, flags=fl)
+
+    def fused():
+        for w, h, d, r, X, outs in sets:
+            w4a16.add_rmsnorm_gemm_qkv(h, gamma, w, splits, eps=1e-6, d=d, r_out=r, out=outs, flags=fl)
+
+    arms = {"chain": chain, "fused": fused}
+    graphs = {name: capture(fn, device) for name, fn in arms.items()}
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    time.sleep(0.2)
+    runs = {name: [] for name in arms}
+    for order in (list(arms), list(arms)[::-1], list(arms)):
+        for name in order:
+            t0 = time.time()
+            us = time_graph(graphs[name], args.steps, args.warmup, device) * 1e3 / len(sets)
+            runs[name].append((us, sampler.summary(t0, time.time())))
+    sampler.stop()
+    for name in arms:
+        us = [u for u, _ in runs[name]]
+        print(json.dumps({"workload": f"add_rmsnorm + qkv {name} M={M} K={K} N={N}",
+                          "us": sum(us) / len(us), "us_each": us,
+                          "sm_mhz_each": [c["sm_mhz"] for _, c in runs[name]],
+                          "reasons": sorted({r for _, c in runs[name] for r in c["reasons"]})}), flush=True)
+    return 0
 
 
 def qkv_fused_workload(args, device, peaks):
@@ -980,7 +1039,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["decode", "qkv_n1", "prefill", "sweep", "shape", "quantize",
-                                           "qkv_fused", "gate_up_fused", "add_rmsnorm"],
+                                           "qkv_fused", "gate_up_fused", "add_rmsnorm", "qkv_norm"],
                     default="decode")
     ap.add_argument("--M", type=int, default=12288)
     ap.add_argument("--K", type=int, default=4096)

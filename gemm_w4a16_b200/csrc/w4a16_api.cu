@@ -410,6 +410,57 @@ w4a16_status w4a16_gemm_qkv(const void* wq_packed, const void* scales_packed, co
                        nullptr, 0, 0u, stream);
 }
 
+w4a16_status w4a16_add_rmsnorm_gemm_qkv(const uint16_t* h, const uint16_t* d, const uint16_t* gamma, float eps,
+                                        uint16_t* r_out, const void* wq_packed, const void* scales_packed,
+                                        const void* zeros_packed, const uint16_t* bias, int Mq, int Mk, int Mv,
+                                        int K, int N, int group, uint16_t* Yq, uint16_t* Yk, uint16_t* Yv,
+                                        unsigned flags, void* stream) {
+  if (!h || !gamma || !wq_packed || !scales_packed || !zeros_packed || !Yq || !Yk || !Yv)
+    return W4A16_ERR_INVALID_ARG;
+  if (Mq <= 0 || Mk <= 0 || Mv <= 0 || N <= 0 || !(eps >= 0.0f) || !(eps <= 3.4028234663852886e38f))
+    return W4A16_ERR_INVALID_ARG;
+  if (flags & ~W4A16_FLAG_EARLY_WEIGHTS) return W4A16_ERR_INVALID_ARG;
+  if ((long long)Mq + Mk + Mv > kMaxM) return W4A16_ERR_UNSUPPORTED;
+  const int M = Mq + Mk + Mv;
+  w4a16_status st = check_shape(M, K, group);
+  if (st != W4A16_OK) return st;
+  if (N > kGemvMaxTokens) return W4A16_ERR_UNSUPPORTED;
+  if (!aligned16(h) || (d && !aligned16(d)) || !aligned16(gamma) || (r_out && !aligned16(r_out)) ||
+      !aligned16(wq_packed) || !aligned16(scales_packed) || !aligned16(zeros_packed) || !aligned16(Yq) ||
+      !aligned16(Yk) || !aligned16(Yv) || (reinterpret_cast<uintptr_t>(bias) & 1u))
+    return W4A16_ERR_MISALIGNED;
+  {
+    // Outputs (Yq, Yk, Yv, r_out) share no byte with an input or with each
+    // other; r_out may not be h or d here (every CTA reads whole rows of h
+    // and d while the first row block's CTAs write r).
+    const PackedBytes pb = packed_bytes(M, K);
+    const size_t nk = (size_t)N * K * 2;
+    const void* outs[4] = {Yq, Yk, Yv, r_out};
+    const size_t out_n[4] = {(size_t)N * Mq * 2, (size_t)N * Mk * 2, (size_t)N * Mv * 2, r_out ? nk : 0};
+    for (int i = 0; i < 4; ++i) {
+      if (overlap(outs[i], out_n[i], h, nk) || overlap(outs[i], out_n[i], d, nk) ||
+          overlap(outs[i], out_n[i], gamma, (size_t)K * 2) || overlap(outs[i], out_n[i], bias, (size_t)M * 2) ||
+          overlaps_weight(outs[i], out_n[i], wq_packed, scales_packed, zeros_packed, pb))
+        return W4A16_ERR_INVALID_ARG;
+      for (int j = i + 1; j < 4; ++j)
+        if (overlap(outs[i], out_n[i], outs[j], out_n[j])) return W4A16_ERR_INVALID_ARG;
+    }
+  }
+  OutMap om = {};
+  om.kind = kEpiQkv;
+  om.y0 = Yq;
+  om.y1 = Yk;
+  om.y2 = Yv;
+  om.end0 = Mq;
+  om.end1 = Mq + Mk;
+  om.bias = bias;
+  const NormIn nin = {h, d, gamma, eps, r_out};
+  return map_cuda(launch_gemv(static_cast<const uint8_t*>(wq_packed), static_cast<const uint16_t*>(scales_packed),
+                              static_cast<const uint8_t*>(zeros_packed), nullptr, nullptr, M, K, N,
+                              static_cast<cudaStream_t>(stream), &om, (flags & W4A16_FLAG_EARLY_WEIGHTS) != 0,
+                              &nin));
+}
+
 w4a16_status w4a16_gemm_qkv_ws(const void* wq_packed, const void* scales_packed, const void* zeros_packed,
                                const uint16_t* X, const uint16_t* bias, int Mq, int Mk, int Mv, int K, int N,
                                int group, uint16_t* Yq, uint16_t* Yk, uint16_t* Yv, void* workspace,

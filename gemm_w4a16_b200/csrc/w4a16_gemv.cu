@@ -199,15 +199,88 @@ __device__ __forceinline__ void gv_step(GvFrag (&f)[kGvDepth], int i0, int ng, c
   }
 }
 
+// The normalising prologue (w4a16_add_rmsnorm_gemm_qkv): X of the CTA's K
+// range computed from the residual stream instead of read.  Each token row's
+// sum of squares is formed over the whole row with exactly the thread
+// mapping, chunk order and fixed-order reduction of add_rmsnorm_kernel (same
+// thread count), so inv, X and r are bit-identical to that kernel's; then
+// r = h + d, X = (r * inv) * gamma for the CTA's groups go to shared memory,
+// and the CTAs of the first row block also write r for their K range.
+template <int NT>
+__device__ __forceinline__ void gv_norm_x(const NormIn& nin, int K, int ga, int ng, uint16_t* xs, int xstride,
+                                          bool write_r) {
+  static_assert(kGvThreads == kNormThreads, "the sum of squares must follow the norm kernel's order");
+  __shared__ float wsum[kNormThreads / 32];
+  __shared__ float s_inv[kGemvMaxTokens];
+  const int chunks = K / 8;
+#pragma unroll 1
+  for (int n = 0; n < NT; ++n) {
+    const uint4* hv = reinterpret_cast<const uint4*>(nin.h) + (size_t)n * chunks;
+    const uint4* dv = nin.d ? reinterpret_cast<const uint4*>(nin.d) + (size_t)n * chunks : nullptr;
+    // The norm kernel's per-thread order: chunks threadIdx.x, + 256, ...
+    // (its batching of the loads does not change the order of the sum).
+    float ss = 0.0f;
+    for (int c = threadIdx.x; c < chunks; c += kNormThreads) {
+      uint4 r = hv[c];
+      if (dv) {
+        const uint4 b = dv[c];
+        r.x = hadd2_rn(r.x, b.x);
+        r.y = hadd2_rn(r.y, b.y);
+        r.z = hadd2_rn(r.z, b.z);
+        r.w = hadd2_rn(r.w, b.w);
+      }
+      ss = sum_sq2(r.x, ss);
+      ss = sum_sq2(r.y, ss);
+      ss = sum_sq2(r.z, ss);
+      ss = sum_sq2(r.w, ss);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if ((threadIdx.x & 31) == 0) wsum[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float tot = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kNormThreads / 32; ++w) tot += wsum[w];
+      s_inv[n] = rms_inv(tot, K, nin.eps);
+    }
+    __syncthreads();
+  }
+  const uint4* gv = reinterpret_cast<const uint4*>(nin.gamma);
+  const int pieces = ng * (kGroup / 8);
+  for (int idx = threadIdx.x; idx < NT * pieces; idx += kGvThreads) {
+    const int n = idx / pieces, p = idx - n * pieces;
+    const size_t c = (size_t)n * chunks + (size_t)ga * (kGroup / 8) + p;
+    const uint4 a = reinterpret_cast<const uint4*>(nin.h)[c];
+    uint4 r = a;
+    if (nin.d) {
+      const uint4 b = reinterpret_cast<const uint4*>(nin.d)[c];
+      r.x = hadd2_rn(a.x, b.x);
+      r.y = hadd2_rn(a.y, b.y);
+      r.z = hadd2_rn(a.z, b.z);
+      r.w = hadd2_rn(a.w, b.w);
+    }
+    if (write_r && nin.r_out) reinterpret_cast<uint4*>(nin.r_out)[c] = r;
+    const uint4 g = gv[ga * (kGroup / 8) + p];
+    const float inv = s_inv[n];
+    uint4 o;
+    o.x = scale2(r.x, g.x, inv);
+    o.y = scale2(r.y, g.y, inv);
+    o.z = scale2(r.z, g.z, inv);
+    o.w = scale2(r.w, g.w, inv);
+    *reinterpret_cast<uint4*>(xs + n * xstride + p * 8) = o;
+  }
+}
+
 // KW = 1: the CTA's 8 warps are the 8 row tiles of a 128-row block; KW = 2:
 // 4 row tiles (half a block) with two warps each, which take the two halves
 // of the CTA's K range and meet in shared memory (more warps per row for
 // shapes with few row blocks).
-template <int NT, int kEpi, int KW>
+template <int NT, int kEpi, int KW, bool kNorm>
 __global__ void __launch_bounds__(kGvThreads, kGvCtasPerSm)
 gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
             const uint8_t* __restrict__ z_p, const uint16_t* __restrict__ X,
-            uint16_t* __restrict__ Y, int M, int K, int cl, int early, OutMap om) {
+            uint16_t* __restrict__ Y, int M, int K, int cl, int early, OutMap om, NormIn nin) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int kg = K / kGroup;
   const int kc_n = K / kChunkK;
@@ -257,14 +330,18 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
-  if (!early) stage_x();
+  if (!early && !kNorm) stage_x();
   // The first groups depend on no earlier kernel: request them before the
   // grid dependency wait (which returns at once unless the launch is
-  // programmatic); X, written by that kernel, only after it.
+  // programmatic); X (or the residual stream it comes from), written by that
+  // kernel, only after it.
   GvFrag f[kGvDepth];
   gv_load_first<0>(f, ngw, pw, ps, pz);
   ptx::griddep_wait();
-  if (early) stage_x();
+  if constexpr (kNorm)
+    gv_norm_x<NT>(nin, K, ga, ng, xs, xstride, chunk == 0);
+  else if (early)
+    stage_x();
   asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
 
@@ -362,11 +439,12 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   }
 }
 
-template <int NT, int kEpi, int KW>
+template <int NT, int kEpi, int KW, bool kNorm = false>
 cudaError_t launch_nt(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p, const uint16_t* X,
-                      uint16_t* Y, int M, int K, int cl, bool pdl, cudaStream_t stream, const OutMap& om) {
+                      uint16_t* Y, int M, int K, int cl, bool pdl, cudaStream_t stream, const OutMap& om,
+                      const NormIn& nin) {
   static std::atomic<unsigned long long> smem_set{0};
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(gemv_kernel<NT, kEpi, KW>), 128 * 1024,
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(gemv_kernel<NT, kEpi, KW, kNorm>), 128 * 1024,
                                     smem_set);
   if (e != cudaSuccess) return e;
   const int blocks = ceil_div(M, kRowBlock);
@@ -385,7 +463,34 @@ cudaError_t launch_nt(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, gemv_kernel<NT, kEpi, KW>, wq, s_p, z_p, X, Y, M, K, cl, pdl ? 1 : 0, om);
+  return cudaLaunchKernelEx(&cfg, gemv_kernel<NT, kEpi, KW, kNorm>, wq, s_p, z_p, X, Y, M, K, cl, pdl ? 1 : 0, om,
+                            nin);
+}
+
+// One launch of nt tokens (1..8) with row split kw (1 or 2).
+template <int kEpi, bool kNorm = false>
+cudaError_t launch_epi(int nt, int kw, const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p,
+                       const uint16_t* X, uint16_t* Y, int M, int K, int cl, bool pdl, cudaStream_t stream,
+                       const OutMap& om, const NormIn& nin) {
+  const bool two = kw == 2;
+  switch (nt) {
+    case 1: return two ? launch_nt<1, kEpi, 2, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin)
+                       : launch_nt<1, kEpi, 1, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
+    case 2: return two ? launch_nt<2, kEpi, 2, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin)
+                       : launch_nt<2, kEpi, 1, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
+    case 3: return two ? launch_nt<3, kEpi, 2, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin)
+                       : launch_nt<3, kEpi, 1, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
+    case 4: return two ? launch_nt<4, kEpi, 2, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin)
+                       : launch_nt<4, kEpi, 1, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
+    case 5: return two ? launch_nt<5, kEpi, 2, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin)
+                       : launch_nt<5, kEpi, 1, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
+    case 6: return two ? launch_nt<6, kEpi, 2, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin)
+                       : launch_nt<6, kEpi, 1, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
+    case 7: return two ? launch_nt<7, kEpi, 2, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin)
+                       : launch_nt<7, kEpi, 1, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
+    default: return two ? launch_nt<8, kEpi, 2, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin)
+                        : launch_nt<8, kEpi, 1, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
+  }
 }
 
 struct GvShape {
@@ -434,13 +539,15 @@ GvShape gemv_shape(int M, int K, int sms, int nt) {
 
 cudaError_t launch_gemv(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros,
                         const uint16_t* X, uint16_t* Y, int M, int K, int N,
-                        cudaStream_t stream, const OutMap* om, bool pdl) {
+                        cudaStream_t stream, const OutMap* om, bool pdl, const NormIn* norm) {
+  if (norm && (N > kGemvMaxTokens || !om || om->kind != kEpiQkv)) return cudaErrorNotSupported;
+  const NormIn nin = norm ? *norm : NormIn{};
   for (int n0 = 0; n0 < N; n0 += kGemvMaxTokens) {
     const int nt = std::min(kGemvMaxTokens, N - n0);
     const GvShape sh = gemv_shape(M, K, num_sms(), nt);
     const int cl = sh.cl;
     if (nt * gv_xstride(ceil_div(K / kGroup, cl)) * 2 > kMaxXSmem) return cudaErrorNotSupported;
-    const uint16_t* Xn = X + (size_t)n0 * K;
+    const uint16_t* Xn = X ? X + (size_t)n0 * K : nullptr;
     uint16_t* Yn = om ? nullptr : Y + (size_t)n0 * M;
     // The fused outputs of tokens n0 .. n0 + nt - 1: each segment moves by
     // n0 of its own rows.
@@ -457,17 +564,14 @@ cudaError_t launch_gemv(const uint8_t* wq, const uint16_t* scales, const uint8_t
     }
     const int kind = om ? om->kind : kEpiPlain;
     cudaError_t e;
-#define W4A16_GEMV_KW(NT, EPI)                                                                           e = sh.kw == 2 ? launch_nt<NT, EPI, 2>(wq, scales, zeros, Xn, Yn, M, K, cl, pdl, stream, on)                        : launch_nt<NT, EPI, 1>(wq, scales, zeros, Xn, Yn, M, K, cl, pdl, stream, on)
-#define W4A16_GEMV_NT(EPI)                                                                              switch (nt) {                                                                                           case 1: W4A16_GEMV_KW(1, EPI); break;                                                                 case 2: W4A16_GEMV_KW(2, EPI); break;                                                                 case 3: W4A16_GEMV_KW(3, EPI); break;                                                                 case 4: W4A16_GEMV_KW(4, EPI); break;                                                                 case 5: W4A16_GEMV_KW(5, EPI); break;                                                                 case 6: W4A16_GEMV_KW(6, EPI); break;                                                                 case 7: W4A16_GEMV_KW(7, EPI); break;                                                                 default: W4A16_GEMV_KW(8, EPI); break;                                                              }
-    if (kind == kEpiGateUp) {
-      W4A16_GEMV_NT(kEpiGateUp)
-    } else if (kind == kEpiQkv) {
-      W4A16_GEMV_NT(kEpiQkv)
-    } else {
-      W4A16_GEMV_NT(kEpiPlain)
-    }
-#undef W4A16_GEMV_NT
-#undef W4A16_GEMV_KW
+    if (norm)
+      e = launch_epi<kEpiQkv, true>(nt, sh.kw, wq, scales, zeros, Xn, Yn, M, K, cl, pdl, stream, on, nin);
+    else if (kind == kEpiGateUp)
+      e = launch_epi<kEpiGateUp>(nt, sh.kw, wq, scales, zeros, Xn, Yn, M, K, cl, pdl, stream, on, nin);
+    else if (kind == kEpiQkv)
+      e = launch_epi<kEpiQkv>(nt, sh.kw, wq, scales, zeros, Xn, Yn, M, K, cl, pdl, stream, on, nin);
+    else
+      e = launch_epi<kEpiPlain>(nt, sh.kw, wq, scales, zeros, Xn, Yn, M, K, cl, pdl, stream, on, nin);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

@@ -102,6 +102,59 @@ __device__ __forceinline__ uint32_t zero_code(const uint8_t* zblock, int r) {
   return (zblock[r >> 1] >> ((r & 1) * 4)) & 0xFu;
 }
 
+// ----------------------------------------------- add + RMS normalisation ----
+
+// The arithmetic of the residual add + RMS normalisation, shared by its own
+// kernel and by the decode kernel's normalising prologue so that both give
+// the same bits: r = fp16_RN(h + d) pairwise, the sum of squares of r in
+// fp32 with one fma per channel in channel order, X = fp16_RN((r * inv) * g).
+__device__ __forceinline__ uint32_t hadd2_rn(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+__device__ __forceinline__ float lo_f(uint32_t w) {
+  return __half2float(__ushort_as_half((unsigned short)(w & 0xFFFFu)));
+}
+
+__device__ __forceinline__ float hi_f(uint32_t w) {
+  return __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+}
+
+__device__ __forceinline__ float sum_sq2(uint32_t w, float ss) {
+  const float a = lo_f(w), b = hi_f(w);
+  return fmaf(b, b, fmaf(a, a, ss));
+}
+
+// Two channels of X from two of r and two of gamma.
+__device__ __forceinline__ uint32_t scale2(uint32_t r, uint32_t g, float inv) {
+  const float x0 = __fmul_rn(__fmul_rn(lo_f(r), inv), lo_f(g));
+  const float x1 = __fmul_rn(__fmul_rn(hi_f(r), inv), hi_f(g));
+  return (uint32_t)__half_as_ushort(__float2half_rn(x0)) |
+         ((uint32_t)__half_as_ushort(__float2half_rn(x1)) << 16);
+}
+
+// 1 / sqrt(mean + eps) from the fixed-order sum of squares of a row.
+__device__ __forceinline__ float rms_inv(float sum_sq, int K, float eps) {
+  return __frsqrt_rn(__fadd_rn(__fdiv_rn(sum_sq, (float)K), eps));
+}
+
+// Threads per row and 16-byte chunks in flight per thread of the sum of
+// squares (its order depends on both).
+constexpr int kNormThreads = 256;
+constexpr int kNormBatch = 4;
+
+// Inputs of the decode kernel's normalising prologue (h null: none; the
+// kernel then reads X).  r_out may be null.
+struct NormIn {
+  const uint16_t* h;
+  const uint16_t* d;
+  const uint16_t* gamma;
+  float eps;
+  uint16_t* r_out;
+};
+
 // ------------------------------------------------------ gate/up rows ----
 
 // The gate/up row order of w4a16_pack_gate_up: packed block b holds the 64
@@ -226,9 +279,11 @@ constexpr int kGemvMaxTokens = 8;
 // With pdl the launch may overlap the previous kernel in the stream: the
 // first weight stages are read before the grid dependency wait, X and Y
 // after it.
+// norm: the normalising prologue (X unused; N <= kGemvMaxTokens).
 cudaError_t launch_gemv(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros,
                         const uint16_t* X, uint16_t* Y, int M, int K, int N,
-                        cudaStream_t stream, const OutMap* om = nullptr, bool pdl = false);
+                        cudaStream_t stream, const OutMap* om = nullptr, bool pdl = false,
+                        const NormIn* norm = nullptr);
 
 // Residual add + RMS normalisation: one CTA per token row, K a multiple of 8
 // and at most kMaxNormK (the row's residual is held in shared memory).

@@ -29,35 +29,6 @@ namespace w4a16 {
 
 namespace {
 
-constexpr int kNormThreads = 256;
-constexpr int kNormBatch = 4;   // 16-byte chunks per thread in flight in pass 1
-
-__device__ __forceinline__ uint32_t hadd2_rn(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
-
-__device__ __forceinline__ float lo_f(uint32_t w) {
-  return __half2float(__ushort_as_half((unsigned short)(w & 0xFFFFu)));
-}
-
-__device__ __forceinline__ float hi_f(uint32_t w) {
-  return __half2float(__ushort_as_half((unsigned short)(w >> 16)));
-}
-
-__device__ __forceinline__ float sum_sq2(uint32_t w, float ss) {
-  const float a = lo_f(w), b = hi_f(w);
-  return fmaf(b, b, fmaf(a, a, ss));
-}
-
-// Two channels of X from two of r and two of gamma.
-__device__ __forceinline__ uint32_t scale2(uint32_t r, uint32_t g, float inv) {
-  const float x0 = __fmul_rn(__fmul_rn(lo_f(r), inv), lo_f(g));
-  const float x1 = __fmul_rn(__fmul_rn(hi_f(r), inv), hi_f(g));
-  return (uint32_t)__half_as_ushort(__float2half_rn(x0)) |
-         ((uint32_t)__half_as_ushort(__float2half_rn(x1)) << 16);
-}
 
 // h, d and r_out may be the same memory as each other (r_out == h or d: each
 // element is read before the same thread writes it); X overlaps none of them.
@@ -116,7 +87,7 @@ add_rmsnorm_kernel(const uint16_t* h, const uint16_t* d, const uint16_t* __restr
   float tot = 0.0f;
 #pragma unroll
   for (int w = 0; w < kNormThreads / 32; ++w) tot += wsum[w];
-  const float inv = __frsqrt_rn(__fadd_rn(__fdiv_rn(tot, (float)K), eps));
+  const float inv = rms_inv(tot, K, eps);
 
   const uint4* gv = reinterpret_cast<const uint4*>(gamma);
   uint4* xv = reinterpret_cast<uint4*>(X) + base;

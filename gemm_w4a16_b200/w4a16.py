@@ -27,7 +27,7 @@ EXPORTED = (
     "w4a16_device_status", "w4a16_selftest_wait_timeout", "w4a16_quantize", "w4a16_gemm_qkv",
     "w4a16_add_rmsnorm", "w4a16_gemm_workspace_size", "w4a16_gemm_ws", "w4a16_gemm_qkv_ws",
     "w4a16_select_path_ws", "w4a16_pack_gate_up", "w4a16_gemm_gate_up", "w4a16_gemm_gate_up_ws",
-    "w4a16_gemm_noalloc",
+    "w4a16_gemm_noalloc", "w4a16_add_rmsnorm_gemm_qkv",
 )
 
 _lib = None
@@ -68,6 +68,9 @@ def lib():
             L.w4a16_gemm.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]
             L.w4a16_gemm.restype = _i
             L.w4a16_gemm_qkv.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp]
+            L.w4a16_add_rmsnorm_gemm_qkv.argtypes = [_vp, _vp, _vp, ctypes.c_float, _vp, _vp, _vp, _vp, _vp,
+                                                     _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _u, _vp]
+            L.w4a16_add_rmsnorm_gemm_qkv.restype = _i
             L.w4a16_gemm_qkv.restype = _i
             L.w4a16_gemm_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
             L.w4a16_gemm_ex.restype = _i
@@ -377,6 +380,30 @@ def gemm_qkv(w: PackedWeight, X, splits, bias=None, out=None, stream=None):
     _check(lib().w4a16_gemm_qkv(_ptr(w.wq), _ptr(w.scales), _ptr(w.zeros), _ptr(X), _ptr(bias), Mq, Mk, Mv,
                                 K, N, w.group, _ptr(outs[0]), _ptr(outs[1]), _ptr(outs[2]),
                                 _stream_ptr(stream)), "w4a16_gemm_qkv")
+    return tuple(outs)
+
+
+def add_rmsnorm_gemm_qkv(h, gamma, w: PackedWeight, splits, eps: float = 1e-6, d=None, r_out=None, bias=None,
+                         out=None, flags: int = 0, stream=None):
+    """gemm_qkv of the normalised residual stream in one launch, via
+    w4a16_add_rmsnorm_gemm_qkv (N <= GEMV_MAX_TOKENS): X = add_rmsnorm(h, d)
+    is formed inside the projection and never stored; r = h + d goes to r_out
+    when given.  Returns (Yq, Yk, Yv)."""
+    import torch
+
+    N, K = h.shape
+    outs = _qkv_outs(w, h, splits, bias, out)
+    if gamma.dtype != torch.float16 or not gamma.is_cuda or not gamma.is_contiguous() or gamma.numel() != K:
+        raise ValueError("gamma must be a contiguous CUDA fp16 tensor of K values")
+    for name, t in (("d", d), ("r_out", r_out)):
+        if t is not None and (t.dtype != torch.float16 or not t.is_cuda or not t.is_contiguous()
+                              or tuple(t.shape) != (N, K)):
+            raise ValueError(f"{name} must be a contiguous CUDA fp16 [N, K] tensor")
+    Mq, Mk, Mv = (int(v) for v in splits)
+    _check(lib().w4a16_add_rmsnorm_gemm_qkv(_ptr(h), _ptr(d), _ptr(gamma), float(eps), _ptr(r_out), _ptr(w.wq),
+                                            _ptr(w.scales), _ptr(w.zeros), _ptr(bias), Mq, Mk, Mv, K, N, w.group,
+                                            _ptr(outs[0]), _ptr(outs[1]), _ptr(outs[2]), int(flags),
+                                            _stream_ptr(stream)), "w4a16_add_rmsnorm_gemm_qkv")
     return tuple(outs)
 
 

@@ -62,6 +62,34 @@ typedef enum {
                                 than GEMV and TC at every N measured) */
 } w4a16_path;
 
+/*
+ * The residual add + RMS normalisation fused into the QKV projection's
+ * prologue ("PerfXLLM on Snapdragon 8 Gen2", section 3.2: the residual
+ * addition and the normalisation are fused so their result does not go
+ * through global memory; here that result, X, is formed inside the
+ * projection itself and never stored).  For N <= 8 tokens, one launch of the
+ * decode kernel computes
+ *     r = fp16_RN(h + d)                      (d NULL: r = h)
+ *     X = fp16_RN((r * inv) * gamma),  inv = 1 / sqrt(mean(r^2) + eps)
+ * exactly as w4a16_add_rmsnorm (the same bits), then the outputs of
+ * w4a16_gemm_qkv from that X, and writes r to r_out when r_out is not NULL.
+ *   h, d, r_out  device fp16 [N][K], 16-byte aligned; r_out must not overlap
+ *                h or d (no in-place update here) nor any other argument.
+ *   gamma        device fp16 [K], 16-byte aligned; eps >= 0.
+ *   flags        0 or W4A16_FLAG_EARLY_WEIGHTS (the weights are read before
+ *                the previous kernel completes, h and d after it).
+ *   weight, bias, Mq, Mk, Mv, outputs: as w4a16_gemm_qkv.
+ * W4A16_ERR_UNSUPPORTED for N > 8 (run w4a16_add_rmsnorm, then
+ * w4a16_gemm_qkv); other errors as w4a16_gemm_qkv and w4a16_add_rmsnorm.
+ */
+W4A16_API w4a16_status w4a16_add_rmsnorm_gemm_qkv(const uint16_t* h, const uint16_t* d,
+                           const uint16_t* gamma, float eps, uint16_t* r_out,
+                           const void* wq_packed, const void* scales_packed,
+                           const void* zeros_packed, const uint16_t* bias,
+                           int Mq, int Mk, int Mv, int K, int N, int group,
+                           uint16_t* Yq, uint16_t* Yk, uint16_t* Yv,
+                           unsigned flags, void* stream);
+
 /* Flags of the workspace entry points (w4a16_gemm_ws, w4a16_gemm_qkv_ws,
  * w4a16_gemm_gate_up_ws). */
 #define W4A16_FLAG_EARLY_WEIGHTS 1u

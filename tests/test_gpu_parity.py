@@ -413,3 +413,92 @@ def test_add_rmsnorm_then_fused_qkv():
     c = np.cumsum((0,) + splits)
     for i, o in enumerate(outs):
         assert_close(to_f64(o), y_ref[:, c[i]:c[i + 1]], f"add_rmsnorm -> qkv split {i}")
+
+
+# ---------------------------- residual add + RMS norm as the QKV prologue ----
+
+@pytest.mark.parametrize("N,K,splits,with_d,with_bias", [
+    (1, 4096, (4096, 1024, 1024), True, False),     # LLaMA-7B-shaped GQA projection, one token
+    (1, 4096, (4096, 4096, 4096), True, True),      # LLaMA-7B QKV with a bias
+    (2, 4096, (4096, 1024, 1024), False, False),    # no d: r = h
+    (8, 4096, (4096, 1024, 1024), True, True),      # a full decode launch of 8 tokens
+    (3, 1152, (200, 72, 72), True, True),           # ragged K and projection borders inside tiles
+    (5, 11008, (1024, 256, 256), True, False),      # a long row: sum of squares over 11008 channels
+])
+def test_add_rmsnorm_fused_into_qkv(N, K, splits, with_d, with_bias):
+    """One launch (w4a16_add_rmsnorm_gemm_qkv) against the two-launch chain
+    (w4a16_add_rmsnorm, then w4a16_gemm_qkv): the same bits for Yq, Yk, Yv and
+    r, since the prologue repeats the norm kernel's arithmetic in its order;
+    and against the oracle's chain within C9, every element.  Outputs
+    NaN-prefilled."""
+    M = sum(splits)
+    h, d, gamma = _norm_inputs(N, K, seed=N + K, outliers=8)
+    p = synth.make_problem(M, K, N, seed=N + K)
+    w, _ = pack_problem(p)
+    ht, gt = torch.from_numpy(h).cuda(), torch.from_numpy(gamma).cuda()
+    dt = torch.from_numpy(d).cuda() if with_d else None
+    bias = (np.random.default_rng(M).normal(0, 1, size=M)).astype(np.float16) if with_bias else None
+    bt = torch.from_numpy(bias).cuda() if with_bias else None
+    r_chain, X = w4a16.add_rmsnorm(ht, gt, eps=NORM_EPS, d=dt, r_out=torch.empty_like(ht))
+    chain = w4a16.gemm_qkv(w, X, splits, bias=bt)
+    outs = tuple(torch.full((N, m), float("nan"), dtype=torch.float16, device="cuda") for m in splits)
+    r_fused = torch.full_like(ht, float("nan"))
+    fused = w4a16.add_rmsnorm_gemm_qkv(ht, gt, w, splits, eps=NORM_EPS, d=dt, r_out=r_fused, bias=bt, out=outs)
+    torch.cuda.synchronize()
+    for a, b in zip(fused, chain):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert torch.equal(r_fused.view(torch.int16), r_chain.view(torch.int16))
+    _, x_ref = oracle.add_rmsnorm(h.view(np.uint16), gamma.view(np.uint16), NORM_EPS,
+                                  d=d.view(np.uint16) if with_d else None)
+    y_ref = oracle.gemm(p.q, p.zeros, p.scales, oracle.fp16_from_double(x_ref))
+    if with_bias:
+        y_ref = y_ref + bias.astype(np.float64)[None, :]
+    c = np.cumsum((0,) + tuple(splits))
+    for i, o in enumerate(fused):
+        assert_close(to_f64(o), y_ref[:, c[i]:c[i + 1]], f"add_rmsnorm + qkv fused, split {i}, N={N}")
+
+
+def test_add_rmsnorm_fused_into_qkv_early_weights_in_a_chain():
+    """Under programmatic launch the prologue reads h and d only after the
+    previous kernel (here the norm kernel writing h in place) completed."""
+    N, K, splits = 1, 4096, (4096, 1024, 1024)
+    M = sum(splits)
+    h, d, gamma = _norm_inputs(N, K, seed=21)
+    p = synth.make_problem(M, K, N, seed=21)
+    w, _ = pack_problem(p)
+    ht, dt, gt = (torch.from_numpy(a).cuda() for a in (h, d, gamma))
+    h2 = ht.clone()
+    d2 = torch.from_numpy(_norm_inputs(N, K, seed=22)[1]).cuda()
+    # Reference: r1 = h + d (in place), then the fused call on (r1, d2).
+    ref_in = ht.clone()
+    w4a16.add_rmsnorm(ref_in, gt, eps=NORM_EPS, d=dt, r_out=ref_in)
+    ref = w4a16.add_rmsnorm_gemm_qkv(ref_in, gt, w, splits, eps=NORM_EPS, d=d2)
+    torch.cuda.synchronize()
+    w4a16.add_rmsnorm(h2, gt, eps=NORM_EPS, d=dt, r_out=h2)
+    got = w4a16.add_rmsnorm_gemm_qkv(h2, gt, w, splits, eps=NORM_EPS, d=d2, flags=w4a16.FLAG_EARLY_WEIGHTS)
+    torch.cuda.synchronize()
+    for a, b in zip(got, ref):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_add_rmsnorm_fused_into_qkv_rejects_without_launching():
+    L = w4a16.lib()
+    N, K, splits = 2, 256, (128, 64, 64)
+    p = synth.make_problem(sum(splits), K, N, seed=3)
+    w, _ = pack_problem(p)
+    h = torch.zeros((16, K), dtype=torch.float16, device="cuda")
+    g = torch.ones(K, dtype=torch.float16, device="cuda")
+    ys = [torch.empty((16, m), dtype=torch.float16, device="cuda") for m in splits]
+    s = torch.cuda.current_stream().cuda_stream
+
+    def call(N=2, r_out=None, eps=1e-6, flags=0, h_ptr=None):
+        return L.w4a16_add_rmsnorm_gemm_qkv(h.data_ptr() if h_ptr is None else h_ptr, None, g.data_ptr(), eps,
+                                            r_out, w.wq.data_ptr(), w.scales.data_ptr(), w.zeros.data_ptr(), None,
+                                            *splits, K, N, 128, ys[0].data_ptr(), ys[1].data_ptr(),
+                                            ys[2].data_ptr(), flags, s)
+    assert call(N=9) == w4a16.ERR_UNSUPPORTED              # more tokens than one decode launch
+    assert call(r_out=h.data_ptr()) == w4a16.ERR_INVALID_ARG   # in place over h
+    assert call(eps=-1.0) == w4a16.ERR_INVALID_ARG
+    assert call(flags=2) == w4a16.ERR_INVALID_ARG
+    assert call(h_ptr=h.data_ptr() + 8) == w4a16.ERR_MISALIGNED
+    assert call(r_out=ys[0].data_ptr()) == w4a16.ERR_INVALID_ARG   # r over Yq
