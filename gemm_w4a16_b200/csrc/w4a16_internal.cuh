@@ -239,12 +239,16 @@ __device__ __forceinline__ void store_row(const RowDst& d, bool has_bias, int n,
 // (0..127, thread = row, all 32 lanes of the warp calling together) of block
 // b.  Lanes 0..15 hold gate rows and take their channel's up value from lane
 // + 16, then write H[n][i] = fp16_RN(silu(g) * u), silu(g) = g / (1 + e^-g),
-// in fp32 (e^-g overflowing to infinity gives silu = -0, not NaN).
+// in fp32 with the hardware exponential and approximate division (a few fp32
+// ulps, far below the one fp16 rounding of H; e^-g overflowing to infinity
+// gives silu = -0, not NaN).  At large N this runs on the tile kernel's
+// critical path, where the accurate forms cost 8 % more (LLaMA-7B gate/up,
+// N = 4096: 707 against 654 us).
 __device__ __forceinline__ void store_gate_up(const OutMap& o, int b, int r, int n, float v, bool valid) {
   const float u = __shfl_down_sync(0xffffffffu, v, 16);
   const int i = gate_up_channel(b, r);
   if (valid && (r & 16) == 0 && i < o.mi) {
-    const float silu = v / (1.0f + expf(-v));
+    const float silu = __fdividef(v, 1.0f + __expf(-v));
     o.h[(size_t)n * o.mi + i] = __half_as_ushort(__float2half_rn(silu * u));
   }
 }
