@@ -272,10 +272,12 @@ __device__ __forceinline__ void gv_norm_x(const NormIn& nin, int K, int ga, int 
   }
 }
 
-// KW = 1: the CTA's 8 warps are the 8 row tiles of a 128-row block; KW = 2:
-// 4 row tiles (half a block) with two warps each, which take the two halves
-// of the CTA's K range and meet in shared memory (more warps per row for
-// shapes with few row blocks).
+// KW = 1: the CTA's 8 warps are the 8 row tiles of a 128-row block; KW = 2
+// or 4: 8 / KW row tiles (a half or a quarter of a block) with KW warps
+// each, which take KW parts of the CTA's K range and meet in shared memory
+// in a fixed order (more warps per row, and fewer or no cluster ranks, for
+// shapes with few row blocks).  A CTA's rows stay whole 32-row groups, which
+// the gate/up pairing needs.
 template <int NT, int kEpi, int KW, bool kNorm>
 __global__ void __launch_bounds__(kGvThreads, kGvCtasPerSm)
 gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
@@ -467,30 +469,31 @@ cudaError_t launch_nt(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p
                             nin);
 }
 
-// One launch of nt tokens (1..8) with row split kw (1 or 2).
+template <int kEpi, int KW, bool kNorm>
+cudaError_t launch_kw(int nt, const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p, const uint16_t* X,
+                      uint16_t* Y, int M, int K, int cl, bool pdl, cudaStream_t stream, const OutMap& om,
+                      const NormIn& nin) {
+  switch (nt) {
+    case 1: return launch_nt<1, kEpi, KW, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
+    case 2: return launch_nt<2, kEpi, KW, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
+    case 3: return launch_nt<3, kEpi, KW, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
+    case 4: return launch_nt<4, kEpi, KW, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
+    case 5: return launch_nt<5, kEpi, KW, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
+    case 6: return launch_nt<6, kEpi, KW, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
+    case 7: return launch_nt<7, kEpi, KW, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
+    default: return launch_nt<8, kEpi, KW, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
+  }
+}
+
+// One launch of nt tokens (1..8) with row split kw (1, 2, or 4 at nt = 1).
 template <int kEpi, bool kNorm = false>
 cudaError_t launch_epi(int nt, int kw, const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p,
                        const uint16_t* X, uint16_t* Y, int M, int K, int cl, bool pdl, cudaStream_t stream,
                        const OutMap& om, const NormIn& nin) {
-  const bool two = kw == 2;
-  switch (nt) {
-    case 1: return two ? launch_nt<1, kEpi, 2, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin)
-                       : launch_nt<1, kEpi, 1, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
-    case 2: return two ? launch_nt<2, kEpi, 2, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin)
-                       : launch_nt<2, kEpi, 1, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
-    case 3: return two ? launch_nt<3, kEpi, 2, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin)
-                       : launch_nt<3, kEpi, 1, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
-    case 4: return two ? launch_nt<4, kEpi, 2, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin)
-                       : launch_nt<4, kEpi, 1, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
-    case 5: return two ? launch_nt<5, kEpi, 2, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin)
-                       : launch_nt<5, kEpi, 1, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
-    case 6: return two ? launch_nt<6, kEpi, 2, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin)
-                       : launch_nt<6, kEpi, 1, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
-    case 7: return two ? launch_nt<7, kEpi, 2, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin)
-                       : launch_nt<7, kEpi, 1, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
-    default: return two ? launch_nt<8, kEpi, 2, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin)
-                        : launch_nt<8, kEpi, 1, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
-  }
+  if (kw == 4 && nt == 1)   // the chooser takes KW = 4 for one token only
+    return launch_nt<1, kEpi, 4, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
+  if (kw == 2) return launch_kw<kEpi, 2, kNorm>(nt, wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
+  return launch_kw<kEpi, 1, kNorm>(nt, wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
 }
 
 struct GvShape {
@@ -499,21 +502,24 @@ struct GvShape {
 
 }  // namespace
 
-// Row split KW (1 or 2 CTAs per 128-row block, see gemv_kernel) and cluster
+// Row split KW (1, 2 or 4 CTAs per 128-row block, see gemv_kernel) and cluster
 // size along K (1..8), from the measured LLaMA N = 1 shapes: all CTAs
 // resident in one wave (kGvCtasPerSm per SM, set by the registers of one
 // CTA), and at least 2.5 CTAs per SM on average when the shape allows it
 // (fewer warps per SM hide the load and MMA latencies badly); among those
 // the smallest busiest-SM work, ceil(CTAs / SMs) x the groups of one warp,
-// then the larger KW (measured: gate/up 15.7 against 16.3 us at equal CTA
-// counts), then the smaller cluster.  When no choice reaches 2.5
+// then the larger KW (measured at equal CTA counts: gate/up 15.7 against
+// 16.3 us, QKV 9.1 against 9.7 us with KW = 4 and no cluster), then the
+// smaller cluster.  When no choice reaches 2.5
 // CTAs per SM, the most CTAs.  The staged activation slice must fit.
 GvShape gemv_shape(int M, int K, int sms, int nt) {
   const int blocks = ceil_div(M, kRowBlock);
   const int kg = K / kGroup;
   GvShape best = {0, 0};
   long long best_key[4] = {0, 0, 0, 0};
-  for (int kw = 1; kw <= 2; ++kw) {
+  // KW = 4 only for one token: at N = 8 it was slower on every LLaMA-7B shape
+  // (down 17.4 against 11.9 us).
+  for (int kw = 1; kw <= (nt == 1 ? 4 : 2); kw *= 2) {
     for (int cl = 1; cl <= kMaxCluster && cl <= kg; ++cl) {
       if (nt * gv_xstride(ceil_div(kg, cl)) * 2 > kMaxXSmem) continue;
       const long long ctas = (long long)blocks * kw * cl;
