@@ -540,7 +540,12 @@ GvShape gemv_shape(int M, int K, int sms, int nt) {
       }
     }
   }
-  return best.cl > 0 ? best : GvShape{1, kMaxCluster};
+  if (best.cl > 0) return best;
+  // Nothing fits in one wave (many row blocks and a wide activation slice):
+  // the smallest cluster whose slice fits, over several waves.
+  for (int cl = 1; cl <= kMaxCluster && cl <= kg; ++cl)
+    if (nt * gv_xstride(ceil_div(kg, cl)) * 2 <= kMaxXSmem) return GvShape{1, cl};
+  return GvShape{1, kMaxCluster};
 }
 
 cudaError_t launch_gemv(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros,
