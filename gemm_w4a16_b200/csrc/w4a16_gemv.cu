@@ -49,6 +49,7 @@ constexpr int kGvCtasPerSm = 3;                       // resident CTAs per SM (r
 constexpr int kGvWBytes = 4 * kRowBlock * 16;         // one group of 128 rows: 8 KB
 constexpr int kMaxCluster = 8;
 constexpr int kMaxXSmem = 64 * 1024;                  // largest staged activation slice
+constexpr int kGvSmemLimit = 128 * 1024;              // dynamic shared memory a CTA may ask for
 
 // D += A B for one m16n8k16 tile: A 16 x 16 f16 (row), B 16 x 8 f16 (col),
 // fp32 accumulators, in the warp-level fragment layout of mma.sync.
@@ -446,11 +447,12 @@ cudaError_t launch_nt(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p
                       uint16_t* Y, int M, int K, int cl, bool pdl, cudaStream_t stream, const OutMap& om,
                       const NormIn& nin) {
   static std::atomic<unsigned long long> smem_set{0};
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(gemv_kernel<NT, kEpi, KW, kNorm>), 128 * 1024,
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(gemv_kernel<NT, kEpi, KW, kNorm>), kGvSmemLimit,
                                     smem_set);
   if (e != cudaSuccess) return e;
   const int blocks = ceil_div(M, kRowBlock);
   const GvLayout L = gv_layout(NT, ceil_div(K / kGroup, cl), cl, KW);
+  if (L.total > kGvSmemLimit) return cudaErrorNotSupported;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(blocks * KW * cl), 1, 1);
   cfg.blockDim = dim3(kGvThreads, 1, 1);
@@ -522,6 +524,7 @@ GvShape gemv_shape(int M, int K, int sms, int nt) {
   for (int kw = 1; kw <= (nt == 1 ? 4 : 2); kw *= 2) {
     for (int cl = 1; cl <= kMaxCluster && cl <= kg; ++cl) {
       if (nt * gv_xstride(ceil_div(kg, cl)) * 2 > kMaxXSmem) continue;
+      if (gv_layout(nt, ceil_div(kg, cl), cl, kw).total > kGvSmemLimit) continue;
       const long long ctas = (long long)blocks * kw * cl;
       if ((kw > 1 || cl > 1) && ctas > (long long)kGvCtasPerSm * sms) continue;
       const bool dense = 2 * ctas >= 5LL * sms;
@@ -544,7 +547,9 @@ GvShape gemv_shape(int M, int K, int sms, int nt) {
   // Nothing fits in one wave (many row blocks and a wide activation slice):
   // the smallest cluster whose slice fits, over several waves.
   for (int cl = 1; cl <= kMaxCluster && cl <= kg; ++cl)
-    if (nt * gv_xstride(ceil_div(kg, cl)) * 2 <= kMaxXSmem) return GvShape{1, cl};
+    if (nt * gv_xstride(ceil_div(kg, cl)) * 2 <= kMaxXSmem &&
+        gv_layout(nt, ceil_div(kg, cl), cl, 1).total <= kGvSmemLimit)
+      return GvShape{1, cl};
   return GvShape{1, kMaxCluster};
 }
 
