@@ -51,7 +51,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # capture of this repository's kernel; it holds only while the kernel source
 # is the one captured (sha256 prefix of csrc/w4a16_gemv.cu), and the bench
 # reports null otherwise.
-DECODE_TRAFFIC = {"src_sha256_prefix": "bdeaa3fb35a9c9a3", "qkv_dram_bytes": 26202880, "qkv_alg_bytes": 26181632}
+DECODE_TRAFFIC = {"src_sha256_prefix": "197e93164b6ccb59", "qkv_dram_bytes": 26202880, "qkv_alg_bytes": 26181632}
 NOMINAL_DENSE_FP16_TFLOPS = 2250.0   # B200 dense fp16/bf16 tensor rate, NVIDIA's figure
 
 
@@ -482,6 +482,7 @@ def main_ours(args):
         extra["prefill"] = prefill_measure(device, peaks, sampler)
         extra["n_sweep"] = n_sweep_measure(device, peaks, sampler)
         extra["llama3"] = llama3_measure(device, peaks, sampler)
+        extra["fused"] = fused_measure(device, peaks, sampler)
 
     res = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -649,6 +650,124 @@ def n_sweep_measure(device, peaks, sampler, copies=16, reps=20):
     torch.cuda.empty_cache()
     return {"M": M, "K": K, "columns": ["N", "path", "us", "roof_frac", "auto_choice"], "rows": rows,
             "clocks": sampler.summary(t0, t1)}
+
+
+def fused_measure(device, peaks, sampler, reps=20):
+    """The fused forms and the secondary kernels, compactly: per-call
+    microseconds (median over `reps` graph replays, each graph several
+    rotated copies, beyond L2) with the clock summary of each window.
+      qkv_norm_n1     add_rmsnorm + gemm_qkv_ws chained vs add_rmsnorm_gemm_qkv
+                      (LLaMA-7B QKV, N = 1, early weights);
+      qkv_epilogue    plain product vs the QKV split + bias form, N = 1 and 4096;
+      gate_up         plain product vs SiLU(gate)*up form vs plain + torch, N = 1
+                      and 4096;
+      add_rmsnorm     16384 x 4096 (HBM bytes 8 per channel);
+      quantize_qkv    the group quantiser on the 12288 x 4096 weight."""
+    import torch
+
+    from gemm_w4a16_b200 import synth, w4a16
+
+    out = {}
+    fl = w4a16.FLAG_EARLY_WEIGHTS
+
+    def timed(fns, per_graph):
+        res = {}
+        for name, fn in fns.items():
+            g = capture(fn, device)
+            t0 = time.time()
+            _, per = time_steps(g, reps, 3, device)
+            res[name] = {"us": pct(per, 1e3 / per_graph)["median"], "clocks": sampler.summary(t0, time.time())}
+            del g
+        return res
+
+    # Residual add + RMS norm folded into the QKV projection, N = 1.
+    M, K, splits = 12288, 4096, (4096, 4096, 4096)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(31)
+    gamma = (1.0 + 0.1 * torch.randn(K, device=device, generator=gen)).half()
+    sets = []
+    for c in range(8):
+        w, _ = make_device_problem(device, M, K, 1, seed=60 + c)
+        h = torch.randn((1, K), device=device, generator=gen).half()
+        d = torch.randn((1, K), device=device, generator=gen).half()
+        sets.append((w, h, d, torch.empty_like(h), torch.empty_like(h),
+                     tuple(torch.empty((1, m), dtype=torch.float16, device=device) for m in splits)))
+    ws = w4a16.Workspace(device, w4a16.workspace_size(M, K, 1))
+    out["qkv_norm_n1"] = timed({
+        "chain": lambda: [(w4a16.add_rmsnorm(h, gamma, d=d, r_out=r, X=X),
+                           w4a16.gemm_qkv_ws(w, X, splits, out=o, workspace=ws, flags=fl))
+                          for w, h, d, r, X, o in sets],
+        "fused": lambda: [w4a16.add_rmsnorm_gemm_qkv(h, gamma, w, splits, d=d, r_out=r, out=o, flags=fl)
+                          for w, h, d, r, X, o in sets]}, len(sets))
+    del sets
+
+    # QKV split + bias epilogue against the plain product.
+    res = {}
+    for N, copies in ((1, 8), (4096, 2)):
+        probs = [make_device_problem(device, M, K, N, seed=70 + c) for c in range(copies)]
+        bias = torch.randn(M, device=device, generator=gen).half()
+        ys = [torch.empty((N, M), dtype=torch.float16, device=device) for _ in probs]
+        os_ = [tuple(torch.empty((N, m), dtype=torch.float16, device=device) for m in splits) for _ in probs]
+        ws.ensure(w4a16.workspace_size(M, K, N))
+        res[f"n{N}"] = timed({
+            "plain": lambda: [w4a16.gemm_ws(w, x, Y=y, workspace=ws, flags=fl) for (w, x), y in zip(probs, ys)],
+            "fused_split_bias": lambda: [w4a16.gemm_qkv_ws(w, x, splits, bias=bias, out=o, workspace=ws, flags=fl)
+                                         for (w, x), o in zip(probs, os_)]}, copies)
+        del probs, ys, os_
+        torch.cuda.empty_cache()
+    out["qkv_epilogue"] = res
+
+    # SiLU(gate) * up epilogue.
+    Mi = 11008
+    res = {}
+    for N, copies in ((1, 8), (4096, 2)):
+        sets = []
+        for _ in range(copies):
+            q, z, sc = synth.make_weights_torch(2 * Mi, K, GROUP, gen, device)
+            sets.append((w4a16.pack_gate_up(q, sc, z), w4a16.pack(q, sc, z),
+                         synth.make_activations_torch(N, K, gen, device),
+                         torch.empty((N, Mi), dtype=torch.float16, device=device),
+                         torch.empty((N, 2 * Mi), dtype=torch.float16, device=device)))
+            del q, z, sc
+        ws.ensure(w4a16.workspace_size(2 * Mi, K, N))
+        res[f"n{N}"] = timed({
+            "plain": lambda: [w4a16.gemm_ws(wp, x, Y=y, workspace=ws, flags=fl) for _, wp, x, _, y in sets],
+            "fused": lambda: [w4a16.gemm_gate_up_ws(wg, x, H=h, workspace=ws, flags=fl)
+                              for wg, _, x, h, _ in sets],
+            "plain_then_torch": lambda: [(w4a16.gemm_ws(wp, x, Y=y, workspace=ws, flags=fl),
+                                          torch.mul(torch.nn.functional.silu(y[:, :Mi]), y[:, Mi:], out=h))
+                                         for _, wp, x, h, y in sets]}, copies)
+        del sets
+        torch.cuda.empty_cache()
+    out["gate_up"] = res
+
+    # Residual add + RMS norm at prefill width, and the group quantiser.
+    Nn = 16384
+    h = torch.randn((Nn, K), device=device, generator=gen).half()
+    d = torch.randn((Nn, K), device=device, generator=gen).half()
+    r, X = torch.empty_like(h), torch.empty_like(h)
+    t = timed({"add_rmsnorm": lambda: w4a16.add_rmsnorm(h, gamma, d=d, r_out=r, X=X)}, 1)["add_rmsnorm"]
+    gbs = (8 * Nn * K + 2 * K) / (t["us"] * 1e-6) / 1e9
+    out["add_rmsnorm_n16384"] = dict(t, GBps=gbs, frac_hbm=gbs / peaks["hbm_gbs"])
+    del h, d, r, X
+    wts = [torch.randn((M, K), device=device, dtype=torch.float32).mul_(0.05).half() for _ in range(4)]
+    qs = [(torch.empty((M, K), dtype=torch.uint8, device=device),
+           torch.empty((M, K // GROUP), dtype=torch.float16, device=device),
+           torch.empty((M, K // GROUP), dtype=torch.uint8, device=device)) for _ in wts]
+    lib = w4a16.lib()
+
+    def quantize_all():
+        stream = torch.cuda.current_stream(device).cuda_stream   # the capture stream inside capture
+        for w, (q, s, z) in zip(wts, qs):
+            if lib.w4a16_quantize(w.data_ptr(), M, K, GROUP, q.data_ptr(), s.data_ptr(), z.data_ptr(), stream):
+                raise RuntimeError("w4a16_quantize failed")
+
+    t = timed({"quantize": quantize_all}, len(wts))["quantize"]
+    gbs = (3 * M * K + 3 * M * (K // GROUP)) / (t["us"] * 1e-6) / 1e9
+    out["quantize_qkv"] = dict(t, GBps=gbs, frac_hbm=gbs / peaks["hbm_gbs"])
+    del wts, qs
+    torch.cuda.empty_cache()
+    return out
 
 
 LLAMA3_SHAPES = [("qkv", 6144, 4096), ("o", 4096, 4096), ("gate_up", 28672, 4096), ("down", 4096, 14336),
