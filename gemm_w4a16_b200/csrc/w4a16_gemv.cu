@@ -283,11 +283,18 @@ template <int NT, int kEpi, int KW, bool kNorm>
 __global__ void __launch_bounds__(kGvThreads, kGvCtasPerSm)
 gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
             const uint8_t* __restrict__ z_p, const uint16_t* __restrict__ X,
-            uint16_t* __restrict__ Y, int M, int K, int cl, int early, OutMap om, NormIn nin) {
+            uint16_t* __restrict__ Y, int M, int K, uint32_t cl_magic, int early, OutMap om, NormIn nin) {
   extern __shared__ __align__(128) uint8_t smem[];
+  // Grid (row-block parts, cl): the cluster spans y, so blockIdx.y is the
+  // CTA's rank along K and blockIdx.x its part of a row block; n / cl is
+  // the high word of n * ceil(2^32 / cl) (exact for n < 2^32 / cl^2).
+  const int cl = (int)gridDim.y;
+  const int crank = (int)blockIdx.y;
+  const int chunk = (int)blockIdx.x;
+  auto div_cl = [&](int n) { return cl == 1 ? n : (int)__umulhi((uint32_t)n, cl_magic); };
   const int kg = K / kGroup;
   const int kc_n = K / kChunkK;
-  const int gspan = ceil_div(kg, cl);
+  const int gspan = div_cl(kg + cl - 1);
   const GvLayout L = gv_layout(NT, gspan, cl, KW);
   constexpr int kRows = kRowBlock / KW;    // rows of the CTA
   constexpr int kTiles = kGvWarps / KW;    // 16-row tiles of the CTA
@@ -298,11 +305,9 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
-  const int chunk = blockIdx.x / cl;       // (row block, part of it)
   const int b = chunk / KW;
   const int ro = (chunk % KW) * kRows;     // the CTA's first row in the block
-  const int crank = blockIdx.x % cl;
-  const int ga = (kg * crank) / cl, gb = (kg * (crank + 1)) / cl;
+  const int ga = div_cl(kg * crank), gb = div_cl(kg * (crank + 1));
   const int ng = gb - ga;
   const int xstride = gv_xstride(ng);
   // This warp's tile and its share [gw0, gw0 + ngw) of the CTA's groups.
@@ -327,9 +332,14 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   // requested first, so they do not queue behind the weight stream.
   auto stage_x = [&]() {
     const int pieces = ng * (kGroup / 8);
-    for (int idx = threadIdx.x; idx < NT * pieces; idx += kGvThreads) {
-      const int n = idx / pieces, p = idx - n * pieces;
-      cp_async16(xs + n * xstride + p * 8, X + (size_t)n * K + (size_t)ga * kGroup + p * 8);
+    if constexpr (NT == 1) {
+      for (int p = threadIdx.x; p < pieces; p += kGvThreads)
+        cp_async16(xs + p * 8, X + (size_t)ga * kGroup + p * 8);
+    } else {
+      for (int idx = threadIdx.x; idx < NT * pieces; idx += kGvThreads) {
+        const int n = idx / pieces, p = idx - n * pieces;
+        cp_async16(xs + n * xstride + p * 8, X + (size_t)n * K + (size_t)ga * kGroup + p * 8);
+      }
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
@@ -454,21 +464,22 @@ cudaError_t launch_nt(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p
   const GvLayout L = gv_layout(NT, ceil_div(K / kGroup, cl), cl, KW);
   if (L.total > kGvSmemLimit) return cudaErrorNotSupported;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(blocks * KW * cl), 1, 1);
+  cfg.gridDim = dim3((unsigned)(blocks * KW), (unsigned)cl, 1);
   cfg.blockDim = dim3(kGvThreads, 1, 1);
   cfg.dynamicSmemBytes = (size_t)L.total;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)cl;
-  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = (unsigned)cl;
   attr[0].val.clusterDim.z = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, gemv_kernel<NT, kEpi, KW, kNorm>, wq, s_p, z_p, X, Y, M, K, cl, pdl ? 1 : 0, om,
-                            nin);
+  const uint32_t cl_magic = cl > 1 ? (uint32_t)((0x100000000ull + (unsigned)cl - 1) / (unsigned)cl) : 0u;
+  return cudaLaunchKernelEx(&cfg, gemv_kernel<NT, kEpi, KW, kNorm>, wq, s_p, z_p, X, Y, M, K, cl_magic,
+                            pdl ? 1 : 0, om, nin);
 }
 
 template <int kEpi, int KW, bool kNorm>
