@@ -9,7 +9,7 @@
 //  * a CTA owns one 128-row block of the packed weight and a range of whole
 //    groups along K; each of its 8 warps owns one 16-row tile of that block
 //    and streams the tile's codes, scales and zeros straight from HBM into
-//    registers with 16-byte non-allocating loads, kGvDepth groups ahead of
+//    registers with 16-byte non-allocating loads, 3 or 4 groups ahead of
 //    the one it computes (no shared-memory staging, no barriers);
 //  * the first groups are requested before the grid dependency wait, so with
 //    programmatic dependent launch the weight stream starts while the
@@ -44,7 +44,12 @@ namespace {
 
 constexpr int kGvWarps = 8;                           // one 16-row MMA tile each
 constexpr int kGvThreads = kGvWarps * 32;
-constexpr int kGvDepth = 3;                           // groups of codes in flight per warp
+// Groups of codes in flight per warp, in registers: 4 for one token (80
+// registers still hold them without spills; the decode step ran 1.255 ->
+// 1.224 ms), 3 with more tokens (4 was slower at N = 8) or the normalising
+// prologue (which would spill).
+template <int NT, bool kNorm>
+__host__ __device__ constexpr int gv_depth() { return NT == 1 && !kNorm ? 4 : 3; }
 constexpr int kGvCtasPerSm = 3;                       // resident CTAs per SM (register budget)
 constexpr int kGvWBytes = 4 * kRowBlock * 16;         // one group of 128 rows: 8 KB
 constexpr int kMaxCluster = 8;
@@ -165,37 +170,37 @@ __device__ __forceinline__ void gv_consume(const GvFrag& f, const uint16_t* xg, 
   }
 }
 
-template <int U>
-__device__ __forceinline__ void gv_load_first(GvFrag (&f)[kGvDepth], int ng, const uint8_t* pw, const uint16_t* ps,
+template <int D, int U>
+__device__ __forceinline__ void gv_load_first(GvFrag (&f)[D], int ng, const uint8_t* pw, const uint16_t* ps,
                                               const uint8_t* pz) {
-  if constexpr (U < kGvDepth) {
+  if constexpr (U < D) {
     if (U < ng) gv_load<U>(f[U], pw, ps, pz);
-    gv_load_first<U + 1>(f, ng, pw, ps, pz);
+    gv_load_first<D, U + 1>(f, ng, pw, ps, pz);
   }
 }
 
 // Slots U.. of a step whose groups and refills all exist (no checks).
-template <int U>
-__device__ __forceinline__ void gv_step_full(GvFrag (&f)[kGvDepth], const uint8_t* pw, const uint16_t* ps,
+template <int D, int U>
+__device__ __forceinline__ void gv_step_full(GvFrag (&f)[D], const uint8_t* pw, const uint16_t* ps,
                                              const uint8_t* pz, const uint16_t* xg, float (&acc)[4]) {
-  if constexpr (U < kGvDepth) {
+  if constexpr (U < D) {
     gv_consume(f[U], xg + U * kGroup, acc);
-    gv_load<U + kGvDepth>(f[U], pw, ps, pz);
-    gv_step_full<U + 1>(f, pw, ps, pz, xg, acc);
+    gv_load<U + D>(f[U], pw, ps, pz);
+    gv_step_full<D, U + 1>(f, pw, ps, pz, xg, acc);
   }
 }
 
-// Slots U.. of one step of kGvDepth groups starting at group i0: consume
-// group i0 + U from slot U, refill the slot with group i0 + U + kGvDepth.
-template <int U>
-__device__ __forceinline__ void gv_step(GvFrag (&f)[kGvDepth], int i0, int ng, const uint8_t* pw,
+// Slots U.. of one step of D groups starting at group i0: consume group
+// i0 + U from slot U, refill the slot with group i0 + U + D.
+template <int D, int U>
+__device__ __forceinline__ void gv_step(GvFrag (&f)[D], int i0, int ng, const uint8_t* pw,
                                         const uint16_t* ps, const uint8_t* pz, const uint16_t* xg,
                                         float (&acc)[4]) {
-  if constexpr (U < kGvDepth) {
+  if constexpr (U < D) {
     if (i0 + U < ng) {
       gv_consume(f[U], xg + U * kGroup, acc);
-      if (i0 + U + kGvDepth < ng) gv_load<U + kGvDepth>(f[U], pw, ps, pz);
-      gv_step<U + 1>(f, i0, ng, pw, ps, pz, xg, acc);
+      if (i0 + U + D < ng) gv_load<U + D>(f[U], pw, ps, pz);
+      gv_step<D, U + 1>(f, i0, ng, pw, ps, pz, xg, acc);
     }
   }
 }
@@ -348,8 +353,9 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   // grid dependency wait (which returns at once unless the launch is
   // programmatic); X (or the residual stream it comes from), written by that
   // kernel, only after it.
-  GvFrag f[kGvDepth];
-  gv_load_first<0>(f, ngw, pw, ps, pz);
+  constexpr int kDepth = gv_depth<NT, kNorm>();
+  GvFrag f[kDepth];
+  gv_load_first<kDepth, 0>(f, ngw, pw, ps, pz);
   ptx::griddep_wait();
   if constexpr (kNorm)
     gv_norm_x<NT>(nin, K, ga, ng, xs, xstride, chunk == 0);
@@ -363,19 +369,19 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   const uint16_t* xg = xs + (g < NT ? g : NT - 1) * xstride + 32 * c + gw0 * kGroup;
   int i0 = 0;
-  for (; i0 + 2 * kGvDepth <= ngw; i0 += kGvDepth) {   // every refill exists
-    gv_step_full<0>(f, pw, ps, pz, xg, acc);
-    pw += kGvDepth * kGvWBytes;
-    ps += kGvDepth * kRowBlock;
-    pz += kGvDepth * (kRowBlock / 2);
-    xg += kGvDepth * kGroup;
+  for (; i0 + 2 * kDepth <= ngw; i0 += kDepth) {   // every refill exists
+    gv_step_full<kDepth, 0>(f, pw, ps, pz, xg, acc);
+    pw += kDepth * kGvWBytes;
+    ps += kDepth * kRowBlock;
+    pz += kDepth * (kRowBlock / 2);
+    xg += kDepth * kGroup;
   }
-  for (; i0 < ngw; i0 += kGvDepth) {
-    gv_step<0>(f, i0, ngw, pw, ps, pz, xg, acc);
-    pw += kGvDepth * kGvWBytes;
-    ps += kGvDepth * kRowBlock;
-    pz += kGvDepth * (kRowBlock / 2);
-    xg += kGvDepth * kGroup;
+  for (; i0 < ngw; i0 += kDepth) {
+    gv_step<kDepth, 0>(f, i0, ngw, pw, ps, pz, xg, acc);
+    pw += kDepth * kGvWBytes;
+    ps += kDepth * kRowBlock;
+    pz += kDepth * (kRowBlock / 2);
+    xg += kDepth * kGroup;
   }
   // Accumulator fragment: MMA rows g (entries 0, 1: block row rl) and g + 8
   // (entries 2, 3: block row rl + 1), tokens 2 c and 2 c + 1.
