@@ -522,51 +522,66 @@ struct GvShape {
 }  // namespace
 
 // Row split KW (1, 2 or 4 CTAs per 128-row block, see gemv_kernel) and cluster
-// size along K (1..8), from the measured LLaMA N = 1 shapes: all CTAs
-// resident in one wave (kGvCtasPerSm per SM, set by the registers of one
+// size along K (1..8), from the measured LLaMA N = 1 shapes.  First pass: all
+// CTAs resident in one wave (kGvCtasPerSm per SM, set by the registers of one
 // CTA), and at least 2.5 CTAs per SM on average when the shape allows it
 // (fewer warps per SM hide the load and MMA latencies badly); among those
 // the smallest busiest-SM work, ceil(CTAs / SMs) x the groups of one warp,
 // then the larger KW (measured at equal CTA counts: gate/up 15.7 against
 // 16.3 us, QKV 9.1 against 9.7 us with KW = 4 and no cluster), then the
-// smaller cluster.  When no choice reaches 2.5
-// CTAs per SM, the most CTAs.  The staged activation slice must fit.
+// smaller cluster; when no choice reaches 2.5 CTAs per SM, the most CTAs.
+// For one token, when that finds no dense single wave because the weight
+// has too many row blocks for KW = 4 to fit in one wave, KW = 4 without a
+// cluster over several waves instead (gate/up 22016 x 4096: 14.9 against
+// 15.7 us; 28672 x 4096: 20.8 against 29.2 us; 128256 x 4096: 76.5 against
+// 78.3 us; splitting such weights further along K was slower).  The staged
+// activation slice must fit.
 GvShape gemv_shape(int M, int K, int sms, int nt) {
   const int blocks = ceil_div(M, kRowBlock);
   const int kg = K / kGroup;
+  const long long wave = (long long)kGvCtasPerSm * sms;
   GvShape best = {0, 0};
   long long best_key[4] = {0, 0, 0, 0};
+  auto consider = [&](int kw, int cl, const long long (&key)[4]) {
+    bool better = best.cl == 0;
+    for (int i = 0; i < 4 && !better; ++i) {
+      if (key[i] != best_key[i]) {
+        better = key[i] < best_key[i];
+        break;
+      }
+    }
+    if (better) {
+      best = {kw, cl};
+      for (int i = 0; i < 4; ++i) best_key[i] = key[i];
+    }
+  };
+  auto fits = [&](int kw, int cl) {
+    return nt * gv_xstride(ceil_div(kg, cl)) * 2 <= kMaxXSmem &&
+           gv_layout(nt, ceil_div(kg, cl), cl, kw).total <= kGvSmemLimit;
+  };
+  auto load = [&](int kw, int cl) {
+    const long long ctas = (long long)blocks * kw * cl;
+    return (long long)ceil_div((int)ctas, sms) * ceil_div(ceil_div(kg, cl), kw);
+  };
   // KW = 4 only for one token: at N = 8 it was slower on every LLaMA-7B shape
   // (down 17.4 against 11.9 us).
   for (int kw = 1; kw <= (nt == 1 ? 4 : 2); kw *= 2) {
     for (int cl = 1; cl <= kMaxCluster && cl <= kg; ++cl) {
-      if (nt * gv_xstride(ceil_div(kg, cl)) * 2 > kMaxXSmem) continue;
-      if (gv_layout(nt, ceil_div(kg, cl), cl, kw).total > kGvSmemLimit) continue;
+      if (!fits(kw, cl)) continue;
       const long long ctas = (long long)blocks * kw * cl;
-      if ((kw > 1 || cl > 1) && ctas > (long long)kGvCtasPerSm * sms) continue;
+      if ((kw > 1 || cl > 1) && ctas > wave) continue;
       const bool dense = 2 * ctas >= 5LL * sms;
-      const long long load = (long long)ceil_div((int)ctas, sms) * ceil_div(ceil_div(kg, cl), kw);
-      const long long key[4] = {dense ? 0 : 1, dense ? load : -ctas, -kw, cl};
-      bool better = best.cl == 0;
-      for (int i = 0; i < 4 && !better; ++i) {
-        if (key[i] != best_key[i]) {
-          better = key[i] < best_key[i];
-          break;
-        }
-      }
-      if (better) {
-        best = {kw, cl};
-        for (int i = 0; i < 4; ++i) best_key[i] = key[i];
-      }
+      const long long key[4] = {dense ? 0 : 1, dense ? load(kw, cl) : -ctas, -kw, cl};
+      consider(kw, cl, key);
     }
   }
+  const bool single_dense = best.cl > 0 && best_key[0] == 0 && (long long)blocks * best.kw * best.cl <= wave;
+  if (nt == 1 && !single_dense && 4LL * blocks > wave && fits(4, 1)) return GvShape{4, 1};
   if (best.cl > 0) return best;
   // Nothing fits in one wave (many row blocks and a wide activation slice):
   // the smallest cluster whose slice fits, over several waves.
   for (int cl = 1; cl <= kMaxCluster && cl <= kg; ++cl)
-    if (nt * gv_xstride(ceil_div(kg, cl)) * 2 <= kMaxXSmem &&
-        gv_layout(nt, ceil_div(kg, cl), cl, 1).total <= kGvSmemLimit)
-      return GvShape{1, cl};
+    if (fits(1, cl)) return GvShape{1, cl};
   return GvShape{1, kMaxCluster};
 }
 
