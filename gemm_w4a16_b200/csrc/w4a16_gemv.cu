@@ -49,12 +49,15 @@ constexpr int kGvThreads = kGvWarps * 32;
 // 1.224 ms), 3 with more tokens (4 was slower at N = 8) or the normalising
 // prologue (which would spill).
 template <int NT, bool kNorm>
-__host__ __device__ constexpr int gv_depth() { return NT == 1 && !kNorm ? 4 : 3; }
+__host__ __device__ constexpr int gv_depth() { return NT == 1 && !kNorm ? 4 : NT > 8 ? 2 : 3; }
 constexpr int kGvCtasPerSm = 3;                       // resident CTAs per SM (register budget)
 constexpr int kGvWBytes = 4 * kRowBlock * 16;         // one group of 128 rows: 8 KB
 constexpr int kMaxCluster = 8;
 constexpr int kMaxXSmem = 64 * 1024;                  // largest staged activation slice
 constexpr int kGvSmemLimit = 128 * 1024;              // dynamic shared memory a CTA may ask for
+constexpr int kSmemPerSm = 228 * 1024;                // shared memory of one SM (sm_100)
+constexpr int kSmemPerCta = 1024;                     // of it reserved per resident CTA
+constexpr int kWideMaxM = 4096;                       // tallest weight given 16-token launches
 
 // D += A B for one m16n8k16 tile: A 16 x 16 f16 (row), B 16 x 8 f16 (col),
 // fp32 accumulators, in the warp-level fragment layout of mma.sync.
@@ -152,21 +155,37 @@ __device__ __forceinline__ void gv_consts(const GvFrag& f, GroupConsts& lo, Grou
   hi.s2 = prmt<0x3232>(f.s, f.s);
 }
 
-// Dequantise one group of the lane's two rows and accumulate its eight MMAs;
-// xg points at token g's activations at k = 32 c of the group.
-__device__ __forceinline__ void gv_consume(const GvFrag& f, const uint16_t* xg, float (&acc)[4]) {
+// The lane's accumulators: one m16n8 fragment per block of 8 tokens (NB = 2
+// for 9 to 16 tokens, whose second block shares the dequantised A
+// fragments), and the offset in halves of block j's activation row from
+// block 0's.
+template <int NB>
+struct GvAcc {
+  float c[NB][4];
+  int xoff[NB];
+};
+
+// Dequantise one group of the lane's two rows and accumulate its eight MMAs
+// per token block; xg points at token g's activations at k = 32 c of the
+// group.
+template <int NB>
+__device__ __forceinline__ void gv_consume(const GvFrag& f, const uint16_t* xg, GvAcc<NB>& A) {
   GroupConsts clo, chi;
   gv_consts(f, clo, chi);
   const uint32_t wl[4] = {f.lo.x, f.lo.y, f.lo.z, f.lo.w};
   const uint32_t wh[4] = {f.hi.x, f.hi.y, f.hi.z, f.hi.w};
 #pragma unroll
   for (int t = 0; t < 4; ++t) {
-    const uint4 xb = *reinterpret_cast<const uint4*>(xg + 8 * t);
+    uint4 xb[NB];
+#pragma unroll
+    for (int j = 0; j < NB; ++j) xb[j] = *reinterpret_cast<const uint4*>(xg + A.xoff[j] + 8 * t);
     uint32_t al[4], ah[4];
     dequant_word(wl[t], clo, al);
     dequant_word(wh[t], chi, ah);
-    mma_16816(acc, al[0], ah[0], al[1], ah[1], xb.x, xb.y);
-    mma_16816(acc, al[2], ah[2], al[3], ah[3], xb.z, xb.w);
+#pragma unroll
+    for (int j = 0; j < NB; ++j) mma_16816(A.c[j], al[0], ah[0], al[1], ah[1], xb[j].x, xb[j].y);
+#pragma unroll
+    for (int j = 0; j < NB; ++j) mma_16816(A.c[j], al[2], ah[2], al[3], ah[3], xb[j].z, xb[j].w);
   }
 }
 
@@ -180,27 +199,27 @@ __device__ __forceinline__ void gv_load_first(GvFrag (&f)[D], int ng, const uint
 }
 
 // Slots U.. of a step whose groups and refills all exist (no checks).
-template <int D, int U>
+template <int D, int U, int NB>
 __device__ __forceinline__ void gv_step_full(GvFrag (&f)[D], const uint8_t* pw, const uint16_t* ps,
-                                             const uint8_t* pz, const uint16_t* xg, float (&acc)[4]) {
+                                             const uint8_t* pz, const uint16_t* xg, GvAcc<NB>& acc) {
   if constexpr (U < D) {
     gv_consume(f[U], xg + U * kGroup, acc);
     gv_load<U + D>(f[U], pw, ps, pz);
-    gv_step_full<D, U + 1>(f, pw, ps, pz, xg, acc);
+    gv_step_full<D, U + 1, NB>(f, pw, ps, pz, xg, acc);
   }
 }
 
 // Slots U.. of one step of D groups starting at group i0: consume group
 // i0 + U from slot U, refill the slot with group i0 + U + D.
-template <int D, int U>
+template <int D, int U, int NB>
 __device__ __forceinline__ void gv_step(GvFrag (&f)[D], int i0, int ng, const uint8_t* pw,
                                         const uint16_t* ps, const uint8_t* pz, const uint16_t* xg,
-                                        float (&acc)[4]) {
+                                        GvAcc<NB>& acc) {
   if constexpr (U < D) {
     if (i0 + U < ng) {
       gv_consume(f[U], xg + U * kGroup, acc);
       if (i0 + U + D < ng) gv_load<U + D>(f[U], pw, ps, pz);
-      gv_step<D, U + 1>(f, i0, ng, pw, ps, pz, xg, acc);
+      gv_step<D, U + 1, NB>(f, i0, ng, pw, ps, pz, xg, acc);
     }
   }
 }
@@ -288,8 +307,12 @@ template <int NT, int kEpi, int KW, bool kNorm>
 __global__ void __launch_bounds__(kGvThreads, kGvCtasPerSm)
 gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
             const uint8_t* __restrict__ z_p, const uint16_t* __restrict__ X,
-            uint16_t* __restrict__ Y, int M, int K, uint32_t cl_magic, int early, OutMap om, NormIn nin) {
+            uint16_t* __restrict__ Y, int M, int K, uint32_t cl_magic, int early, OutMap om, NormIn nin,
+            int ntok) {
   extern __shared__ __align__(128) uint8_t smem[];
+  // Tokens present: NT, or 9..NT for the two-block kernel (ntok).  X rows
+  // past them are neither read nor staged and their outputs not stored.
+  const int nt = NT > 8 ? ntok : NT;
   // Grid (row-block parts, cl): the cluster spans y, so blockIdx.y is the
   // CTA's rank along K and blockIdx.x its part of a row block; n / cl is
   // the high word of n * ceil(2^32 / cl) (exact for n < 2^32 / cl^2).
@@ -341,7 +364,7 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
       for (int p = threadIdx.x; p < pieces; p += kGvThreads)
         cp_async16(xs + p * 8, X + (size_t)ga * kGroup + p * 8);
     } else {
-      for (int idx = threadIdx.x; idx < NT * pieces; idx += kGvThreads) {
+      for (int idx = threadIdx.x; idx < nt * pieces; idx += kGvThreads) {
         const int n = idx / pieces, p = idx - n * pieces;
         cp_async16(xs + n * xstride + p * 8, X + (size_t)n * K + (size_t)ga * kGroup + p * 8);
       }
@@ -364,33 +387,43 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
 
-  // Lanes of tokens g >= NT read token NT - 1: MMA columns are independent,
-  // and those columns are never stored.
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  const uint16_t* xg = xs + (g < NT ? g : NT - 1) * xstride + 32 * c + gw0 * kGroup;
+  // Lane g's MMA column is token g of each block of 8; lanes of tokens
+  // >= NT read token NT - 1: MMA columns are independent, and those columns
+  // are never stored.
+  constexpr int kNB = NT > 8 ? 2 : 1;
+  GvAcc<kNB> acc;
+#pragma unroll
+  for (int j = 0; j < kNB; ++j) {
+    acc.c[j][0] = acc.c[j][1] = acc.c[j][2] = acc.c[j][3] = 0.f;
+    acc.xoff[j] = (min(8 * j + g, nt - 1) - min(g, nt - 1)) * xstride;
+  }
+  const uint16_t* xg = xs + min(g, nt - 1) * xstride + 32 * c + gw0 * kGroup;
   int i0 = 0;
   for (; i0 + 2 * kDepth <= ngw; i0 += kDepth) {   // every refill exists
-    gv_step_full<kDepth, 0>(f, pw, ps, pz, xg, acc);
+    gv_step_full<kDepth, 0, kNB>(f, pw, ps, pz, xg, acc);
     pw += kDepth * kGvWBytes;
     ps += kDepth * kRowBlock;
     pz += kDepth * (kRowBlock / 2);
     xg += kDepth * kGroup;
   }
   for (; i0 < ngw; i0 += kDepth) {
-    gv_step<kDepth, 0>(f, i0, ngw, pw, ps, pz, xg, acc);
+    gv_step<kDepth, 0, kNB>(f, i0, ngw, pw, ps, pz, xg, acc);
     pw += kDepth * kGvWBytes;
     ps += kDepth * kRowBlock;
     pz += kDepth * (kRowBlock / 2);
     xg += kDepth * kGroup;
   }
-  // Accumulator fragment: MMA rows g (entries 0, 1: block row rl) and g + 8
-  // (entries 2, 3: block row rl + 1), tokens 2 c and 2 c + 1.
+  // Accumulator fragment j: MMA rows g (entries 0, 1: block row rl) and
+  // g + 8 (entries 2, 3: block row rl + 1), tokens 8 j + 2 c and 8 j + 2 c + 1.
 #pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    const int n = 2 * c + e;
-    if (n < NT) {
-      red[(ks * NT + n) * kRowBlock + rl] = acc[e];
-      red[(ks * NT + n) * kRowBlock + rl + 1] = acc[2 + e];
+  for (int j = 0; j < kNB; ++j) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int n = 8 * j + 2 * c + e;
+      if (n < nt) {
+        red[(ks * NT + n) * kRowBlock + rl] = acc.c[j][e];
+        red[(ks * NT + n) * kRowBlock + rl + 1] = acc.c[j][2 + e];
+      }
     }
   }
   __syncthreads();
@@ -446,14 +479,17 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
     // Threads 0 .. kRows - 1 are whole warps here: the gate/up pairing
     // shuffles within 32-row groups, which a CTA's rows never split.
 #pragma unroll
-    for (int n = 0; n < NT; ++n) store_gate_up(om, b, r, n, tot[n], true);
+    for (int n = 0; n < NT; ++n)
+      if (n < nt) store_gate_up(om, b, r, n, tot[n], true);
   } else if (m < M) {
     if constexpr (kEpi == kEpiQkv) {
 #pragma unroll
-      for (int n = 0; n < NT; ++n) store_row(dst, om.bias != nullptr, n, tot[n]);
+      for (int n = 0; n < NT; ++n)
+        if (n < nt) store_row(dst, om.bias != nullptr, n, tot[n]);
     } else {
 #pragma unroll
-      for (int n = 0; n < NT; ++n) Y[(size_t)n * M + m] = __half_as_ushort(__float2half_rn(tot[n]));
+      for (int n = 0; n < NT; ++n)
+        if (n < nt) Y[(size_t)n * M + m] = __half_as_ushort(__float2half_rn(tot[n]));
     }
   }
 }
@@ -461,7 +497,7 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
 template <int NT, int kEpi, int KW, bool kNorm = false>
 cudaError_t launch_nt(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p, const uint16_t* X,
                       uint16_t* Y, int M, int K, int cl, bool pdl, cudaStream_t stream, const OutMap& om,
-                      const NormIn& nin) {
+                      const NormIn& nin, int ntok) {
   static std::atomic<unsigned long long> smem_set{0};
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(gemv_kernel<NT, kEpi, KW, kNorm>), kGvSmemLimit,
                                     smem_set);
@@ -485,32 +521,35 @@ cudaError_t launch_nt(const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p
   cfg.numAttrs = pdl ? 2 : 1;
   const uint32_t cl_magic = cl > 1 ? (uint32_t)((0x100000000ull + (unsigned)cl - 1) / (unsigned)cl) : 0u;
   return cudaLaunchKernelEx(&cfg, gemv_kernel<NT, kEpi, KW, kNorm>, wq, s_p, z_p, X, Y, M, K, cl_magic,
-                            pdl ? 1 : 0, om, nin);
+                            pdl ? 1 : 0, om, nin, ntok);
 }
 
 template <int kEpi, int KW, bool kNorm>
 cudaError_t launch_kw(int nt, const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p, const uint16_t* X,
                       uint16_t* Y, int M, int K, int cl, bool pdl, cudaStream_t stream, const OutMap& om,
                       const NormIn& nin) {
+  if constexpr (!kNorm)
+    if (nt > 8) return launch_nt<16, kEpi, KW, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin, nt);
   switch (nt) {
-    case 1: return launch_nt<1, kEpi, KW, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
-    case 2: return launch_nt<2, kEpi, KW, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
-    case 3: return launch_nt<3, kEpi, KW, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
-    case 4: return launch_nt<4, kEpi, KW, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
-    case 5: return launch_nt<5, kEpi, KW, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
-    case 6: return launch_nt<6, kEpi, KW, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
-    case 7: return launch_nt<7, kEpi, KW, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
-    default: return launch_nt<8, kEpi, KW, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
+    case 1: return launch_nt<1, kEpi, KW, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin, nt);
+    case 2: return launch_nt<2, kEpi, KW, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin, nt);
+    case 3: return launch_nt<3, kEpi, KW, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin, nt);
+    case 4: return launch_nt<4, kEpi, KW, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin, nt);
+    case 5: return launch_nt<5, kEpi, KW, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin, nt);
+    case 6: return launch_nt<6, kEpi, KW, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin, nt);
+    case 7: return launch_nt<7, kEpi, KW, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin, nt);
+    default: return launch_nt<8, kEpi, KW, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin, nt);
   }
 }
 
-// One launch of nt tokens (1..8) with row split kw (1, 2, or 4 at nt = 1).
+// One launch of nt tokens (1..16; 9..16 as the 16-token kernel, whose extra
+// columns repeat the last token) with row split kw (1, 2, or 4 at nt = 1).
 template <int kEpi, bool kNorm = false>
 cudaError_t launch_epi(int nt, int kw, const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p,
                        const uint16_t* X, uint16_t* Y, int M, int K, int cl, bool pdl, cudaStream_t stream,
                        const OutMap& om, const NormIn& nin) {
   if (kw == 4 && nt == 1)   // the chooser takes KW = 4 for one token only
-    return launch_nt<1, kEpi, 4, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
+    return launch_nt<1, kEpi, 4, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin, 1);
   if (kw == 2) return launch_kw<kEpi, 2, kNorm>(nt, wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
   return launch_kw<kEpi, 1, kNorm>(nt, wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
 }
@@ -555,9 +594,16 @@ GvShape gemv_shape(int M, int K, int sms, int nt) {
       for (int i = 0; i < 4; ++i) best_key[i] = key[i];
     }
   };
+  const int ntk = nt > 8 ? kGemvWideTokens : nt;   // tokens the launched kernel stages
   auto fits = [&](int kw, int cl) {
-    return nt * gv_xstride(ceil_div(kg, cl)) * 2 <= kMaxXSmem &&
-           gv_layout(nt, ceil_div(kg, cl), cl, kw).total <= kGvSmemLimit;
+    return ntk * gv_xstride(ceil_div(kg, cl)) * 2 <= kMaxXSmem &&
+           gv_layout(ntk, ceil_div(kg, cl), cl, kw).total <= kGvSmemLimit;
+  };
+  // CTAs one SM holds: the register budget, or fewer when the activation
+  // slice and the partial sums fill its shared memory.
+  auto wave_of = [&](int kw, int cl) {
+    const int smem = gv_layout(ntk, ceil_div(kg, cl), cl, kw).total;
+    return (long long)std::min(kGvCtasPerSm, kSmemPerSm / (smem + kSmemPerCta)) * sms;
   };
   auto load = [&](int kw, int cl) {
     const long long ctas = (long long)blocks * kw * cl;
@@ -569,7 +615,7 @@ GvShape gemv_shape(int M, int K, int sms, int nt) {
     for (int cl = 1; cl <= kMaxCluster && cl <= kg; ++cl) {
       if (!fits(kw, cl)) continue;
       const long long ctas = (long long)blocks * kw * cl;
-      if ((kw > 1 || cl > 1) && ctas > wave) continue;
+      if ((kw > 1 || cl > 1) && ctas > wave_of(kw, cl)) continue;
       const bool dense = 2 * ctas >= 5LL * sms;
       const long long key[4] = {dense ? 0 : 1, dense ? load(kw, cl) : -ctas, -kw, cl};
       consider(kw, cl, key);
@@ -582,7 +628,8 @@ GvShape gemv_shape(int M, int K, int sms, int nt) {
   // the smallest cluster whose slice fits, over several waves.
   for (int cl = 1; cl <= kMaxCluster && cl <= kg; ++cl)
     if (fits(1, cl)) return GvShape{1, cl};
-  return GvShape{1, kMaxCluster};
+  return GvShape{0, 0};   // no launch of this many tokens fits
+
 }
 
 cudaError_t launch_gemv(const uint8_t* wq, const uint16_t* scales, const uint8_t* zeros,
@@ -590,11 +637,25 @@ cudaError_t launch_gemv(const uint8_t* wq, const uint16_t* scales, const uint8_t
                         cudaStream_t stream, const OutMap* om, bool pdl, const NormIn* norm) {
   if (norm && (N > kGemvMaxTokens || !om || om->kind != kEpiQkv)) return cudaErrorNotSupported;
   const NormIn nin = norm ? *norm : NormIn{};
-  for (int n0 = 0; n0 < N; n0 += kGemvMaxTokens) {
-    const int nt = std::min(kGemvMaxTokens, N - n0);
-    const GvShape sh = gemv_shape(M, K, num_sms(), nt);
+  // 9..16 tokens as one two-block launch on weights of up to kWideMaxM rows
+  // (N = 9 / 16 on O 4096 x 4096: 8.2 / 8.5 against 11.3 / 12.5 us for
+  // 8-token launches; taller weights ran slower that way: QKV 12288 x 4096
+  // 17.9 against 17.4 us on the tile kernel, LLaMA-3 gate/up 28672 x 4096
+  // 40.7 against 31.2 us); 8-token launches otherwise.
+  const int per_launch = norm || M > kWideMaxM ? kGemvMaxTokens : kGemvWideTokens;
+  for (int n0 = 0; n0 < N;) {
+    int nt = std::min(per_launch, N - n0);
+    GvShape sh = gemv_shape(M, K, num_sms(), nt);
+    // A wide K leaves no room for 16 tokens' activations and partial sums in
+    // one CTA: 8-token launches then.
+    if (sh.cl == 0 && nt > kGemvMaxTokens) {
+      nt = kGemvMaxTokens;
+      sh = gemv_shape(M, K, num_sms(), nt);
+    }
+    if (sh.cl == 0) return cudaErrorNotSupported;
+    const int ntk = nt > 8 ? kGemvWideTokens : nt;   // tokens the launched kernel stages
     const int cl = sh.cl;
-    if (nt * gv_xstride(ceil_div(K / kGroup, cl)) * 2 > kMaxXSmem) return cudaErrorNotSupported;
+    if (ntk * gv_xstride(ceil_div(K / kGroup, cl)) * 2 > kMaxXSmem) return cudaErrorNotSupported;
     const uint16_t* Xn = X ? X + (size_t)n0 * K : nullptr;
     uint16_t* Yn = om ? nullptr : Y + (size_t)n0 * M;
     // The fused outputs of tokens n0 .. n0 + nt - 1: each segment moves by
@@ -621,6 +682,7 @@ cudaError_t launch_gemv(const uint8_t* wq, const uint16_t* scales, const uint8_t
     else
       e = launch_epi<kEpiPlain>(nt, sh.kw, wq, scales, zeros, Xn, Yn, M, K, cl, pdl, stream, on, nin);
     if (e != cudaSuccess) return e;
+    n0 += nt;
   }
   return cudaSuccess;
 }

@@ -278,6 +278,10 @@ inline cudaError_t ensure_smem_limit(const void* fn, int bytes, std::atomic<unsi
 
 // GEMV (CUDA cores): N in 1..kGemvMaxTokens per launch.
 constexpr int kGemvMaxTokens = 8;
+// Tokens of one plain / QKV / gate-up launch: 9 to 16 run as two 8-token
+// MMA column blocks sharing the dequantised weights (the normalising
+// prologue keeps kGemvMaxTokens).
+constexpr int kGemvWideTokens = 16;
 
 // om: null for the plain [N][M] output Y, else the fused output map (Y unused).
 // With pdl the launch may overlap the previous kernel in the stream: the

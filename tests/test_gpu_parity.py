@@ -106,10 +106,19 @@ def test_ragged_shapes(M, K, N, path):
 
 @pytest.mark.parametrize("N", list(range(1, 18)))
 def test_gemv_every_token_count(N):
-    """Every token count of one CUDA-core decode launch (1..8, the eight
+    """Every token count of one 8-token decode launch (1..8, the eight
     columns of its MMA tile), then two launches (9..16) and a third (17), on
-    a shape with a ragged row block and a K split across a cluster."""
-    full_case(1500, 2048, N, w4a16.PATH_GEMV, seed=300 + N)
+    a weight taller than 4096 rows with a ragged row block."""
+    full_case(4200, 2048, N, w4a16.PATH_GEMV, seed=300 + N)
+
+
+@pytest.mark.parametrize("N", list(range(9, 34)))
+def test_gemv_two_block_launches(N):
+    """Weights of at most 4096 rows take 9..16 tokens in one launch of two
+    8-token MMA column blocks sharing the dequantised weights: every count
+    9..16, then two launches (17..32) and a third (33), on a ragged row block
+    with a K split across a cluster."""
+    full_case(1000, 2048, N, w4a16.PATH_GEMV, seed=400 + N)
 
 
 @pytest.mark.parametrize("path", PATHS, ids=lambda p: PATH_NAMES[p])
