@@ -55,7 +55,7 @@ typedef enum {
     W4A16_PATH_AUTO = 0,     /* choose by N and M: GEMV for N <= 8, and for N <= 16
                                 when M <= 8192; TC above */
     W4A16_PATH_GEMV = 1,     /* decode kernel: weights streamed to registers, warp-level
-                                MMAs (any N, 8 tokens per launch) */
+                                MMAs (any N; 8 tokens per launch, 16 when M <= 4096) */
     W4A16_PATH_TC = 2,       /* tcgen05 tile kernel (any N) */
     W4A16_PATH_GEMV_TC = 3   /* tcgen05 decode kernel, weight stream split over every SM
                                 (N <= 64; needs a workspace; never chosen by AUTO: slower
