@@ -28,7 +28,9 @@
 //    about 2.5 instructions per weight, 1.6 of them the exact dequant;
 //  * split-K: CTAs of a thread-block cluster (up to 8 along K) reduce through
 //    distributed shared memory into the cluster's rank-0 CTA in a fixed order
-//    (deterministic, no atomics).
+//    (deterministic, no atomics); the other ranks store their partial sums,
+//    arrive on an mbarrier of rank 0 and leave at once, rank 0 waiting on it
+//    (bounded).
 #include "w4a16_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -36,8 +38,8 @@
 
 namespace w4a16 {
 
-// Status word of the decode kernel's family.  The kernel has no waits, so it
-// stays 0; it is kept so every kernel family reports through the same call.
+// Status word of the decode kernel's family: set when rank 0 of a cluster
+// gives up waiting for the other ranks' partial sums (a bounded wait).
 __device__ int g_gemv_status = 0;
 
 namespace {
@@ -344,7 +346,14 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   const int ngw = ((ks + 1) * ng) / KW - gw0;
 
   ptx::griddep_launch_dependents();
-  if (cl > 1) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+  __shared__ __align__(8) uint64_t s_done;
+  if (cl > 1) {
+    if (crank == 0 && threadIdx.x == 0) {
+      ptx::mbar_init(&s_done, (uint32_t)((cl - 1) * kRows));
+      ptx::fence_mbar_init();
+    }
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+  }
 
   // This lane's rows within the block: MMA rows g and g + 8 of the warp's
   // tile are the adjacent block rows rl and rl + 1.  Its group streams
@@ -449,21 +458,41 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   }
 
   if (cl > 1) {
-    // Every CTA of the cluster has started once this wait returns, so its
-    // shared memory may be written remotely.
+    // Every CTA of the cluster has started once this wait returns, so rank
+    // 0's shared memory and its arrival barrier may be used remotely.
     asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-    if (rr < kRows) {
+    if (rr >= kRows) return;
 #pragma unroll
-      for (int n = 0; n < NT; ++n) {
-        const uint32_t local = ptx::smem_addr(&cred[(crank * NT + n) * kRowBlock + r]);
-        uint32_t remote;
-        asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(0));
-        asm volatile("st.shared::cluster.f32 [%0], %1;" :: "r"(remote), "f"(tot[n]) : "memory");
+    for (int n = 0; n < NT; ++n) {
+      const uint32_t local = ptx::smem_addr(&cred[(crank * NT + n) * kRowBlock + r]);
+      uint32_t remote;
+      asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(0));
+      asm volatile("st.shared::cluster.f32 [%0], %1;" :: "r"(remote), "f"(tot[n]) : "memory");
+    }
+    if (crank != 0) {
+      // The other ranks announce their partial sums on rank 0's barrier
+      // (release at cluster scope orders the stores above) and leave.
+      uint32_t rbar;
+      asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rbar) : "r"(ptx::smem_addr(&s_done)), "r"(0));
+      asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" :: "r"(rbar) : "memory");
+      return;
+    }
+    // Rank 0: a bounded wait for every other rank's rows.
+    {
+      const long long t0 = clock64();
+      while (true) {
+        uint32_t ok;
+        asm volatile("{\n\t.reg .pred p;\n\t"
+                     "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], 0, 200000;\n\t"
+                     "selp.u32 %0, 1, 0, p;\n\t}"
+                     : "=r"(ok) : "r"(ptx::smem_addr(&s_done)) : "memory");
+        if (ok) break;
+        if (clock64() - t0 > kWaitLimitCycles) {
+          atomicExch(&g_gemv_status, 1);
+          return;
+        }
       }
     }
-    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-    if (crank != 0 || rr >= kRows) return;
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
       float sum = 0.f;
