@@ -79,7 +79,7 @@ def test_pack_order_matches_the_documented_interleave():
 
 @pytest.mark.parametrize("path", [GEMV, TC, GT, w4a16.PATH_AUTO], ids=lambda p: NAMES[p])
 @pytest.mark.parametrize("Mi,K,N", [(128, 256, 1), (200, 384, 2), (37, 128, 3), (1000, 1024, 5),
-                                    (64, 512, 16), (4104, 2048, 9)])
+                                    (64, 512, 16), (1000, 1024, 11), (4104, 2048, 9)])
 def test_gate_up_small_full(Mi, K, N, path):
     p = synth.make_problem(2 * Mi, K, N, seed=Mi + K + N)
     w, x = _packed(p)

@@ -284,7 +284,8 @@ def test_quantize_pack_gemm_pipeline():
 # ------------------------------------------------- fused QKV split + bias ----
 
 @pytest.mark.parametrize("splits,K,N", [((200, 72, 72), 384, 1), ((200, 72, 72), 384, 2),
-                                        ((200, 72, 72), 384, 5), ((128, 64, 64), 256, 130),
+                                        ((200, 72, 72), 384, 5), ((200, 72, 72), 384, 12),
+                                        ((128, 64, 64), 256, 130),
                                         ((4096, 1024, 1024), 4096, 1), ((4096, 1024, 1024), 4096, 16)])
 def test_gemm_qkv_split_and_bias(splits, K, N):
     """Three outputs = the plain product's column ranges bit for bit without
