@@ -51,7 +51,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # capture of this repository's kernel; it holds only while the kernel source
 # is the one captured (sha256 prefix of csrc/w4a16_gemv.cu), and the bench
 # reports null otherwise.
-DECODE_TRAFFIC = {"src_sha256_prefix": "fa7640bda3adc753", "qkv_dram_bytes": 26184704, "qkv_alg_bytes": 26181632}
+DECODE_TRAFFIC = {"src_sha256_prefix": "ad06eac62b9462f1", "qkv_dram_bytes": 26184704, "qkv_alg_bytes": 26181632}
 NOMINAL_DENSE_FP16_TFLOPS = 2250.0   # B200 dense fp16/bf16 tensor rate, NVIDIA's figure
 
 
@@ -461,7 +461,7 @@ def main_ours(args):
     torch.cuda.set_device(device)
     dist = dist_init("nccl") if world > 1 else None
     if rank == 0:
-        lib_build.build()
+        lib_build.build(debug=False)
     if dist is not None:
         dist.barrier()
     w4a16.lib()

@@ -193,6 +193,7 @@ const char* w4a16_status_string(int status) {
     case W4A16_ERR_MISALIGNED: return "pointer not 16-byte aligned";
     case W4A16_ERR_CUDA: return "CUDA error";
     case W4A16_ERR_TIMEOUT: return "device wait timed out";
+    case W4A16_ERR_BOUNDS: return "in-kernel index check failed (debug build)";
     default: return "unknown status";
   }
 }
@@ -501,7 +502,12 @@ w4a16_status w4a16_device_status(void* stream, int* status) {
   if (e == cudaSuccess) e = read_and_clear_gemv_status(&b);
   if (e == cudaSuccess) e = read_and_clear_gvtc_status(&c);
   if (e != cudaSuccess) return map_cuda(e);
-  *status = (a || b || c) ? W4A16_ERR_TIMEOUT : W4A16_OK;
+  // The decode kernel's word: 1 = a cluster wait gave up, 2 = (debug build)
+  // an index check failed; the other families record timeouts only.
+  if (a || c || b == 1)
+    *status = W4A16_ERR_TIMEOUT;
+  else
+    *status = b ? W4A16_ERR_BOUNDS : W4A16_OK;
   return W4A16_OK;
 }
 

@@ -125,10 +125,41 @@ struct GvFrag {
   uint32_t s, z;
 };
 
+#ifdef W4A16_DEBUG_BOUNDS
+// Index-check build: the extent of every buffer the CTA touches, set by
+// thread 0 before any access.  A failed check records 2 in the status word
+// (w4a16_device_status: W4A16_ERR_BOUNDS) and the access is skipped.
+struct GvChk {
+  const uint8_t *w0, *w1;     // packed codes
+  const uint16_t *s0, *s1;    // packed scales
+  const uint8_t *z0, *z1;     // packed zeros
+  const uint16_t *x0, *x1;    // this launch's activations (global)
+  const uint16_t *xs0, *xs1;  // the staged activation slice (shared)
+  int red_n, cred_n;          // floats of the two partial-sum regions
+};
+__shared__ GvChk g_chk;
+
+__device__ __forceinline__ bool gv_ok(bool ok) {
+  if (!ok) atomicExch(&g_gemv_status, 2);
+  return ok;
+}
+#endif
+
 // Group J of the lane's streams: pw points at chunk c of row r of group 0,
 // ps at the scale of row r, pz at the zero byte of rows r and r + 1.
 template <int J>
 __device__ __forceinline__ void gv_load(GvFrag& f, const uint8_t* pw, const uint16_t* ps, const uint8_t* pz) {
+#ifdef W4A16_DEBUG_BOUNDS
+  const uint8_t* w = pw + J * kGvWBytes;
+  const uint16_t* sp = ps + J * kRowBlock;
+  const uint8_t* zp = pz + J * (kRowBlock / 2);
+  if (!gv_ok(w >= g_chk.w0 && w + 32 <= g_chk.w1 && sp >= g_chk.s0 && sp + 2 <= g_chk.s1 && zp >= g_chk.z0 &&
+             zp + 1 <= g_chk.z1)) {
+    f.lo = f.hi = make_uint4(0u, 0u, 0u, 0u);
+    f.s = f.z = 0u;
+    return;
+  }
+#endif
   f.lo = ldg_v4_at<J * kGvWBytes>(pw);
   f.hi = ldg_v4_at<J * kGvWBytes + 16>(pw);
   f.s = ldg_u32_at<J * kRowBlock * 2>(ps);
@@ -180,7 +211,13 @@ __device__ __forceinline__ void gv_consume(const GvFrag& f, const uint16_t* xg, 
   for (int t = 0; t < 4; ++t) {
     uint4 xb[NB];
 #pragma unroll
-    for (int j = 0; j < NB; ++j) xb[j] = *reinterpret_cast<const uint4*>(xg + A.xoff[j] + 8 * t);
+    for (int j = 0; j < NB; ++j) {
+      const uint16_t* xp = xg + A.xoff[j] + 8 * t;
+#ifdef W4A16_DEBUG_BOUNDS
+      if (!gv_ok(xp >= g_chk.xs0 && xp + 8 <= g_chk.xs1)) xp = g_chk.xs0;
+#endif
+      xb[j] = *reinterpret_cast<const uint4*>(xp);
+    }
     uint32_t al[4], ah[4];
     dequant_word(wl[t], clo, al);
     dequant_word(wh[t], chi, ah);
@@ -346,6 +383,25 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   const int ngw = ((ks + 1) * ng) / KW - gw0;
 
   ptx::griddep_launch_dependents();
+#ifdef W4A16_DEBUG_BOUNDS
+  if (threadIdx.x == 0) {
+    const size_t blocks_all = (size_t)ceil_div(M, kRowBlock);
+    g_chk.w0 = wq;
+    g_chk.w1 = wq + blocks_all * kc_n * kRowBlock * 16;
+    g_chk.s0 = s_p;
+    g_chk.s1 = s_p + blocks_all * kg * kRowBlock;
+    g_chk.z0 = z_p;
+    g_chk.z1 = z_p + blocks_all * kg * (kRowBlock / 2);
+    g_chk.x0 = X;
+    g_chk.x1 = X ? X + (size_t)nt * K : X;
+    const uint16_t* xs_base = reinterpret_cast<const uint16_t*>(smem + L.x_off);
+    g_chk.xs0 = xs_base;
+    g_chk.xs1 = xs_base + NT * xstride;
+    g_chk.red_n = KW * NT * kRowBlock;
+    g_chk.cred_n = cl > 1 ? cl * NT * kRowBlock : 0;
+  }
+  __syncthreads();
+#endif
   __shared__ __align__(8) uint64_t s_done;
   if (cl > 1) {
     if (crank == 0 && threadIdx.x == 0) {
@@ -370,11 +426,20 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
   auto stage_x = [&]() {
     const int pieces = ng * (kGroup / 8);
     if constexpr (NT == 1) {
-      for (int p = threadIdx.x; p < pieces; p += kGvThreads)
+      for (int p = threadIdx.x; p < pieces; p += kGvThreads) {
+#ifdef W4A16_DEBUG_BOUNDS
+        const uint16_t* src = X + (size_t)ga * kGroup + p * 8;
+        if (!gv_ok(src >= g_chk.x0 && src + 8 <= g_chk.x1 && xs + p * 8 + 8 <= g_chk.xs1)) continue;
+#endif
         cp_async16(xs + p * 8, X + (size_t)ga * kGroup + p * 8);
+      }
     } else {
       for (int idx = threadIdx.x; idx < nt * pieces; idx += kGvThreads) {
         const int n = idx / pieces, p = idx - n * pieces;
+#ifdef W4A16_DEBUG_BOUNDS
+        const uint16_t* src = X + (size_t)n * K + (size_t)ga * kGroup + p * 8;
+        if (!gv_ok(src >= g_chk.x0 && src + 8 <= g_chk.x1 && xs + n * xstride + p * 8 + 8 <= g_chk.xs1)) continue;
+#endif
         cp_async16(xs + n * xstride + p * 8, X + (size_t)n * K + (size_t)ga * kGroup + p * 8);
       }
     }
@@ -430,6 +495,9 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
     for (int e = 0; e < 2; ++e) {
       const int n = 8 * j + 2 * c + e;
       if (n < nt) {
+#ifdef W4A16_DEBUG_BOUNDS
+        if (!gv_ok((ks * NT + n) * kRowBlock + rl + 1 < g_chk.red_n)) continue;
+#endif
         red[(ks * NT + n) * kRowBlock + rl] = acc.c[j][e];
         red[(ks * NT + n) * kRowBlock + rl + 1] = acc.c[j][2 + e];
       }
@@ -464,6 +532,9 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
     if (rr >= kRows) return;
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
+#ifdef W4A16_DEBUG_BOUNDS
+      if (!gv_ok((crank * NT + n) * kRowBlock + r < g_chk.cred_n)) continue;
+#endif
       const uint32_t local = ptx::smem_addr(&cred[(crank * NT + n) * kRowBlock + r]);
       uint32_t remote;
       asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(0));
@@ -518,7 +589,12 @@ gemv_kernel(const uint8_t* __restrict__ wq, const uint16_t* __restrict__ s_p,
     } else {
 #pragma unroll
       for (int n = 0; n < NT; ++n)
-        if (n < nt) Y[(size_t)n * M + m] = __half_as_ushort(__float2half_rn(tot[n]));
+        if (n < nt) {
+#ifdef W4A16_DEBUG_BOUNDS
+          if (!gv_ok(m < M)) continue;
+#endif
+          Y[(size_t)n * M + m] = __half_as_ushort(__float2half_rn(tot[n]));
+        }
     }
   }
 }

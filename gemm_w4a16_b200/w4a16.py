@@ -6,6 +6,7 @@ missing the calls raise; there is no fallback of any kind.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import threading
@@ -13,8 +14,9 @@ from dataclasses import dataclass
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libw4a16.so")
+DEBUG_LIB_PATH = os.path.join(HERE, "libw4a16_debug.so")   # the index-check build (-DW4A16_DEBUG_BOUNDS)
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_CUDA, ERR_TIMEOUT = range(6)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED, ERR_CUDA, ERR_TIMEOUT, ERR_BOUNDS = range(7)
 PATH_AUTO, PATH_GEMV, PATH_TC, PATH_GEMV_TC = 0, 1, 2, 3
 FLAG_EARLY_WEIGHTS = 1
 GEMV_TC_MAX_TOKENS = 64      # forced W4A16_PATH_GEMV_TC
@@ -101,6 +103,22 @@ def lib():
             L.w4a16_selftest_wait_timeout.restype = _i
             _lib = L
     return _lib
+
+
+@contextlib.contextmanager
+def library(path: str):
+    """Route every call made in the block through the library at `path`
+    (DEBUG_LIB_PATH: the same API with the decode kernel's index checks),
+    then go back to the previous one."""
+    global LIB_PATH, _lib
+    with _lock:
+        saved = (LIB_PATH, _lib)
+        LIB_PATH, _lib = path, None
+    try:
+        yield
+    finally:
+        with _lock:
+            LIB_PATH, _lib = saved
 
 
 def status_string(status: int) -> str:

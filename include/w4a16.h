@@ -47,7 +47,10 @@ typedef enum {
     W4A16_ERR_UNSUPPORTED = 2,  /* group != 128, K % 128 != 0, sizes too big */
     W4A16_ERR_MISALIGNED = 3,   /* a pointer is not 16-byte aligned */
     W4A16_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
-    W4A16_ERR_TIMEOUT = 5       /* a bounded device-side wait ran out */
+    W4A16_ERR_TIMEOUT = 5,      /* a bounded device-side wait ran out */
+    W4A16_ERR_BOUNDS = 6        /* libw4a16_debug.so only (built with -DW4A16_DEBUG_BOUNDS):
+                                   an in-kernel index check of the decode kernel found an
+                                   access outside its buffer; the access was skipped */
 } w4a16_status;
 
 /* Kernel selection for w4a16_gemm_ex and w4a16_gemm_ws. */
@@ -379,7 +382,8 @@ W4A16_API w4a16_status w4a16_dequant_debug(const void* wq_packed, const void* sc
 /*
  * Synchronises `stream`, then reads and clears the device-side status words
  * that bounded waits inside the kernels set when they give up.
- * Writes W4A16_OK or W4A16_ERR_TIMEOUT to *status.  Not for the hot path.
+ * Writes W4A16_OK, W4A16_ERR_TIMEOUT or (debug build) W4A16_ERR_BOUNDS to
+ * *status.  Not for the hot path.
  * The words are per device, shared by every stream, and read and cleared by
  * two separate copies: the answer is exact only while no other stream runs
  * this library's kernels on the device (a timeout recorded between the two

@@ -36,8 +36,18 @@ def test_exports_every_declared_symbol(L):
         assert hasattr(L, n), n
 
 
+def test_debug_library_exports_the_same_symbols(L):
+    """The index-check build (libw4a16_debug.so) is the same API."""
+    import ctypes
+
+    assert os.path.exists(w4a16.DEBUG_LIB_PATH)
+    D = ctypes.CDLL(w4a16.DEBUG_LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(D, n), n
+
+
 def test_status_strings(L):
-    for code in range(6):
+    for code in range(7):
         assert w4a16.status_string(code)
     assert w4a16.status_string(99) == "unknown status"
 
