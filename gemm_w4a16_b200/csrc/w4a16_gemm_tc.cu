@@ -507,12 +507,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
           if (lane == 0) ptx::mbar_arrive(&sh.acc_empty[b]);
         }
         if constexpr (kEpi == kEpiGateUp) {
-          // Whole warps: the gate/up pairing shuffles.
+          // Whole warps: the gate/up pairing shuffles, two tokens at a time.
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int n = n0 + 16 * c + j;
-            store_gate_up(om, mt, row, n, sum[j], n < N);
-          }
+          for (int j = 0; j < 16; j += 2) store_gate_up_pair(om, mt, row, n0 + 16 * c + j, sum[j], sum[j + 1], N);
         } else if (m < M) {
 #pragma unroll
           for (int j = 0; j < 16; ++j) {

@@ -253,6 +253,26 @@ __device__ __forceinline__ void store_gate_up(const OutMap& o, int b, int r, int
   }
 }
 
+// The same for two consecutive tokens n and n + 1 (v0, v1: this lane's
+// accumulators of both; tokens >= N are not stored) with every lane busy:
+// a gate lane hands g(n + 1) to its up partner and takes u(n) in one
+// exchange, then writes H[n]; the up lane writes H[n + 1].  Per output the
+// arithmetic is store_gate_up's, so the bits are the same; a warp issues one
+// exchange and one SiLU sequence per two tokens instead of per token.
+__device__ __forceinline__ void store_gate_up_pair(const OutMap& o, int b, int r, int n, float v0, float v1,
+                                                   int N) {
+  const bool up = (r & 16) != 0;
+  const float recv = __shfl_xor_sync(0xffffffffu, up ? v0 : v1, 16);
+  const float g = up ? recv : v0;
+  const float u = up ? v1 : recv;
+  const int nn = up ? n + 1 : n;
+  const int i = gate_up_channel(b, r & ~16);
+  if (nn < N && i < o.mi) {
+    const float silu = __fdividef(g, 1.0f + __expf(-g));
+    o.h[(size_t)nn * o.mi + i] = __half_as_ushort(__float2half_rn(silu * u));
+  }
+}
+
 // ------------------------------------------------------- launch helpers ----
 
 // SM count of the current device (cached per device; 148 if it cannot be read).
