@@ -237,21 +237,32 @@ def run_calls(calls, path=0):
             w4a16.gemm(w, x, Y=y)
 
 
-def capture_e2e(calls, ws, flags, x_flat, y_flat, x_host, y_host, device, chunks=4):
+def capture_e2e(calls, ws, flags, x_flat, y_flat, x_host, y_host, device, sizes=None):
     """One CUDA graph of the decode step with its host traffic pipelined
-    against the kernels: the calls in `chunks` consecutive groups (8 layers
-    each), every group's X copied in from pinned host memory on an H2D
-    stream (all groups queued at once, each group's calls waiting for its
-    own copy) and every group's Y copied out on a D2H stream as soon as the
-    group's calls are done, overlapping the next group's kernels; both
+    against the kernels: the calls in consecutive groups of `sizes` calls
+    (default: the first layer, 15 layers, 15 layers, the last layer, so that
+    only one layer's X waits before the first kernel and one layer's Y
+    after the last), every group's X copied in from pinned host memory on
+    an H2D stream (all groups queued at once, each group's calls waiting for
+    its own copy) and every group's Y copied out on a D2H stream as soon as
+    the group's calls are done, overlapping the next group's kernels; both
     streams join the replay stream before the graph ends."""
     import torch
 
-    per = (len(calls) + chunks - 1) // chunks
+    if sizes is None:
+        per_layer = len(LLAMA7B_LAYER)
+        mid = len(calls) // per_layer - 2
+        if mid < 2:
+            sizes = [len(calls)]
+        else:
+            sizes = [per_layer, per_layer * (mid // 2), per_layer * (mid - mid // 2), per_layer]
+    assert sum(sizes) == len(calls)
     groups = []
     xo = yo = 0
-    for c0 in range(0, len(calls), per):
-        cs = calls[c0:c0 + per]
+    c0 = 0
+    for size in sizes:
+        cs = calls[c0:c0 + size]
+        c0 += size
         xk = sum(w.K for _, w, _, _ in cs)
         ym = sum(w.M for _, w, _, _ in cs)
         groups.append((xo, xo + xk, yo, yo + ym, cs))
@@ -514,7 +525,7 @@ def main_ours(args):
 
     # End to end: every step copies every call's X in from pinned host
     # memory and every Y back out, inside the event-timed region: pipelined
-    # per 8-layer group against the kernels in one graph, and also (reported
+    # per layer group against the kernels in one graph, and also (reported
     # beside it) serialised around the step's graph.
     x_host = torch.empty(x_flat.shape, dtype=x_flat.dtype, pin_memory=True)
     y_host = torch.empty(y_flat.shape, dtype=y_flat.dtype, pin_memory=True)
@@ -577,7 +588,7 @@ def main_ours(args):
                 "h2d_bytes_per_step": int(x_host.numel() * 2),
                 "d2h_bytes_per_step": int(y_host.numel() * 2), "ms_per_step": ms_e2e_max,
                 "api": "w4a16_gemm_ws (128 calls captured in a CUDA graph) + pinned H2D/D2H by torch copy_, "
-                       "per 8-layer group on copy streams overlapping the kernels",
+                       "per layer group (1, 15, 15, 1 layers) on copy streams overlapping the kernels",
                 "serialised": {"value": e2e_serial_value,
                                "ms_per_step": ms_e2e_serial_max,
                                "api": "all X in, the step's graph, all Y out, on one stream"}},
