@@ -349,6 +349,18 @@ def time_steps(g, steps, warmup, device, pre=None, post=None):
     return ev[0].elapsed_time(ev[steps]), per
 
 
+def settle(g, device, ms=25.0):
+    """Replay g for about `ms` milliseconds before a measurement, so that a
+    leg that follows a power-hungry one starts at its steady clocks."""
+    import torch
+
+    t_end = time.time() + ms * 1e-3
+    while time.time() < t_end:
+        for _ in range(4):
+            g.replay()
+        torch.cuda.synchronize(device)
+
+
 def time_graph(g, steps, warmup, device, pre=None, post=None):
     """Mean ms per replay of graph g over `steps` timed replays."""
     total, _ = time_steps(g, steps, warmup, device, pre, post)
@@ -708,7 +720,8 @@ def n_sweep_measure(device, peaks, sampler, copies=16, reps=20):
             flags = w4a16.FLAG_EARLY_WEIGHTS if path != w4a16.PATH_TC else 0
             g = capture(lambda path=path, flags=flags: [w4a16.gemm_ws(w, x, Y=y, path=path, workspace=wsp,
                                                                      flags=flags) for w in ws_copies], device)
-            _, per = time_steps(g, reps, 3, device)
+            settle(g, device)
+            _, per = time_steps(g, reps, 10, device)
             us = pct(per, 1e3 / copies)["median"]
             gbs = alg_bytes(M, K, N) / (us * 1e-6) / 1e9
             tfs = alg_flops(M, K, N) / (us * 1e-6) / 1e12
@@ -746,7 +759,8 @@ def fused_measure(device, peaks, sampler, reps=20):
         for name, fn in fns.items():
             g = capture(fn, device)
             t0 = time.time()
-            _, per = time_steps(g, reps, 3, device)
+            settle(g, device)
+            _, per = time_steps(g, reps, 10, device)
             res[name] = {"us": pct(per, 1e3 / per_graph)["median"], "clocks": sampler.summary(t0, time.time())}
             del g
         return res
@@ -867,7 +881,8 @@ def llama3_measure(device, peaks, sampler, reps=20):
             wsp = w4a16.Workspace(device, w4a16.workspace_size(M, K, N))
             g = capture(lambda: [w4a16.gemm_ws(w, x, Y=y, workspace=wsp, flags=w4a16.FLAG_EARLY_WEIGHTS)
                                  for w in wts], device)
-            _, per = time_steps(g, reps, 3, device)
+            settle(g, device)
+            _, per = time_steps(g, reps, 10, device)
             us = pct(per, 1e3 / copies)["median"]
             gbs = alg_bytes(M, K, N) / (us * 1e-6) / 1e9
             tfs = alg_flops(M, K, N) / (us * 1e-6) / 1e12
