@@ -72,6 +72,8 @@ def build(force: bool = False, verbose: bool = False, extra=None, debug: bool = 
         if proc.returncode != 0:
             sys.stderr.write(out)
             failed.append(os.path.basename(lib))
+            if os.path.exists(tmp):
+                os.remove(tmp)
         else:
             os.replace(tmp, lib)
     if failed:
