@@ -507,16 +507,49 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __rest
           if (lane == 0) ptx::mbar_arrive(&sh.acc_empty[b]);
         }
         if constexpr (kEpi == kEpiGateUp) {
-          // Whole warps: the gate/up pairing shuffles, two tokens at a time.
+          // Whole warps, two tokens at a time with every lane busy: a gate
+          // lane hands g(n + 1) to its up partner (lane ^ 16) and takes u(n)
+          // in one exchange, then writes H[n]; the up lane writes H[n + 1].
+          // Per output the arithmetic is store_gate_up's (the same bits); the
+          // lane's H pointer steps two token rows per pair.
+          const bool up = (row & 16) != 0;
+          const int i = gate_up_channel(mt, row & ~16);
+          const int nb = n0 + 16 * c + (up ? 1 : 0);
+          uint16_t* hp = om.h + (size_t)nb * om.mi + i;
+          const size_t step = 2 * (size_t)om.mi;
 #pragma unroll
-          for (int j = 0; j < 16; j += 2) store_gate_up_pair(om, mt, row, n0 + 16 * c + j, sum[j], sum[j + 1], N);
+          for (int j = 0; j < 16; j += 2) {
+            const float recv = __shfl_xor_sync(0xffffffffu, up ? sum[j] : sum[j + 1], 16);
+            const float g = up ? recv : sum[j];
+            const float u = up ? sum[j + 1] : recv;
+            if (nb + j < N && i < om.mi) {
+              const float silu = __fdividef(g, 1.0f + __expf(-g));
+              *hp = __half_as_ushort(__float2half_rn(silu * u));
+            }
+            hp += step;
+          }
         } else if (m < M) {
+          if constexpr (kEpi == kEpiQkv) {
+            // The row's destination pointer steps by its pitch from token to
+            // token (store_row's arithmetic, without a 64-bit multiply per
+            // element).
+            const int nb = n0 + 16 * c;
+            uint16_t* p = dst.y + (size_t)nb * dst.ld;
+            const bool has_bias = om.bias != nullptr;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int n = n0 + 16 * c + j;
-            if (n < N) {
-              if constexpr (kEpi == kEpiQkv) store_row(dst, om.bias != nullptr, n, sum[j]);
-              else Y[(size_t)n * M + m] = __half_as_ushort(__float2half_rn(sum[j]));
+            for (int j = 0; j < 16; ++j) {
+              if (nb + j < N) {
+                float v = sum[j];
+                if (has_bias) v = __fadd_rn(v, dst.bias);
+                *p = __half_as_ushort(__float2half_rn(v));
+              }
+              p += dst.ld;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int n = n0 + 16 * c + j;
+              if (n < N) Y[(size_t)n * M + m] = __half_as_ushort(__float2half_rn(sum[j]));
             }
           }
         }

@@ -241,35 +241,15 @@ __device__ __forceinline__ void store_row(const RowDst& d, bool has_bias, int n,
 // + 16, then write H[n][i] = fp16_RN(silu(g) * u), silu(g) = g / (1 + e^-g),
 // in fp32 with the hardware exponential and approximate division (a few fp32
 // ulps, far below the one fp16 rounding of H; e^-g overflowing to infinity
-// gives silu = -0, not NaN).  At large N this runs on the tile kernel's
-// critical path, where the accurate forms cost 8 % more (LLaMA-7B gate/up,
-// N = 4096: 707 against 654 us).
+// gives silu = -0, not NaN; the accurate forms cost the tile kernel 8 % more
+// at LLaMA-7B gate/up, N = 4096).  The decode kernels call this per token;
+// the tile kernel pairs tokens with the same arithmetic in its epilogue.
 __device__ __forceinline__ void store_gate_up(const OutMap& o, int b, int r, int n, float v, bool valid) {
   const float u = __shfl_down_sync(0xffffffffu, v, 16);
   const int i = gate_up_channel(b, r);
   if (valid && (r & 16) == 0 && i < o.mi) {
     const float silu = __fdividef(v, 1.0f + __expf(-v));
     o.h[(size_t)n * o.mi + i] = __half_as_ushort(__float2half_rn(silu * u));
-  }
-}
-
-// The same for two consecutive tokens n and n + 1 (v0, v1: this lane's
-// accumulators of both; tokens >= N are not stored) with every lane busy:
-// a gate lane hands g(n + 1) to its up partner and takes u(n) in one
-// exchange, then writes H[n]; the up lane writes H[n + 1].  Per output the
-// arithmetic is store_gate_up's, so the bits are the same; a warp issues one
-// exchange and one SiLU sequence per two tokens instead of per token.
-__device__ __forceinline__ void store_gate_up_pair(const OutMap& o, int b, int r, int n, float v0, float v1,
-                                                   int N) {
-  const bool up = (r & 16) != 0;
-  const float recv = __shfl_xor_sync(0xffffffffu, up ? v0 : v1, 16);
-  const float g = up ? recv : v0;
-  const float u = up ? v1 : recv;
-  const int nn = up ? n + 1 : n;
-  const int i = gate_up_channel(b, r & ~16);
-  if (nn < N && i < o.mi) {
-    const float silu = __fdividef(g, 1.0f + __expf(-g));
-    o.h[(size_t)nn * o.mi + i] = __half_as_ushort(__float2half_rn(silu * u));
   }
 }
 
