@@ -10,18 +10,23 @@ from HBM into registers, warp-level MMAs on the exact dequant, the first
 weight groups requested before the grid dependency wait under programmatic
 dependent launch), the step captured once in a CUDA graph.  The metric is algorithmic HBM bytes per second (packed int4 weights +
 2.5 B per group of metadata + fp16 X and Y), reported against the measured HBM
-copy bandwidth.  The same JSON line carries, each with its own clock summary
-and median / p10 / p90 over its repeats: every projection alone, the two
-prefill GEMMs (TFLOP/s), the fused-QKV N sweep on every kernel, the
-LLaMA-3-8B batched-decode shapes, and the CPU oracle at all cores and at one
-thread.
+copy bandwidth.  `e2e` is the same step with every call's X copied in from
+pinned host memory and every Y copied back each step, pipelined per layer
+group on copy streams inside the step's graph (the serialised form beside
+it).  The same JSON line carries, each with its own clock summary and median
+/ p10 / p90 over its repeats: every projection alone, the fused-QKV N sweep
+on every kernel, the LLaMA-3-8B batched-decode shapes, the fused forms and
+secondary kernels, the two prefill GEMMs (TFLOP/s; last, since their power
+draw slows the memory-bound points timed after them), and the CPU oracle at
+all cores and at one thread.  Each secondary graph replays for 25 ms (250 ms
+before the LLaMA-3 leg) before it is timed.
 
 One JSON line on stdout (rank 0).  Multi-GPU runs (torchrun) are replicas:
 every rank runs its own copy of the step (weak scaling), no collective on the
 data path; time is the max over ranks.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-    python bench.py --workload qkv_n1|prefill|sweep|quantize|qkv_fused|gate_up_fused|add_rmsnorm ...
+    python bench.py --workload qkv_n1|prefill|sweep|quantize|qkv_fused|qkv_norm|gate_up_fused|add_rmsnorm ...
                                                           (secondary workloads)
 """
 from __future__ import annotations
