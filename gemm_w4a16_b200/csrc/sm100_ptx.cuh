@@ -1,5 +1,5 @@
 // Thin inline-PTX wrappers for the sm_100a features the tensor-core kernel
-// uses: mbarriers, TMA (tiled and bulk, never multicast), tcgen05 TMEM
+// uses: mbarriers, TMA (tiled and bulk, each copy into its own CTA only), tcgen05 TMEM
 // allocation, MMA, commit, and TMEM loads/stores.
 #pragma once
 
