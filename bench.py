@@ -56,7 +56,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # capture of this repository's kernel; it holds only while the kernel source
 # is the one captured (sha256 prefix of csrc/w4a16_gemv.cu), and the bench
 # reports null otherwise.
-DECODE_TRAFFIC = {"src_sha256_prefix": "ad06eac62b9462f1", "qkv_dram_bytes": 26184704, "qkv_alg_bytes": 26181632}
+DECODE_TRAFFIC = {"src_sha256_prefix": "a308e7b7e1ad5ecb", "qkv_dram_bytes": 26184704, "qkv_alg_bytes": 26181632}
 NOMINAL_DENSE_FP16_TFLOPS = 2250.0   # B200 dense fp16/bf16 tensor rate, NVIDIA's figure
 
 

@@ -46,12 +46,13 @@ namespace {
 
 constexpr int kGvWarps = 8;                           // one 16-row MMA tile each
 constexpr int kGvThreads = kGvWarps * 32;
-// Groups of codes in flight per warp, in registers: 4 for one token (80
-// registers still hold them without spills; the decode step ran 1.255 ->
-// 1.224 ms), 3 with more tokens (4 was slower at N = 8) or the normalising
-// prologue (which would spill).
+// Groups of codes in flight per warp, in registers: 4 for one or two tokens
+// (80 registers still hold them without spills; the decode step ran 1.255
+// -> 1.224 ms, QKV at N = 2 9.7 -> 9.1 us with the 4-way row split), 3 with
+// more tokens (4 was no faster at N = 4 and slower at N = 8) or the
+// normalising prologue (which would spill).
 template <int NT, bool kNorm>
-__host__ __device__ constexpr int gv_depth() { return NT == 1 && !kNorm ? 4 : NT > 8 ? 2 : 3; }
+__host__ __device__ constexpr int gv_depth() { return NT <= 2 && !kNorm ? 4 : NT > 8 ? 2 : 3; }
 constexpr int kGvCtasPerSm = 3;                       // resident CTAs per SM (register budget)
 constexpr int kGvWBytes = 4 * kRowBlock * 16;         // one group of 128 rows: 8 KB
 constexpr int kMaxCluster = 8;
@@ -653,8 +654,9 @@ template <int kEpi, bool kNorm = false>
 cudaError_t launch_epi(int nt, int kw, const uint8_t* wq, const uint16_t* s_p, const uint8_t* z_p,
                        const uint16_t* X, uint16_t* Y, int M, int K, int cl, bool pdl, cudaStream_t stream,
                        const OutMap& om, const NormIn& nin) {
-  if (kw == 4 && nt == 1)   // the chooser takes KW = 4 for one token only
-    return launch_nt<1, kEpi, 4, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin, 1);
+  if (kw == 4 && nt <= 2)   // the chooser takes KW = 4 for one or two tokens only
+    return nt == 1 ? launch_nt<1, kEpi, 4, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin, 1)
+                   : launch_nt<2, kEpi, 4, kNorm>(wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin, 2);
   if (kw == 2) return launch_kw<kEpi, 2, kNorm>(nt, wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
   return launch_kw<kEpi, 1, kNorm>(nt, wq, s_p, z_p, X, Y, M, K, cl, pdl, stream, om, nin);
 }
@@ -714,9 +716,9 @@ GvShape gemv_shape(int M, int K, int sms, int nt) {
     const long long ctas = (long long)blocks * kw * cl;
     return (long long)ceil_div((int)ctas, sms) * ceil_div(ceil_div(kg, cl), kw);
   };
-  // KW = 4 only for one token: at N = 8 it was slower on every LLaMA-7B shape
-  // (down 17.4 against 11.9 us).
-  for (int kw = 1; kw <= (nt == 1 ? 4 : 2); kw *= 2) {
+  // KW = 4 only for one or two tokens: at N = 4 it was no faster and at
+  // N = 8 slower on every LLaMA-7B shape (down 17.4 against 11.9 us).
+  for (int kw = 1; kw <= (nt <= 2 ? 4 : 2); kw *= 2) {
     for (int cl = 1; cl <= kMaxCluster && cl <= kg; ++cl) {
       if (!fits(kw, cl)) continue;
       const long long ctas = (long long)blocks * kw * cl;
