@@ -46,6 +46,22 @@ def test_debug_library_exports_the_same_symbols(L):
         assert hasattr(D, n), n
 
 
+def test_library_switch_restores_the_main_library(L):
+    """w4a16.library(DEBUG_LIB_PATH) routes the binding through the
+    index-check build inside the block (same host-side answers) and back to
+    libw4a16.so after it."""
+    main_path = w4a16.LIB_PATH
+    sizes = w4a16.packed_sizes(12288, 4096)
+    path = w4a16.select_path(12288, 4096, 16)
+    with w4a16.library(w4a16.DEBUG_LIB_PATH):
+        assert w4a16.lib()._name == w4a16.DEBUG_LIB_PATH
+        assert w4a16.packed_sizes(12288, 4096) == sizes
+        assert w4a16.select_path(12288, 4096, 16) == path
+        assert w4a16.status_string(w4a16.ERR_BOUNDS)
+    assert w4a16.LIB_PATH == main_path
+    assert w4a16.lib()._name == main_path
+
+
 def test_status_strings(L):
     for code in range(7):
         assert w4a16.status_string(code)
